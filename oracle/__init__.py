@@ -1,0 +1,152 @@
+"""fp64 CPU oracle for mixture-of-depths attention (MoDA) -- TEST INFRASTRUCTURE.
+
+Only the test suite, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline leg
+may import this package.  The product path (``depth_aware_attention_b200``) never does:
+it shares no code with it, and the oracle shares none with the CUDA library.
+
+The arithmetic lives in ``moda_oracle.c`` (plain C, fp64, POSIX threads).  This module
+only compiles it with gcc, loads it with ctypes and marshals numpy arrays.  Each entry
+point follows the definition of the operator on the hyper.ai summary of arXiv
+2603.15619, section "Mixture-of-Depths Attention (MoDA)": one softmax, jointly
+normalised, over the query's causal sequence keys and its own token's depth keys.
+
+Parity status: forward, backward and the row-weight view are pinned by the
+``-m "not gpu"`` tests in ``tests/test_oracle_pins.py`` (library special cases, closed
+forms, invariants, finite differences and hand-derived golden cases).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moda_oracle.c")
+_LIB = os.path.join(_HERE, "libmoda_oracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle shared library in-tree with gcc; returns its path."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-Wall", "-shared", "-fPIC",
+                               "-o", tmp, _SRC, "-lm", "-lpthread"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        P, I, D = ctypes.c_void_p, ctypes.c_int, ctypes.c_double
+        lib.moda_oracle_forward.argtypes = [P] * 7 + [I] * 8 + [D, I, I]
+        lib.moda_oracle_backward.argtypes = [P] * 13 + [I] * 8 + [D, I, I]
+        lib.moda_oracle_row_weights.argtypes = [P] * 3 + [I] * 9 + [D, I, P, P]
+        for f in (lib.moda_oracle_forward, lib.moda_oracle_backward,
+                  lib.moda_oracle_row_weights):
+            f.restype = I
+        _lib = lib
+    return _lib
+
+
+def _f64(x):
+    """Contiguous float64 numpy copy of a numpy array or torch tensor (bf16 widens exactly)."""
+    if x is None:
+        return None
+    if hasattr(x, "detach"):
+        x = x.detach().to("cpu")
+        import torch
+        x = x.to(torch.float64).numpy()
+    return np.ascontiguousarray(x, dtype=np.float64)
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def default_threads() -> int:
+    return os.cpu_count() or 1
+
+
+def forward(q, k, v, kd, vd, scale, causal=True, t0=0, nthreads=None):
+    """Oracle forward over the query tokens [t0, t0+nt).
+
+    Shapes: q [B,Hq,nt,d]; k,v [B,Hkv,T,d]; kd,vd [B,Hkv,nt,L,d] (L may be 0).
+    Returns (out [B,Hq,nt,d], lse [B,Hq,nt]) as float64 numpy arrays.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Hq, nt, d = q.shape
+    Hkv, T = k.shape[1], k.shape[2]
+    if kd is None or kd.shape[3] == 0:
+        L = 0
+        kd = vd = np.zeros((1,), np.float64)
+    else:
+        kd, vd = _f64(kd), _f64(vd)
+        L = kd.shape[3]
+    out = np.empty((B, Hq, nt, d), np.float64)
+    lse = np.empty((B, Hq, nt), np.float64)
+    rc = _load().moda_oracle_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(kd), _ptr(vd),
+                                     _ptr(out), _ptr(lse), B, Hq, Hkv, T, L, d, t0, nt,
+                                     float(scale), int(bool(causal)),
+                                     nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("moda_oracle_forward rejected the sizes")
+    return out, lse
+
+
+def backward(q, k, v, kd, vd, dout, scale, causal=True, t0=0, nthreads=None):
+    """Oracle backward over the rows of the query tokens [t0, t0+nt).
+
+    Returns dict(dq, dk, dv, dkd, dvd, out, lse) as float64 numpy arrays.  dq, dkd, dvd
+    are exact for the window; dk, dv hold the window rows' contributions (exact for keys
+    s >= t0 when causal and the window ends at T; exact everywhere for the full window).
+    """
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, Hq, nt, d = q.shape
+    Hkv, T = k.shape[1], k.shape[2]
+    if kd is None or kd.shape[3] == 0:
+        L = 0
+        kd = vd = np.zeros((1,), np.float64)
+    else:
+        kd, vd = _f64(kd), _f64(vd)
+        L = kd.shape[3]
+    dq = np.empty((B, Hq, nt, d), np.float64)
+    dk = np.empty((B, Hkv, T, d), np.float64)
+    dv = np.empty((B, Hkv, T, d), np.float64)
+    dkd = np.empty((B, Hkv, nt, L, d), np.float64)
+    dvd = np.empty((B, Hkv, nt, L, d), np.float64)
+    out = np.empty((B, Hq, nt, d), np.float64)
+    lse = np.empty((B, Hq, nt), np.float64)
+    rc = _load().moda_oracle_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(kd), _ptr(vd),
+                                      _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dkd),
+                                      _ptr(dvd), _ptr(out), _ptr(lse), B, Hq, Hkv, T, L, d,
+                                      t0, nt, float(scale), int(bool(causal)),
+                                      nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("moda_oracle_backward rejected the sizes")
+    return dict(dq=dq, dk=dk, dv=dv, dkd=dkd, dvd=dvd, out=out, lse=lse)
+
+
+def row_weights(q, k, kd, b, h, t, scale, causal=True):
+    """Normalised joint-softmax weights of row (b,h,t): (w_seq [n_visible], w_depth [L])."""
+    q, k = _f64(q), _f64(k)
+    B, Hq, T, d = q.shape
+    Hkv = k.shape[1]
+    if kd is None or kd.shape[3] == 0:
+        L, kd = 0, np.zeros((1,), np.float64)
+    else:
+        kd = _f64(kd)
+        L = kd.shape[3]
+    n = t + 1 if causal else T
+    ws = np.empty((n,), np.float64)
+    wd = np.empty((max(L, 1),), np.float64)
+    rc = _load().moda_oracle_row_weights(_ptr(q), _ptr(k), _ptr(kd), b, h, t, B, Hq, Hkv,
+                                         T, L, d, float(scale), int(bool(causal)),
+                                         _ptr(ws), _ptr(wd))
+    if rc != 0:
+        raise ValueError("moda_oracle_row_weights rejected the arguments")
+    return ws, wd[:L]
