@@ -1,0 +1,166 @@
+"""Python binding of the B200 MoDA library (``libmoda_b200.so``, C ABI in include/moda.h).
+
+Argument marshalling only: every step of the operator runs in the library's sm_100a
+kernels.  PyTorch supplies device memory and the current CUDA stream.  There is no CPU
+or PyTorch fallback: if the compiled library is missing, importing the binding raises.
+
+Low-level names mirror the C ABI (``moda_forward``, ``moda_backward``,
+``moda_backward_workspace_size``, ``moda_check_device_errors``, ``moda_status_string``);
+``forward`` / ``backward`` allocate outputs with torch and call them.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoda_b200.so")
+
+MODA_OK = 0
+MODA_ERR_INVALID_ARGUMENT = 1
+MODA_ERR_UNSUPPORTED = 2
+MODA_ERR_CUDA = 3
+MODA_ERR_TIMEOUT = 4
+MODA_ERR_INTERNAL = 5
+
+# Every symbol include/moda.h declares (checked by the ABI tests).
+EXPORTED = ("moda_forward", "moda_backward", "moda_backward_workspace_size",
+            "moda_check_device_errors", "moda_status_string", "moda_last_error_message")
+
+
+class ModaError(RuntimeError):
+    def __init__(self, status: int, where: str, message: str):
+        self.status = status
+        super().__init__(f"{where}: status {status} ({message})")
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python depth_aware_attention_b200/build.py`"
+            " (or __graft_entry__.build()); there is no fallback implementation")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, F, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.moda_forward.argtypes = [P] * 7 + [I] * 6 + [F, I, P]
+    lib.moda_forward.restype = I
+    lib.moda_backward_workspace_size.argtypes = [I] * 6
+    lib.moda_backward_workspace_size.restype = S
+    lib.moda_backward.argtypes = [P] * 14 + [S] + [I] * 6 + [F, I, P]
+    lib.moda_backward.restype = I
+    lib.moda_check_device_errors.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
+    lib.moda_check_device_errors.restype = I
+    lib.moda_status_string.argtypes = [I]
+    lib.moda_status_string.restype = ctypes.c_char_p
+    lib.moda_last_error_message.argtypes = []
+    lib.moda_last_error_message.restype = ctypes.c_char_p
+    return lib
+
+
+lib = _load()
+
+
+def _msg(status):
+    detail = lib.moda_last_error_message().decode()
+    base = lib.moda_status_string(status).decode()
+    return f"{base}: {detail}" if detail else base
+
+
+def _check(status, where):
+    if status != MODA_OK:
+        raise ModaError(status, where, _msg(status))
+
+
+# ---------------------------------------------------------------- C-ABI mirrors
+def moda_forward(q, k, v, kd, vd, out, lse, B, Hq, Hkv, T, L, d, scale, causal, stream):
+    """Direct call of the C entry point with raw pointers (ints) and a stream handle."""
+    return lib.moda_forward(q, k, v, kd, vd, out, lse, B, Hq, Hkv, T, L, d, float(scale),
+                            int(causal), stream)
+
+
+def moda_backward(q, k, v, kd, vd, out, lse, dout, dq, dk, dv, dkd, dvd, workspace,
+                  workspace_bytes, B, Hq, Hkv, T, L, d, scale, causal, stream):
+    return lib.moda_backward(q, k, v, kd, vd, out, lse, dout, dq, dk, dv, dkd, dvd,
+                             workspace, workspace_bytes, B, Hq, Hkv, T, L, d, float(scale),
+                             int(causal), stream)
+
+
+def moda_backward_workspace_size(B, Hq, Hkv, T, L, d):
+    return int(lib.moda_backward_workspace_size(B, Hq, Hkv, T, L, d))
+
+
+def moda_check_device_errors(stream=None):
+    """Synchronise `stream`; returns (status, flags) and clears the device error word."""
+    flags = ctypes.c_uint32(0)
+    st = lib.moda_check_device_errors(stream, ctypes.byref(flags))
+    return st, int(flags.value)
+
+
+def moda_status_string(status):
+    return lib.moda_status_string(status).decode()
+
+
+# ---------------------------------------------------------------- torch conveniences
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(device):
+    import torch
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _dims(q, k, kd):
+    B, Hq, T, d = q.shape
+    Hkv = k.shape[1]
+    L = 0 if kd is None else kd.shape[3]
+    return B, Hq, Hkv, T, L, d
+
+
+def forward(q, k, v, kd=None, vd=None, scale=None, causal=True, out=None, lse=None):
+    """MoDA forward on the current CUDA stream.  Returns (out bf16, lse fp32).
+
+    q [B,Hq,T,d], k/v [B,Hkv,T,d], kd/vd [B,Hkv,T,L,d] (or None for L = 0): contiguous
+    bf16 CUDA tensors.  scale defaults to 1/sqrt(d).
+    """
+    import torch
+    B, Hq, Hkv, T, L, d = _dims(q, k, kd)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, T), device=q.device, dtype=torch.float32)
+    st = lib.moda_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(kd) if L else None,
+                          _ptr(vd) if L else None, _ptr(out), _ptr(lse), B, Hq, Hkv, T, L,
+                          d, float(scale), int(bool(causal)), _stream_handle(q.device))
+    _check(st, "moda_forward")
+    return out, lse
+
+
+def backward(q, k, v, kd, vd, out, lse, dout, scale=None, causal=True, workspace=None):
+    """MoDA backward on the current CUDA stream.  Returns dict(dq, dk, dv, dkd, dvd)."""
+    import torch
+    B, Hq, Hkv, T, L, d = _dims(q, k, kd)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    ws = moda_backward_workspace_size(B, Hq, Hkv, T, L, d)
+    if workspace is None:
+        workspace = torch.empty(ws, device=q.device, dtype=torch.uint8)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dkd = torch.empty_like(kd) if L else None
+    dvd = torch.empty_like(vd) if L else None
+    st = lib.moda_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(kd) if L else None,
+                           _ptr(vd) if L else None, _ptr(out), _ptr(lse), _ptr(dout),
+                           _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dkd), _ptr(dvd), _ptr(workspace),
+                           workspace.numel() * workspace.element_size(), B, Hq, Hkv, T, L, d,
+                           float(scale), int(bool(causal)), _stream_handle(q.device))
+    _check(st, "moda_backward")
+    return dict(dq=dq, dk=dk, dv=dv, dkd=dkd, dvd=dvd)
+
+
+def check_device_errors(device=None):
+    """Raise ModaError if a kernel on the current stream recorded a failure."""
+    import torch
+    st, flags = moda_check_device_errors(_stream_handle(device or torch.cuda.current_device()))
+    _check(st, f"device error word 0x{flags:x}")

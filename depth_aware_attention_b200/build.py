@@ -1,0 +1,56 @@
+"""Build the MoDA CUDA library in-tree: depth_aware_attention_b200/libmoda_b200.so.
+
+nvcc compiles one translation unit for sm_100a only (B200), with the CUDA runtime linked
+statically and the driver's tensor-map encoder looked up at run time, so the library
+loads on a machine without a GPU or driver (its entry points then report MODA_ERR_CUDA).
+"""
+from __future__ import annotations
+
+import os
+import shutil
+import subprocess
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+CSRC = os.path.join(HERE, "csrc")
+LIB = os.path.join(HERE, "libmoda_b200.so")
+SOURCES = ["moda_lib.cu", "moda_api.cu", "moda_fwd.cu", "moda_bwd.cu", "sm100.cuh",
+           "moda_internal.h"]
+ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+
+
+def nvcc_path() -> str:
+    p = shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc"
+    if not os.path.exists(p):
+        raise RuntimeError("nvcc not found")
+    return p
+
+
+def needs_build() -> bool:
+    if not os.path.exists(LIB):
+        return True
+    t = os.path.getmtime(LIB)
+    deps = [os.path.join(CSRC, s) for s in SOURCES] + [os.path.join(ROOT, "include", "moda.h")]
+    return any(os.path.getmtime(d) > t for d in deps if os.path.exists(d))
+
+
+def build(force: bool = False, verbose: bool = False, extra=()) -> str:
+    if not force and not needs_build():
+        return LIB
+    tmp = LIB + f".tmp{os.getpid()}"
+    cmd = [nvcc_path(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "--use_fast_math",
+           "-Xcompiler", "-fPIC,-O2", "-shared", "-cudart", "static",
+           "-I", os.path.join(ROOT, "include"), "-o", tmp,
+           os.path.join(CSRC, "moda_lib.cu"), *extra]
+    if verbose:
+        print(" ".join(cmd), file=sys.stderr)
+    subprocess.check_call(cmd)
+    os.replace(tmp, LIB)
+    return LIB
+
+
+if __name__ == "__main__":
+    build(force="--force" in sys.argv, verbose=True,
+          extra=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else [])
+    print(LIB)

@@ -1,0 +1,56 @@
+// moda_internal.h -- shared declarations between the host entry points (moda_api.cu)
+// and the kernel launchers.  Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moda {
+
+// Geometry of one forward/backward problem after validation.
+struct Problem {
+  int B, Hq, Hkv, T, L, d, G;
+  int causal;
+  float scale;
+};
+
+// Tile geometry shared by the kernels: a query tile holds 128 (token, head) rows, TQ
+// tokens x G heads of one KV group, token-major (row r = token*G + head); depth chunks
+// hold JC depth entries of the tile's TQ tokens.
+struct TileGeom {
+  int TQ;   // tokens per query tile = 128 / G (floor)
+  int JC;   // depth entries per depth chunk = min(8, 128 / TQ)
+  int nqt;  // query tiles per (b, kv head) = ceil(T / TQ)
+};
+
+inline TileGeom tile_geom(const Problem& p) {
+  TileGeom t;
+  t.TQ = 128 / p.G;
+  t.JC = 128 / t.TQ;
+  if (t.JC > 8) t.JC = 8;
+  t.nqt = (p.T + t.TQ - 1) / t.TQ;
+  return t;
+}
+
+// Tensor-map encoder obtained from the driver at run time (no link-time libcuda).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+// Forward launcher: returns a CUDA error code (cudaSuccess when enqueued).
+cudaError_t launch_forward(const Problem& p, const void* q, const void* k, const void* v,
+                           const void* kd, const void* vd, void* out, float* lse,
+                           EncodeTiledFn encode, cudaStream_t stream, const char** why);
+
+cudaError_t launch_backward(const Problem& p, const void* q, const void* k, const void* v,
+                            const void* kd, const void* vd, const void* out,
+                            const float* lse, const void* dout, void* dq, void* dk,
+                            void* dv, void* dkd, void* dvd, void* workspace,
+                            EncodeTiledFn encode, cudaStream_t stream, const char** why);
+
+size_t backward_workspace_bytes(const Problem& p);
+
+}  // namespace moda

@@ -1,0 +1,112 @@
+/*
+ * moda.h -- C ABI of the B200 (sm_100a) mixture-of-depths attention (MoDA) library.
+ *
+ * The operator (hyper.ai summary of arXiv 2603.15619, section "Mixture-of-Depths
+ * Attention (MoDA)"): every query head attends in ONE softmax, with all scores
+ * normalised together, to
+ *   (a) the sequence keys/values of its GQA group at the current layer, causally, and
+ *   (b) the L depth keys/values that preceding attention and FFN sublayers wrote for the
+ *       query's own token position.
+ * For row (b, h, t) with g = h / (Hq / Hkv):
+ *   out[b,h,t] = softmax over { scale*<q,k[b,g,s]> : s <= t } U { scale*<q,kd[b,g,t,j]> : j < L }
+ *                applied to the matching values v[b,g,s] / vd[b,g,t,j]
+ *   lse[b,h,t] = natural log of the softmax normaliser (sum of exp of the scaled logits).
+ * The same page's section "Hardware-efficient implementation" describes the depth cache
+ * flattened along one axis of length T*L so that each query reads one contiguous
+ * range, and a chunk/group-aware tiling; the [B,Hkv,T,L,d] layout below is that
+ * flattening per (batch, KV head).
+ *
+ * Tensors (all row-major and contiguous, all pointers DEVICE pointers, 16-byte aligned):
+ *   q, out, dout, dq : bf16 [B][Hq][T][d]
+ *   k, v, dk, dv     : bf16 [B][Hkv][T][d]
+ *   kd, vd, dkd, dvd : bf16 [B][Hkv][T][L][d]     (may be NULL when L == 0)
+ *   lse              : fp32 [B][Hq][T]
+ * Sizes: B, T >= 1; Hq, Hkv >= 1 with Hq % Hkv == 0 and Hq / Hkv <= 64; L >= 0;
+ * d in {64, 128}.  scale is applied to every logit (typically 1/sqrt(d)).
+ * causal != 0: sequence key s is visible to token t iff s <= t; causal == 0: every
+ * sequence key is visible.  Depth keys are always the query's own token's only.
+ *
+ * Ownership: the caller allocates and owns every buffer (including the backward
+ * workspace).  Calls are asynchronous and stream-ordered on `stream`; the library keeps
+ * no per-call state and never allocates caller-visible memory.  Thread-safe.
+ *
+ * Errors: argument checks run before any launch and nothing is launched on failure.
+ * No entry point aborts or throws.  Kernels that detect an internal failure (a bounded
+ * wait that ran out, an index check) record it in a per-device error word that
+ * moda_check_device_errors() reads and clears.
+ */
+#ifndef MODA_H_
+#define MODA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MODA_OK = 0,
+    MODA_ERR_INVALID_ARGUMENT = 1, /* null/misaligned pointer, bad size, aliasing output */
+    MODA_ERR_UNSUPPORTED = 2,      /* d not in {64,128}, group too large, not sm_100 */
+    MODA_ERR_CUDA = 3,             /* a CUDA runtime/driver call failed */
+    MODA_ERR_TIMEOUT = 4,          /* a kernel's bounded wait ran out */
+    MODA_ERR_INTERNAL = 5          /* a kernel's internal consistency check failed */
+} moda_status_t;
+
+/* Opaque stream handle: a cudaStream_t (CUstream); NULL is the legacy default stream. */
+typedef void *moda_stream_t;
+
+/*
+ * Forward pass.  Writes out (bf16) and lse (fp32, natural log).  Definition: see the
+ * header comment (one joint softmax over causal sequence keys and own-token depth keys).
+ * kd/vd may be NULL iff L == 0, in which case this is plain causal GQA attention.
+ * Returns MODA_OK once the kernel is enqueued on `stream`.
+ */
+moda_status_t moda_forward(const void *q, const void *k, const void *v, const void *kd,
+                           const void *vd, void *out, float *lse, int B, int Hq, int Hkv,
+                           int T, int L, int d, float scale, int causal,
+                           moda_stream_t stream);
+
+/*
+ * Bytes of device workspace moda_backward needs for these sizes (fp32 dQ accumulator
+ * [B][Hq][T][d] plus the fp32 row terms D = <dO, out> [B][Hq][T]).
+ */
+size_t moda_backward_workspace_size(int B, int Hq, int Hkv, int T, int L, int d);
+
+/*
+ * Backward pass: gradients of sum(out * dout) w.r.t. q, k, v, kd, vd.  Recomputes the
+ * softmax weights P = exp(scale*logit - lse) from the forward's lse, with
+ * D = <dout, out> per row and dS = P * (<dout, value> - D):
+ *   dq = scale * sum dS * key,  dk/dkd = scale * sum dS * q,  dv/dvd = sum P * dout.
+ * The pages give no backward design; this is the exact gradient of the definition.
+ * `out` and `lse` must be the forward's outputs for the same inputs.  `workspace`
+ * (device, >= moda_backward_workspace_size bytes, 256-byte aligned) is scratch owned
+ * by the caller; its contents on entry do not matter.
+ */
+moda_status_t moda_backward(const void *q, const void *k, const void *v, const void *kd,
+                            const void *vd, const void *out, const float *lse,
+                            const void *dout, void *dq, void *dk, void *dv, void *dkd,
+                            void *dvd, void *workspace, size_t workspace_bytes, int B,
+                            int Hq, int Hkv, int T, int L, int d, float scale, int causal,
+                            moda_stream_t stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the calling device's kernel error word.
+ * *flags (may be NULL) receives the raw bits: 1 = a bounded wait ran out, 2 = an
+ * internal index/consistency check failed.  Returns MODA_ERR_TIMEOUT / MODA_ERR_INTERNAL
+ * if the corresponding bit was set, MODA_ERR_CUDA if synchronisation failed, else MODA_OK.
+ */
+moda_status_t moda_check_device_errors(moda_stream_t stream, uint32_t *flags);
+
+/* Static English description of a status code.  Never NULL. */
+const char *moda_status_string(moda_status_t status);
+
+/* Description of the last failure on the calling host thread (or ""). Never NULL. */
+const char *moda_last_error_message(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MODA_H_ */

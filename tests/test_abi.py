@@ -1,0 +1,105 @@
+"""The C-ABI library loads, exports every entry point include/moda.h declares, and
+rejects bad arguments before touching the GPU (CPU only: no compute calls)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import depth_aware_attention_b200 as moda
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moda.h")
+
+A = 1 << 20  # a fake, 16-byte aligned "device pointer" that is never dereferenced
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(moda_[a-z_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_functions()
+    assert set(names) == set(moda.EXPORTED)
+    lib = ctypes.CDLL(moda.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_library_is_sm100a_only_and_self_contained():
+    # no link-time dependency on the CUDA driver or a shared CUDA runtime
+    deps = os.popen(f"ldd {moda.LIB_PATH}").read()
+    assert "libcuda.so" not in deps
+    assert "libcudart" not in deps
+
+
+def test_status_strings():
+    for s in range(6):
+        assert moda.moda_status_string(s)
+    assert moda.moda_status_string(99) == "unknown status"
+
+
+def fwd(**kw):
+    args = dict(q=A, k=A * 2, v=A * 3, kd=A * 4, vd=A * 5, out=A * 64, lse=A * 128, B=1,
+                Hq=4, Hkv=2, T=16, L=2, d=64, scale=0.125, causal=1, stream=None)
+    args.update(kw)
+    return moda.moda_forward(**args)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(B=0), moda.MODA_ERR_INVALID_ARGUMENT),
+    (dict(T=0), moda.MODA_ERR_INVALID_ARGUMENT),
+    (dict(L=-1), moda.MODA_ERR_INVALID_ARGUMENT),
+    (dict(Hq=3, Hkv=2), moda.MODA_ERR_INVALID_ARGUMENT),
+    (dict(d=96), moda.MODA_ERR_UNSUPPORTED),
+    (dict(Hq=256, Hkv=2), moda.MODA_ERR_UNSUPPORTED),
+    (dict(q=None), moda.MODA_ERR_INVALID_ARGUMENT),
+    (dict(kd=None), moda.MODA_ERR_INVALID_ARGUMENT),
+    (dict(q=A + 8), moda.MODA_ERR_INVALID_ARGUMENT),
+    (dict(lse=A * 3 + 4), moda.MODA_ERR_INVALID_ARGUMENT),
+    (dict(out=A * 2), moda.MODA_ERR_INVALID_ARGUMENT),  # out aliases k
+    (dict(scale=float("nan")), moda.MODA_ERR_INVALID_ARGUMENT),
+    (dict(scale=float("inf")), moda.MODA_ERR_INVALID_ARGUMENT),
+])
+def test_forward_rejects_bad_arguments_before_launch(kw, status):
+    assert fwd(**kw) == status
+
+
+def test_forward_L0_allows_null_depth():
+    # valid arguments: without a GPU the call gets as far as the device check
+    st = fwd(L=0, kd=None, vd=None)
+    if not _has_gpu():
+        assert st == moda.MODA_ERR_CUDA
+
+
+def _has_gpu():
+    import torch
+    return torch.cuda.is_available()
+
+
+def test_backward_workspace_size():
+    B, Hq, Hkv, T, L, d = 1, 16, 4, 16384, 48, 128
+    ws = moda.moda_backward_workspace_size(B, Hq, Hkv, T, L, d)
+    assert ws >= B * Hq * T * d * 4 + B * Hq * T * 4
+    assert moda.moda_backward_workspace_size(0, Hq, Hkv, T, L, d) == 0
+
+
+def test_backward_rejects_small_workspace_and_aliasing():
+    args = dict(q=A, k=A * 2, v=A * 3, kd=A * 4, vd=A * 5, out=A * 6, lse=A * 7, dout=A * 8,
+                dq=A * 9, dk=A * 10, dv=A * 11, dkd=A * 12, vd_=None)
+    args.pop("vd_")
+    base = dict(dvd=A * 13, workspace=A * 64, workspace_bytes=1 << 20, B=1, Hq=4, Hkv=2,
+                T=16, L=2, d=64, scale=0.125, causal=1, stream=None)
+    st = moda.moda_backward(**args, **dict(base, workspace_bytes=16))
+    assert st == moda.MODA_ERR_INVALID_ARGUMENT
+    st = moda.moda_backward(**dict(args, dq=A * 2), **base)  # dq aliases k
+    assert st == moda.MODA_ERR_INVALID_ARGUMENT
+    st = moda.moda_backward(**args, **dict(base, workspace=A * 64 + 16))  # not 256-aligned
+    assert st == moda.MODA_ERR_INVALID_ARGUMENT
+
+
+def test_binding_has_no_fallback():
+    src = open(os.path.join(ROOT, "depth_aware_attention_b200", "__init__.py")).read()
+    assert "oracle" not in src.lower().replace("no cpu", "")
