@@ -1,0 +1,459 @@
+"""Benchmark of the MoDA (mixture-of-depths attention) hot path on B200.
+
+One step is one pass of the whole operator over one batch of seeded synthetic input: the
+fused forward (moda_forward) followed by the recompute-based backward (moda_backward),
+through the library's C ABI.  The default workload is the long-context problem the
+headline metric is quoted on: B=1, T=65536, Hq=16, Hkv=4, d=128, L=32, bf16, inputs
+i.i.d. N(0,1).  The FLOP count is the algorithmic one, 4*B*Hq*d*(T^2/2 + T*L) for the
+forward and 2.5x that for the backward (five matmul-shaped products instead of two).
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl moda|reference]
+Under torchrun (N > 1) every rank runs an independent replica of the workload (the
+operator needs no exchange between GPUs), and the job value is the sum of the ranks'
+FLOPs over the slowest rank's time.
+
+``--impl reference`` times the fp64 CPU oracle (the only reference implementation that
+exists for this operator) on bounded samples of the same workload and reports it in the
+same metric.  The oracle is imported only by that arm and by the cpu_baseline leg.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "MoDA fwd(+bwd) TFLOP/s, % bf16 peak & HBM GB/s at T=64K; ratio to L=0 causal"
+UNIT = "TFLOP/s"
+BWD_FLOP_FACTOR = 2.5
+PROFILES = os.path.join(ROOT, "profiles")
+KERNEL_SOURCES = [os.path.join(ROOT, "depth_aware_attention_b200", "csrc", f)
+                  for f in ("moda_fwd.cu", "moda_bwd.cu", "sm100.cuh", "moda_internal.h")]
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["moda", "reference"], default="moda")
+    ap.add_argument("--workload", default="long-64k", choices=sorted(workloads.CONFIGS))
+    ap.add_argument("--fwd-only", action="store_true",
+                    help="time the forward alone (not the headline step)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU time of the oracle sample")
+    return ap.parse_args()
+
+
+def peaks():
+    """Measured denominators (generated file), else the machine's fallback figures."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return dict(bf16=float(p["bf16_tflops"]), bf16_sustained=float(p["bf16_tflops_sustained"]),
+                    hbm=float(p["hbm_gbs"]), source="measured")
+    except (OSError, KeyError, ValueError):
+        return dict(bf16=1590.0, bf16_sustained=1400.0, hbm=6650.0, source="fallback")
+
+
+def kernel_hash():
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        if os.path.exists(p):
+            with open(p, "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the current
+    kernel sources (profiles/traffic.json: {kernel: {workload: {bytes, source_hash}}})."""
+    try:
+        with open(os.path.join(PROFILES, "traffic.json")) as f:
+            rec = json.load(f)[kernel][workload]
+    except (OSError, KeyError, ValueError):
+        return None
+    return float(rec["bytes"]) if rec.get("source_hash") == kernel_hash() else None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.t.join(timeout=5)
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(n):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group(
+            "nccl", timeout=datetime.timedelta(seconds=300),
+            device_id=torch.device("cuda", local))
+    elif n > 1:
+        print(json.dumps({"warning": f"--gpus {n} without torchrun: running one replica"}),
+              file=sys.stderr)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def step_flops(cfg, fwd_only):
+    f = workloads.forward_flops(**cfg)
+    return f if fwd_only else f * (1.0 + BWD_FLOP_FACTOR)
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def run_moda(args, world, rank, local):
+    import depth_aware_attention_b200 as moda
+
+    cfg = workloads.CONFIGS[args.workload]
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    scale = workloads.default_scale(cfg["d"])
+    x = workloads.make_inputs(cfg, workloads.SEED_BASE[args.workload] + 7919 * rank, dev,
+                              with_dout=True)
+    q, k, v, kd, vd, dout = (x[n] for n in ("q", "k", "v", "kd", "vd", "dout"))
+    out = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], device=dev, dtype=torch.float32)
+    B, Hq, T, d = q.shape
+    Hkv, L = k.shape[1], cfg["L"]
+    ws_bytes = moda.moda_backward_workspace_size(B, Hq, Hkv, T, L, d)
+    ws = torch.empty(ws_bytes, device=dev, dtype=torch.uint8)
+    grads = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
+                 dkd=torch.empty_like(kd) if L else None,
+                 dvd=torch.empty_like(vd) if L else None)
+    stream = torch.cuda.current_stream(dev)
+    fwd_events = []
+
+    def step(record=False):
+        if record:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+        moda.forward(q, k, v, kd, vd, scale, True, out=out, lse=lse)
+        if record:
+            e1.record(stream)
+            fwd_events.append((e0, e1))
+        if not args.fwd_only:
+            moda.backward(q, k, v, kd, vd, out, lse, dout, scale, True, workspace=ws,
+                          grads=grads)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    moda.check_device_errors()
+
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        t_start.record(stream)
+        for _ in range(args.steps):
+            step(record=True)
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    moda.check_device_errors()
+    ms_local = t_start.elapsed_time(t_end) / args.steps
+    ms = max_over_ranks(ms_local, world)
+    flops = step_flops(cfg, args.fwd_only)
+    value = flops * world / (ms * 1e-3) / 1e12
+    fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in fwd_events)
+    launches_per_step = 1 if args.fwd_only else 1 + moda.BACKWARD_LAUNCHES
+
+    pk = peaks()
+    fwd_flops = workloads.forward_flops(**cfg)
+    fwd_tflops = fwd_flops / (fwd_ms * 1e-3) / 1e12
+    traffic = recorded_traffic("moda_fwd_kernel", args.workload)
+    roofline = {"kernel": "moda_fwd_kernel", "bound": "tensor", "achieved": round(fwd_tflops, 1),
+                "peak": pk["bf16_sustained"], "unit": "TFLOP/s",
+                "frac": round(fwd_tflops / pk["bf16_sustained"], 4), "traffic": traffic,
+                "peak_kind": f"{pk['source']} bf16 dense, sustained (kernel timed inside a "
+                             "long step)",
+                "algorithmic_flops_per_launch": fwd_flops,
+                "avg_launch_ms": round(fwd_ms, 4)}
+
+    # Extras the metric names: the L=0 causal ratio and the depth stream's HBM rate.
+    extras = {}
+    if args.workload.startswith("long-64k") and L > 0:
+        def t_fwd(kdx, vdx, n=3):
+            for _ in range(2):
+                moda.forward(q, k, v, kdx, vdx, scale, True, out=out, lse=lse)
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            for _ in range(n):
+                moda.forward(q, k, v, kdx, vdx, scale, True, out=out, lse=lse)
+            a1.record(stream)
+            torch.cuda.synchronize(dev)
+            return a0.elapsed_time(a1) / n
+        ms_l = t_fwd(kd, vd)
+        ms_0 = t_fwd(None, None)
+        cfg0 = dict(cfg, L=0)
+        tf_l = fwd_flops / (ms_l * 1e-3) / 1e12
+        tf_0 = workloads.forward_flops(**cfg0) / (ms_0 * 1e-3) / 1e12
+        dbytes = workloads.depth_bytes(**cfg)
+        extras["l0_ratio"] = {"fwd_ms_L": round(ms_l, 3), "fwd_ms_L0": round(ms_0, 3),
+                              "time_ratio_L0_over_L": round(ms_0 / ms_l, 4),
+                              "tflops_ratio_L_over_L0": round(tf_l / tf_0, 4)}
+        extra_ms = ms_l - ms_0
+        extras["depth_stream"] = {
+            "bytes": dbytes,
+            "gbs_from_time_difference": (round(dbytes / (extra_ms * 1e-3) / 1e9, 1)
+                                         if extra_ms > 0.02 * ms_l else "hidden"),
+            "hbm_peak_gbs": pk["hbm"]}
+        extras["fwd_pct_bf16_peak"] = {
+            "of_measured_burst": round(tf_l / pk["bf16"], 4),
+            "of_measured_sustained": round(tf_l / pk["bf16_sustained"], 4),
+            "of_spec_2250": round(tf_l / 2250.0, 4)}
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, moda, cfg, x, scale, dev, stream, world)
+
+    del x, q, k, v, kd, vd, dout, out, lse, ws, grads
+    torch.cuda.empty_cache()
+    return dict(ms=ms, value=value, clocks=clocks.summary(), roofline=roofline,
+                launches=launches_per_step * args.steps, extras=extras, e2e=e2e)
+
+
+def run_e2e(args, moda, cfg, x, scale, dev, stream, world):
+    """Same metric through the public API from pinned HOST buffers: every step copies its
+    inputs host->device, runs the operator and reads the results back to the host."""
+    names = ["q", "k", "v", "kd", "vd"] + ([] if args.fwd_only else ["dout"])
+    host = {n: torch.empty(x[n].shape, dtype=x[n].dtype, pin_memory=True)
+            for n in names if x[n] is not None}
+    for n, h in host.items():
+        h.copy_(x[n])
+    dbuf = {n: torch.empty_like(x[n]) for n in host}
+    h2d = sum(h.numel() * h.element_size() for h in host.values())
+    B, Hq, T, d = x["q"].shape
+    L = cfg["L"]
+    out_h = torch.empty(x["q"].shape, dtype=torch.bfloat16, pin_memory=True)
+    lse_h = torch.empty((B, Hq, T), dtype=torch.float32, pin_memory=True)
+    res_h = {}
+    if not args.fwd_only:
+        for n in ["q", "k", "v"] + (["kd", "vd"] if L else []):
+            res_h["d" + n] = torch.empty(x[n].shape, dtype=torch.bfloat16, pin_memory=True)
+    d2h = out_h.numel() * 2 + lse_h.numel() * 4 + sum(r.numel() * 2 for r in res_h.values())
+
+    def step():
+        for n, h in host.items():
+            dbuf[n].copy_(h, non_blocking=True)
+        out, lse = moda.forward(dbuf["q"], dbuf["k"], dbuf["v"], dbuf.get("kd"), dbuf.get("vd"),
+                                scale, True)
+        out_h.copy_(out, non_blocking=True)
+        lse_h.copy_(lse, non_blocking=True)
+        if not args.fwd_only:
+            g = moda.backward(dbuf["q"], dbuf["k"], dbuf["v"], dbuf.get("kd"), dbuf.get("vd"),
+                              out, lse, dbuf["dout"], scale, True)
+            for n, r in res_h.items():
+                r.copy_(g[n], non_blocking=True)
+
+    steps = max(1, min(args.steps, 3))
+    step()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, world)
+    value = step_flops(cfg, args.fwd_only) * world / (ms * 1e-3) / 1e12
+    del host, dbuf, out_h, lse_h, res_h
+    return {"value": round(value, 2), "unit": UNIT, "ms_per_step": round(ms, 3),
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def oracle_sample(cfg, seed_base, cpu_seconds, fwd_only):
+    """Times the fp64 CPU oracle on a bounded sample of the workload.
+
+    The sample is a window of the LAST nt query tokens (the most expensive rows of the
+    causal problem) with all heads; its algorithmic FLOPs are summed row by row with the
+    same per-row count as the full problem (4*d*(|visible keys| + L) forward, x2.5 for the
+    backward).  nt grows until the sample takes about cpu_seconds.
+    """
+    import oracle
+    g = torch.Generator().manual_seed(seed_base)
+    B, Hq, Hkv, T, L, d = (cfg[n] for n in ("B", "Hq", "Hkv", "T", "L", "d"))
+    scale = workloads.default_scale(d)
+    k = torch.randn((B, Hkv, T, d), generator=g).to(torch.bfloat16)
+    v = torch.randn((B, Hkv, T, d), generator=g).to(torch.bfloat16)
+    threads = oracle.default_threads()
+
+    def sample(nt):
+        t0 = T - nt
+        q = torch.randn((B, Hq, nt, d), generator=g).to(torch.bfloat16)
+        kd = vd = None
+        if L:
+            kd = torch.randn((B, Hkv, nt, L, d), generator=g).to(torch.bfloat16)
+            vd = torch.randn((B, Hkv, nt, L, d), generator=g).to(torch.bfloat16)
+        rows_keys = sum((t + 1) + L for t in range(t0, T)) * B * Hq
+        fl = 4.0 * d * rows_keys
+        start = time.perf_counter()
+        if fwd_only:
+            oracle.forward(q, k, v, kd, vd, scale, True, t0=t0, nthreads=threads)
+        else:
+            dout = torch.randn((B, Hq, nt, d), generator=g).to(torch.bfloat16)
+            oracle.backward(q, k, v, kd, vd, dout, scale, True, t0=t0, nthreads=threads)
+            fl *= 1.0 + BWD_FLOP_FACTOR
+        return fl, time.perf_counter() - start
+
+    nt = 1
+    fl, sec = sample(nt)
+    while sec < cpu_seconds / 8 and nt < T:
+        nt = min(T, nt * 4)
+        fl, sec = sample(nt)
+    if sec < cpu_seconds / 2 and nt < T:
+        nt = min(T, max(nt + 1, int(nt * cpu_seconds / max(sec, 1e-3))))
+        fl, sec = sample(nt)
+    what = "forward" if fwd_only else "forward+backward"
+    return {"value": round(fl / sec / 1e12, 6), "unit": UNIT, "cores": threads, "kind": "oracle",
+            "seconds": round(sec, 2),
+            "sample": f"fp64 oracle {what} on the last {nt} query tokens (all {B * Hq} "
+                      f"heads) of the {cfg['T']}-token workload, L={L}; FLOPs counted "
+                      f"row by row as 4*d*(visible keys + L)"
+                      + ("" if fwd_only else " x (1 + 2.5)")}
+
+
+def run_reference(args, world, rank):
+    """The reference arm: the CPU oracle, timed on bounded samples, in the same metric."""
+    cfg = workloads.CONFIGS[args.workload]
+    if rank != 0:
+        return None
+    per_step = max(1.0, args.cpu_seconds / max(1, args.steps))
+    oracle_sample(cfg, 1, 0.5, args.fwd_only)  # warm-up: builds and loads the library
+    vals = []
+    last = None
+    for _ in range(args.steps):
+        last = oracle_sample(cfg, 1, per_step, args.fwd_only)
+        vals.append(last["value"])
+    value = statistics.mean(vals)
+    flops = step_flops(cfg, args.fwd_only)
+    return dict(value=value, ms=flops / (value * 1e12) * 1e3, cpu=dict(last, value=value))
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup(args.gpus)
+    cfg = workloads.CONFIGS[args.workload]
+    config = {"workload": args.workload, **{k: cfg[k] for k in ("B", "T", "Hq", "Hkv", "d", "L")},
+              "causal": True, "scale": "1/sqrt(d)",
+              "step": "forward" if args.fwd_only else "forward+backward",
+              "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas x{world}"}
+    base = {"metric": METRIC, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "data": "synthetic, seeded N(0,1) bf16", "config": config}
+
+    if args.impl == "reference":
+        r = run_reference(args, world, rank)
+        if rank == 0:
+            line = dict(base, impl="reference", value=round(r["value"], 6),
+                        ms_per_step=round(r["ms"], 3), dtype="f64",
+                        cpu_baseline=r["cpu"],
+                        e2e={"value": round(r["value"], 6), "unit": UNIT,
+                             "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0})
+            print(json.dumps(line), flush=True)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+
+    r = run_moda(args, world, rank, local)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_sample(cfg, 1, args.cpu_seconds, args.fwd_only)
+    if rank == 0:
+        line = dict(base, value=round(r["value"], 2), ms_per_step=round(r["ms"], 3),
+                    dtype="bf16", clocks=r["clocks"], roofline=r["roofline"],
+                    cpu_baseline=cpu, e2e=r["e2e"], gpu_launches=r["launches"], **r["extras"])
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -24,6 +24,9 @@ MODA_ERR_CUDA = 3
 MODA_ERR_TIMEOUT = 4
 MODA_ERR_INTERNAL = 5
 
+# Kernel launches one moda_backward call makes (row terms + depth, sequence, dQ convert).
+BACKWARD_LAUNCHES = 3
+
 # Every symbol include/moda.h declares (checked by the ABI tests).
 EXPORTED = ("moda_forward", "moda_backward", "moda_backward_workspace_size",
             "moda_check_device_errors", "moda_status_string", "moda_last_error_message")
@@ -138,8 +141,14 @@ def forward(q, k, v, kd=None, vd=None, scale=None, causal=True, out=None, lse=No
     return out, lse
 
 
-def backward(q, k, v, kd, vd, out, lse, dout, scale=None, causal=True, workspace=None):
-    """MoDA backward on the current CUDA stream.  Returns dict(dq, dk, dv, dkd, dvd)."""
+def backward(q, k, v, kd, vd, out, lse, dout, scale=None, causal=True, workspace=None,
+             grads=None):
+    """MoDA backward on the current CUDA stream.  Returns dict(dq, dk, dv, dkd, dvd).
+
+    ``out``/``lse`` are the forward's results for the same inputs.  ``workspace`` (uint8
+    CUDA tensor of at least moda_backward_workspace_size bytes) and ``grads`` (a dict of
+    preallocated gradient tensors) are optional; missing ones are allocated with torch.
+    """
     import torch
     B, Hq, Hkv, T, L, d = _dims(q, k, kd)
     if scale is None:
@@ -147,16 +156,27 @@ def backward(q, k, v, kd, vd, out, lse, dout, scale=None, causal=True, workspace
     ws = moda_backward_workspace_size(B, Hq, Hkv, T, L, d)
     if workspace is None:
         workspace = torch.empty(ws, device=q.device, dtype=torch.uint8)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    dkd = torch.empty_like(kd) if L else None
-    dvd = torch.empty_like(vd) if L else None
+    g = dict(grads or {})
+    if g.get("dq") is None:
+        g["dq"] = torch.empty_like(q)
+    if g.get("dk") is None:
+        g["dk"] = torch.empty_like(k)
+    if g.get("dv") is None:
+        g["dv"] = torch.empty_like(v)
+    if L and g.get("dkd") is None:
+        g["dkd"] = torch.empty_like(kd)
+    if L and g.get("dvd") is None:
+        g["dvd"] = torch.empty_like(vd)
+    if not L:
+        g["dkd"] = g["dvd"] = None
     st = lib.moda_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(kd) if L else None,
                            _ptr(vd) if L else None, _ptr(out), _ptr(lse), _ptr(dout),
-                           _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dkd), _ptr(dvd), _ptr(workspace),
+                           _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dkd"]),
+                           _ptr(g["dvd"]), _ptr(workspace),
                            workspace.numel() * workspace.element_size(), B, Hq, Hkv, T, L, d,
                            float(scale), int(bool(causal)), _stream_handle(q.device))
     _check(st, "moda_backward")
-    return dict(dq=dq, dk=dk, dv=dv, dkd=dkd, dvd=dvd)
+    return g
 
 
 def check_device_errors(device=None):

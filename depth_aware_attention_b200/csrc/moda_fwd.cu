@@ -11,15 +11,17 @@
 // the group ("group-aware") and the tile touches only its own tokens' depth rows
 // (TQ x L of them -- "chunk-aware"), read once from HBM.
 //
-// Warp roles (192 threads):
+// Warp roles (224 threads):
 //   warps 0-3  softmax/depth/epilogue: thread r owns tile row r (TMEM lane r).
 //              1. depth fold: logits q.kd and the running sums over the tile's depth
 //                 chunks on CUDA cores, accumulator written into TMEM as O's start;
 //              2. per sequence block: S row from TMEM -> mask -> exp2 -> P (bf16) back
 //                 into TMEM over S; rescales O only when the row max grows by > 2^8;
 //              3. epilogue: O / l -> bf16 out, lse = ln(sum exp).
-//   warp 4     TMA producer: Q tile, then depth chunks (kd, vd), then K/V blocks, all
-//              through one ring of equally sized shared-memory stages.
+//   warp 4     TMA producer: Q tile, then the K/V blocks through the K/V ring.
+//   warp 6     TMA producer: the tile's depth chunks (kd, vd) through the depth ring.
+//              Each ring has exactly one consumer (tensor cores / softmax warps), which
+//              waits on every stage use in order, so the parity waits are unambiguous.
 //   warp 5     tcgen05 issuer: S = Q K^T (both operands in shared memory) and
 //              O += P V (P from tensor memory, V in shared memory), fp32 in TMEM.
 // TMEM columns: S/P double buffer at [0,128) and [128,256), O at [256, 256+D).
@@ -42,13 +44,15 @@ constexpr int kRegion = 16384;     // one 128-row x 128-byte swizzled region
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only past 256x
+constexpr int kFwdThreads = 224;           // 7 warps, roles below
 
 template <int D>
 struct FwdCfg {
   static constexpr int kRegions = D / 64;                 // 64-column swizzled regions
   static constexpr int kTileBytes = kRegions * kRegion;   // Q tile or one ring stage
-  static constexpr int kStages = (D == 128) ? 5 : 8;
-  static constexpr int kBarOff = kTileBytes * (1 + kStages);
+  static constexpr int kKV = (D == 128) ? 4 : 6;          // K/V ring stages
+  static constexpr int kDS = (D == 128) ? 2 : 4;          // depth ring stages
+  static constexpr int kBarOff = kTileBytes * (1 + kKV + kDS);
   static constexpr int kSmemBytes = 1024 + kBarOff + 256;
 };
 
@@ -62,8 +66,10 @@ struct FwdArgs {
 // Shared-memory barrier block (after the tiles).
 struct Bars {
   uint64_t q_full;
-  uint64_t full[8];
-  uint64_t empty[8];
+  uint64_t full[6];    // K/V ring: data landed
+  uint64_t empty[6];   // K/V ring: stage released by the tensor cores
+  uint64_t dfull[4];   // depth ring: data landed
+  uint64_t dempty[4];  // depth ring: stage released by the softmax warps
   uint64_t s_full[2];
   uint64_t p_full[2];
   uint64_t o_done;
@@ -85,19 +91,21 @@ __device__ __forceinline__ float dot8(const float (&a)[8], uint4 w) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kFwdThreads, 1)
     moda_fwd_kernel(const __grid_constant__ CUtensorMap tmQ,
                     const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV,
                     const __grid_constant__ CUtensorMap tmKD,
                     const __grid_constant__ CUtensorMap tmVD, const FwdArgs a) {
   using Cfg = FwdCfg<D>;
-  constexpr int NS = Cfg::kStages;
+  constexpr int NKV = Cfg::kKV;
+  constexpr int NDS = Cfg::kDS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sQ = smem_u32(smem);
-  const uint32_t sRing = sQ + Cfg::kTileBytes;
+  const uint32_t sRing = sQ + Cfg::kTileBytes;               // K/V ring
+  const uint32_t sDRing = sRing + NKV * Cfg::kTileBytes;      // depth ring
   Bars* bars = reinterpret_cast<Bars*>(smem + Cfg::kBarOff);
   volatile int* abort_flag = &bars->abort;
 
@@ -113,12 +121,17 @@ __global__ void __launch_bounds__(192, 1)
 
   auto bar = [&](uint64_t& b) { return smem_u32(&b); };
   auto stage_addr = [&](int s) { return sRing + uint32_t(s) * Cfg::kTileBytes; };
+  auto dstage_addr = [&](int s) { return sDRing + uint32_t(s) * Cfg::kTileBytes; };
 
   if (threadIdx.x == 0) {
     mbar_init(bar(bars->q_full), 1);
-    for (int s = 0; s < NS; ++s) {
+    for (int s = 0; s < NKV; ++s) {
       mbar_init(bar(bars->full[s]), 1);
       mbar_init(bar(bars->empty[s]), 1);
+    }
+    for (int s = 0; s < NDS; ++s) {
+      mbar_init(bar(bars->dfull[s]), 1);
+      mbar_init(bar(bars->dempty[s]), 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(bars->s_full[i]), 1);
@@ -148,49 +161,42 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t tmem = bars->tmem_base;
 
   if (warp == 4) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------------ TMA producer: Q tile, K/V blocks
     if (elect_one()) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      if (has_depth) {
-        tma_prefetch_desc(&tmKD);
-        tma_prefetch_desc(&tmVD);
-      }
       mbar_expect_tx(bar(bars->q_full), Cfg::kRegions * 128 * a.G * a.TQ);
       for (int rg = 0; rg < Cfg::kRegions; ++rg)
         tma_load_4d(sQ + rg * kRegion, &tmQ, bar(bars->q_full), rg * 64, 0, t0, bg);
-      int idx = 0;
-      auto acquire = [&]() -> int {
-        const int s = idx % NS;
-        if (idx >= NS) mbar_wait(bar(bars->empty[s]), ((idx / NS) - 1) & 1, abort_flag);
-        ++idx;
-        return s;
-      };
-      const uint32_t dbytes = Cfg::kRegions * 128 * a.TQ * a.JC;
-      for (int ci = 0; ci < NC; ++ci) {
-        int s = acquire();
-        mbar_expect_tx(bar(bars->full[s]), dbytes);
+      for (int idx = 0; idx < 2 * NB; ++idx) {
+        const int s = idx % NKV;
+        if (idx >= NKV) mbar_wait(bar(bars->empty[s]), ((idx / NKV) - 1) & 1, abort_flag);
+        const CUtensorMap* map = (idx & 1) ? &tmV : &tmK;
+        mbar_expect_tx(bar(bars->full[s]), Cfg::kTileBytes);
         for (int rg = 0; rg < Cfg::kRegions; ++rg)
-          tma_load_4d(stage_addr(s) + rg * kRegion, &tmKD, bar(bars->full[s]), rg * 64, t0,
-                      ci * a.JC, bg);
-        s = acquire();
-        mbar_expect_tx(bar(bars->full[s]), dbytes);
-        for (int rg = 0; rg < Cfg::kRegions; ++rg)
-          tma_load_4d(stage_addr(s) + rg * kRegion, &tmVD, bar(bars->full[s]), rg * 64, t0,
-                      ci * a.JC, bg);
+          tma_load_3d(stage_addr(s) + rg * kRegion, map, bar(bars->full[s]), rg * 64,
+                      (idx >> 1) * kBN, bg);
       }
-      for (int jb = 0; jb < NB; ++jb) {
-        int s = acquire();
-        mbar_expect_tx(bar(bars->full[s]), Cfg::kTileBytes);
+    }
+    __syncwarp();
+  } else if (warp == 6) {
+    // ------------------------------------------------ TMA producer: depth chunks
+    // Chunk ci holds entries [ci*JC, ci*JC+JC) of the tile's TQ tokens, rows
+    // (token, entry) with the entry fastest: each token's entries are one contiguous
+    // run of the [B,Hkv,T,L,d] cache.
+    if (has_depth && elect_one()) {
+      tma_prefetch_desc(&tmKD);
+      tma_prefetch_desc(&tmVD);
+      const uint32_t dbytes = Cfg::kRegions * 128 * a.TQ * a.JC;
+      for (int idx = 0; idx < 2 * NC; ++idx) {
+        const int s = idx % NDS;
+        if (idx >= NDS) mbar_wait(bar(bars->dempty[s]), ((idx / NDS) - 1) & 1, abort_flag);
+        const CUtensorMap* map = (idx & 1) ? &tmVD : &tmKD;
+        mbar_expect_tx(bar(bars->dfull[s]), dbytes);
         for (int rg = 0; rg < Cfg::kRegions; ++rg)
-          tma_load_3d(stage_addr(s) + rg * kRegion, &tmK, bar(bars->full[s]), rg * 64,
-                      jb * kBN, bg);
-        s = acquire();
-        mbar_expect_tx(bar(bars->full[s]), Cfg::kTileBytes);
-        for (int rg = 0; rg < Cfg::kRegions; ++rg)
-          tma_load_3d(stage_addr(s) + rg * kRegion, &tmV, bar(bars->full[s]), rg * 64,
-                      jb * kBN, bg);
+          tma_load_4d(dstage_addr(s) + rg * kRegion, map, bar(bars->dfull[s]), rg * 64,
+                      (idx >> 1) * a.JC, t0, bg);
       }
     }
     __syncwarp();
@@ -203,9 +209,9 @@ __global__ void __launch_bounds__(192, 1)
       mbar_wait(bar(bars->q_full), 0, abort_flag);
       auto issue_pv = [&](int j) {
         mbar_wait(bar(bars->p_full[j & 1]), (j >> 1) & 1, abort_flag);
-        const int vidx = 2 * NC + 2 * j + 1;
-        const int vs = vidx % NS;
-        mbar_wait(bar(bars->full[vs]), (vidx / NS) & 1, abort_flag);
+        const int vidx = 2 * j + 1;
+        const int vs = vidx % NKV;
+        mbar_wait(bar(bars->full[vs]), (vidx / NKV) & 1, abort_flag);
         tc_fence_after();
         const uint32_t vbase = stage_addr(vs);
 #pragma unroll
@@ -219,9 +225,9 @@ __global__ void __launch_bounds__(192, 1)
         if (j == NB - 1) tc_commit(bar(bars->o_final));
       };
       for (int jb = 0; jb < NB; ++jb) {
-        const int kidx = 2 * NC + 2 * jb;
-        const int ks_ = kidx % NS;
-        mbar_wait(bar(bars->full[ks_]), (kidx / NS) & 1, abort_flag);
+        const int kidx = 2 * jb;
+        const int ks_ = kidx % NKV;
+        mbar_wait(bar(bars->full[ks_]), (kidx / NKV) & 1, abort_flag);
         tc_fence_after();
         const uint32_t kbase = stage_addr(ks_);
 #pragma unroll
@@ -258,12 +264,12 @@ __global__ void __launch_bounds__(192, 1)
       const int tokc = tok < a.TQ ? tok : 0;  // padding rows read a valid row
       for (int ci = 0; ci < NC; ++ci) {
         const int kidx = 2 * ci, vidx = 2 * ci + 1;
-        const int kst = kidx % NS, vst = vidx % NS;
+        const int kst = kidx % NDS, vst = vidx % NDS;
         float y[kJCMax];
 #pragma unroll
         for (int jj = 0; jj < kJCMax; ++jj) y[jj] = 0.f;
-        mbar_wait(bar(bars->full[kst]), (kidx / NS) & 1, abort_flag);
-        const uint32_t kb = stage_addr(kst);
+        mbar_wait(bar(bars->dfull[kst]), (kidx / NDS) & 1, abort_flag);
+        const uint32_t kb = dstage_addr(kst);
 #pragma unroll 2
         for (int c8 = 0; c8 < D / 8; ++c8) {
           const uint32_t reg = (c8 >> 3) * kRegion;
@@ -273,13 +279,13 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int jj = 0; jj < kJCMax; ++jj) {
             if (jj < a.JC) {
-              const uint32_t row = jj * a.TQ + tokc;
+              const uint32_t row = tokc * a.JC + jj;
               y[jj] += dot8(qf, lds128(kb + reg + sw128_off(row, c8 & 7)));
             }
           }
         }
         named_bar_sync(1, 128);
-        if (r == 0) mbar_arrive(bar(bars->empty[kst]));
+        if (r == 0) mbar_arrive(bar(bars->dempty[kst]));
         // online update over this chunk's depth logits (log2 domain)
         float mx = -INFINITY;
 #pragma unroll
@@ -298,8 +304,8 @@ __global__ void __launch_bounds__(192, 1)
         }
         l = l * alpha + ps;
         m = m_new;
-        mbar_wait(bar(bars->full[vst]), (vidx / NS) & 1, abort_flag);
-        const uint32_t vb = stage_addr(vst);
+        mbar_wait(bar(bars->dfull[vst]), (vidx / NDS) & 1, abort_flag);
+        const uint32_t vb = dstage_addr(vst);
 #pragma unroll
         for (int c8 = 0; c8 < D / 8; ++c8) {
           const uint32_t reg = (c8 >> 3) * kRegion;
@@ -308,7 +314,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int jj = 0; jj < kJCMax; ++jj) {
             if (jj < a.JC) {
-              const uint32_t row = jj * a.TQ + tokc;
+              const uint32_t row = tokc * a.JC + jj;
               const uint4 w = lds128(vb + reg + sw128_off(row, c8 & 7));
               const float p = y[jj];
               acc[c8 * 8 + 0] = fmaf(p, bf16lo(w.x), acc[c8 * 8 + 0]);
@@ -323,7 +329,7 @@ __global__ void __launch_bounds__(192, 1)
           }
         }
         named_bar_sync(1, 128);
-        if (r == 0) mbar_arrive(bar(bars->empty[vst]));
+        if (r == 0) mbar_arrive(bar(bars->dempty[vst]));
       }
       // depth accumulator becomes O's starting value
 #pragma unroll
@@ -482,13 +488,11 @@ cudaError_t launch_forward_d(const Problem& p, const void* q, const void* k, con
     }
   }
   if (p.L > 0) {
-    // kd viewed as [bg][j][t][c] (token stride outer to the depth-entry stride inside the
-    // box) so one chunk lands rows (entry, token) -- consecutive tokens of one entry
-    // occupy consecutive swizzled rows.
-    const cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(p.T), cuuint64_t(p.L), BG};
-    const cuuint64_t str[3] = {cuuint64_t(p.L) * D * E, cuuint64_t(D) * E,
+    // kd as [bg][t][j][c]: one box lands JC entries of TQ tokens as rows (token, entry).
+    const cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(p.L), cuuint64_t(p.T), BG};
+    const cuuint64_t str[3] = {cuuint64_t(D) * E, cuuint64_t(p.L) * D * E,
                                cuuint64_t(p.T) * p.L * D * E};
-    const cuuint32_t box[4] = {64, cuuint32_t(tg.TQ), cuuint32_t(tg.JC), 1};
+    const cuuint32_t box[4] = {64, cuuint32_t(tg.JC), cuuint32_t(tg.TQ), 1};
     if (!make_map(encode, &mKD, kd, 4, dims, str, box) ||
         !make_map(encode, &mVD, vd, 4, dims, str, box)) {
       *why = "cuTensorMapEncodeTiled failed for kd/vd";
@@ -523,7 +527,7 @@ cudaError_t launch_forward_d(const Problem& p, const void* q, const void* k, con
     }
   }
   const unsigned grid = unsigned(BG) * unsigned(tg.nqt);
-  moda_fwd_kernel<D><<<grid, 192, Cfg::kSmemBytes, stream>>>(mQ, mK, mV, mKD, mVD, args);
+  moda_fwd_kernel<D><<<grid, kFwdThreads, Cfg::kSmemBytes, stream>>>(mQ, mK, mV, mKD, mVD, args);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) *why = "forward kernel launch failed";
   return e;
