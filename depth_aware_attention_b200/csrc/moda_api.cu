@@ -171,6 +171,8 @@ moda_status_t moda_backward(const void* q, const void* k, const void* v, const v
     return fail(MODA_ERR_INVALID_ARGUMENT, "workspace must be 256-byte aligned");
   if (!(scale == scale) || scale == INFINITY || scale == -INFINITY)
     return fail(MODA_ERR_INVALID_ARGUMENT, "scale must be finite");
+  if (Hq / Hkv > 16)
+    return fail(MODA_ERR_UNSUPPORTED, "the backward supports at most 16 query heads per KV head");
   moda::Problem p{B, Hq, Hkv, T, L, d, Hq / Hkv, causal ? 1 : 0, scale};
   const size_t need = moda::backward_workspace_bytes(p);
   if (workspace_bytes < need)

@@ -1,21 +1,699 @@
-// moda_bwd.cu -- MoDA backward for B200 (sm_100a).  (kernels follow)
+// moda_bwd.cu -- MoDA backward for B200 (sm_100a).
+//
+// The pages define the operator (hyper.ai summary of arXiv 2603.15619, section
+// "Mixture-of-Depths Attention (MoDA)": one jointly normalised softmax over the causal
+// sequence keys and the query token's own depth keys) but give no backward design.  This
+// file computes the exact gradient of that definition given dO, recomputing the softmax
+// weights from the forward's log-sum-exp:
+//   P = exp(scale*<q,key> - lse),  D = <dO, out>,  dS = P * (<dO, value> - D)
+//   dq = scale * sum dS * key;  dk, dkd = scale * sum dS * q;  dv, dvd = sum P * dO.
+//
+// Three launches:
+//  1. moda_bwd_depth_kernel (token-major, CUDA cores, bandwidth-bound): per token of one
+//     KV group, D for the G query rows, dkd/dvd for the token's L depth entries, and the
+//     depth share of dq, which initialises the fp32 dq accumulator.  Threads split the
+//     head dimension into 16-byte column chunks; dot products are finished with warp
+//     shuffles, so every depth byte is read from HBM once, with 16-byte coalesced loads.
+//  2. moda_bwd_seq_kernel (KV-block-major, tcgen05): one CTA owns 128 sequence keys of
+//     one KV head and walks every query tile that sees them.  Per tile the tensor cores
+//     compute S^T = K Q^T and dP^T = V dO^T into TMEM; the softmax warps turn them into
+//     P^T and dS^T (bf16, back into TMEM, and dS into shared memory); the tensor cores
+//     accumulate dV += P^T dO and dK += dS^T Q in TMEM for the whole walk and compute
+//     dQ = dS K, which the dQ warps add to the fp32 accumulator with vector atomics.
+//  3. moda_dq_convert_kernel: dq (bf16) from the fp32 accumulator.
+#include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <math.h>
 
 #include "moda_internal.h"
+#include "sm100.cuh"
 
 namespace moda {
+
+namespace {
+
+constexpr int kBwdRegion = 16384;  // one 128-row x 128-byte swizzled region
+constexpr float kLog2eBwd = 1.4426950408889634f;
+
+// ============================================================ 1. depth + row terms
+constexpr int kDepthThreads = 256;
+
+struct BwdDepthArgs {
+  const __nv_bfloat16 *q, *out, *dout, *kd, *vd;
+  const float* lse;
+  __nv_bfloat16 *dkd, *dvd;
+  float* dqacc;  // [B][Hq][T][D] fp32, written (not accumulated) here
+  float* drow;   // [B][Hq][T] fp32: D = <dO, out>
+  long long ntok;  // B * Hkv * T
+  int T, L, G;
+  float scale, scale_log2;
+};
+
+// One token slot = D/8 consecutive threads (one 16-byte column chunk each); a CTA works
+// on kDepthThreads/(D/8) consecutive tokens of the flattened [B*Hkv][T] token list at a
+// time.  The G query rows of the token keep q and dO in shared memory (bf16); the dq
+// partial sums of up to GM heads stay in registers.
+template <int D, int GM>
+__global__ void __launch_bounds__(kDepthThreads) moda_bwd_depth_kernel(const BwdDepthArgs a) {
+  constexpr int NT = D / 8;
+  constexpr int TPB = kDepthThreads / NT;
+  extern __shared__ __align__(16) uint8_t dsm[];
+  const int tid = threadIdx.x;
+  const int slot = tid / NT, cs = tid % NT;
+  const int G = a.G;
+  const uint32_t q_s = smem_u32(dsm) + uint32_t(slot * 2 * G * D * 2);
+  const uint32_t do_s = q_s + uint32_t(G * D * 2);
+  const long long L = a.L;
+
+  for (long long base = (long long)blockIdx.x * TPB; base < a.ntok;
+       base += (long long)gridDim.x * TPB) {
+    const long long tk = base + slot;
+    const bool valid = tk < a.ntok;
+    const long long tkc = valid ? tk : a.ntok - 1;
+    const long long bg = tkc / a.T;
+    const int t = int(tkc - bg * a.T);
+
+    float lse2[GM], drw[GM];
+#pragma unroll
+    for (int h = 0; h < GM; ++h) {
+      lse2[h] = 0.f;
+      drw[h] = 0.f;
+      if (h < G) {
+        const long long row = (bg * G + h) * a.T + t;
+        float part = 0.f;
+        if (valid) {
+          const uint4 qw = ldg_nc_v4(a.q + row * D + cs * 8);
+          const uint4 dw = ldg_nc_v4(a.dout + row * D + cs * 8);
+          const uint4 ow = ldg_nc_v4(a.out + row * D + cs * 8);
+          sts128(q_s + uint32_t((h * D + cs * 8) * 2), qw);
+          sts128(do_s + uint32_t((h * D + cs * 8) * 2), dw);
+          float df[8], of[8];
+          unpack8(dw, df);
+          unpack8(ow, of);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) part = fmaf(df[e], of[e], part);
+          lse2[h] = a.lse[row] * kLog2eBwd;
+        }
+#pragma unroll
+        for (int o = NT / 2; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+        drw[h] = part;
+        if (valid && cs == 0) a.drow[row] = part;
+      }
+    }
+    __syncwarp();
+
+    float dq[GM][8];
+#pragma unroll
+    for (int h = 0; h < GM; ++h)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) dq[h][e] = 0.f;
+
+    const long long tok_off = (bg * a.T + t) * L * D + cs * 8;
+    for (long long j = 0; j < L; ++j) {
+      uint4 kw = make_uint4(0, 0, 0, 0), vw = make_uint4(0, 0, 0, 0);
+      if (valid) {
+        kw = ldg_nc_v4(a.kd + tok_off + j * D);
+        vw = ldg_nc_v4(a.vd + tok_off + j * D);
+      }
+      float kf[8], vf[8];
+      unpack8(kw, kf);
+      unpack8(vw, vf);
+      float y[GM], p[GM];
+#pragma unroll
+      for (int h = 0; h < GM; ++h) {
+        y[h] = 0.f;
+        p[h] = 0.f;
+        if (h < G) {
+          float qf[8], df[8];
+          unpack8(lds128(q_s + uint32_t((h * D + cs * 8) * 2)), qf);
+          unpack8(lds128(do_s + uint32_t((h * D + cs * 8) * 2)), df);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            y[h] = fmaf(qf[e], kf[e], y[h]);
+            p[h] = fmaf(df[e], vf[e], p[h]);
+          }
+        }
+      }
+#pragma unroll
+      for (int o = NT / 2; o > 0; o >>= 1) {
+#pragma unroll
+        for (int h = 0; h < GM; ++h) {
+          if (h < G) {
+            y[h] += __shfl_xor_sync(0xffffffffu, y[h], o);
+            p[h] += __shfl_xor_sync(0xffffffffu, p[h], o);
+          }
+        }
+      }
+      float dv[8], dk[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) dv[e] = dk[e] = 0.f;
+#pragma unroll
+      for (int h = 0; h < GM; ++h) {
+        if (h < G) {
+          const float P = ex2(y[h] * a.scale_log2 - lse2[h]);
+          const float dS = P * (p[h] - drw[h]);
+          float qf[8], df[8];
+          unpack8(lds128(q_s + uint32_t((h * D + cs * 8) * 2)), qf);
+          unpack8(lds128(do_s + uint32_t((h * D + cs * 8) * 2)), df);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            dv[e] = fmaf(P, df[e], dv[e]);
+            dk[e] = fmaf(dS, qf[e], dk[e]);
+            dq[h][e] = fmaf(dS, kf[e], dq[h][e]);
+          }
+        }
+      }
+      if (valid) {
+        *reinterpret_cast<uint4*>(a.dvd + tok_off + j * D) = pack8(dv, 1.f);
+        *reinterpret_cast<uint4*>(a.dkd + tok_off + j * D) = pack8(dk, a.scale);
+      }
+    }
+    if (valid) {
+#pragma unroll
+      for (int h = 0; h < GM; ++h) {
+        if (h < G) {
+          const long long row = (bg * G + h) * a.T + t;
+          float4* dst = reinterpret_cast<float4*>(a.dqacc + row * D + cs * 8);
+          dst[0] = make_float4(dq[h][0] * a.scale, dq[h][1] * a.scale, dq[h][2] * a.scale,
+                               dq[h][3] * a.scale);
+          dst[1] = make_float4(dq[h][4] * a.scale, dq[h][5] * a.scale, dq[h][6] * a.scale,
+                               dq[h][7] * a.scale);
+        }
+      }
+    }
+    __syncwarp();  // the slot's q/dO copies are rewritten by the next pass
+  }
+}
+
+// ============================================================ 2. sequence part
+constexpr int kSeqThreads = 320;  // warps 0-3 P/dS, 4-7 dQ, 8 TMA, 9 tcgen05
+
+template <int D>
+struct SeqCfg {
+  static constexpr int kRegions = D / 64;
+  static constexpr int kTile = kRegions * kBwdRegion;  // 128 rows x D bf16, swizzled
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kTile;
+  static constexpr int kOffQ = 2 * kTile;   // two stages
+  static constexpr int kOffDO = 4 * kTile;  // two stages
+  static constexpr int kOffDS = 6 * kTile;  // dS, 128 rows x 128 keys bf16, MN-major
+  static constexpr int kOffLD = kOffDS + 2 * kBwdRegion;  // [2 stages][lse2 | D][128] f32
+  static constexpr int kOffBar = kOffLD + 2 * 2 * 128 * 4;
+  static constexpr int kSmemBytes = kOffBar + 256;
+};
+
+struct SeqBars {
+  uint64_t kv_full;
+  uint64_t q_full[2], q_empty[2];
+  uint64_t do_full[2], do_empty[2];
+  uint64_t s_full, dp_full, pds_full, dq_full, dq_free, kv_done;
+  uint32_t tmem_base;
+  int abort;
+};
+
+struct SeqArgs {
+  __nv_bfloat16 *dk, *dv;
+  float* dqacc;
+  const float *lse, *drow;
+  int Hkv, T, G, TQ, nqt, BG, causal;
+  float scale, scale_log2;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kSeqThreads, 1)
+    moda_bwd_seq_kernel(const __grid_constant__ CUtensorMap tmQ,
+                        const __grid_constant__ CUtensorMap tmDO,
+                        const __grid_constant__ CUtensorMap tmK,
+                        const __grid_constant__ CUtensorMap tmV, const SeqArgs a) {
+  using Cfg = SeqCfg<D>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  // The swizzled operand layouts need a 1024-byte aligned base, and there is no room
+  // to realign inside the shared-memory budget: refuse to run otherwise.
+  if (smem_u32(smem) & 1023u) {
+    if (threadIdx.x == 0) atomicOr(&g_error_word, kErrInternal);
+    return;
+  }
+  const uint32_t s0 = smem_u32(smem);
+  const uint32_t sK = s0 + Cfg::kOffK, sV = s0 + Cfg::kOffV, sDS = s0 + Cfg::kOffDS;
+  auto sQ = [&](int st) { return s0 + Cfg::kOffQ + uint32_t(st) * Cfg::kTile; };
+  auto sDO = [&](int st) { return s0 + Cfg::kOffDO + uint32_t(st) * Cfg::kTile; };
+  float* ld_s = reinterpret_cast<float*>(smem + Cfg::kOffLD);
+  SeqBars* bars = reinterpret_cast<SeqBars*>(smem + Cfg::kOffBar);
+  volatile int* abort_flag = &bars->abort;
+  auto bar = [&](uint64_t& b) { return smem_u32(&b); };
+
+  const int warp = threadIdx.x >> 5;
+  const int bg = blockIdx.x % a.BG;
+  const int kb = blockIdx.x / a.BG;  // key blocks nearest the start see the most tiles
+  const int key0 = kb * 128;
+  const int first_qt = a.causal ? key0 / a.TQ : 0;
+  const int ntiles = a.nqt - first_qt;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(bars->kv_full), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(bars->q_full[i]), 1);
+      mbar_init(bar(bars->q_empty[i]), 1);
+      mbar_init(bar(bars->do_full[i]), 1);
+      mbar_init(bar(bars->do_empty[i]), 1);
+    }
+    mbar_init(bar(bars->s_full), 1);
+    mbar_init(bar(bars->dp_full), 1);
+    mbar_init(bar(bars->pds_full), 128);
+    mbar_init(bar(bars->dq_full), 1);
+    mbar_init(bar(bars->dq_free), 128);
+    mbar_init(bar(bars->kv_done), 1);
+    bars->abort = 0;
+    fence_barrier_init();
+  }
+  // Q/dO rows past TQ*G (G not dividing 128) never receive TMA data: zero them once.
+  if (threadIdx.x < 128 && threadIdx.x >= a.TQ * a.G) {
+    for (int st = 0; st < 2; ++st)
+      for (int rg = 0; rg < Cfg::kRegions; ++rg) {
+        uint4* rq = reinterpret_cast<uint4*>(smem + Cfg::kOffQ + st * Cfg::kTile +
+                                             rg * kBwdRegion + threadIdx.x * 128);
+        uint4* rd = reinterpret_cast<uint4*>(smem + Cfg::kOffDO + st * Cfg::kTile +
+                                             rg * kBwdRegion + threadIdx.x * 128);
+        for (int c = 0; c < 8; ++c) rq[c] = rd[c] = make_uint4(0, 0, 0, 0);
+      }
+    fence_proxy_async_smem();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(&bars->tmem_base), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  // TMEM columns: S^T/P^T [0,128), dP^T/dS^T and then dQ [128,256), dV [256,256+D),
+  // dK [256+D, 256+2D).  P^T and dS^T are stored as bf16 hi/lo pairs: each 32-row chunk
+  // occupies 32 columns, 16 of packed hi values then 16 of packed lo values.
+  const uint32_t tS = tmem, tDP = tmem + 128, tDV = tmem + 256, tDK = tmem + 256 + D;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
+    if (elect_one()) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmDO);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      mbar_expect_tx(bar(bars->kv_full), 2 * Cfg::kTile);
+      for (int rg = 0; rg < Cfg::kRegions; ++rg) {
+        tma_load_3d(sK + rg * kBwdRegion, &tmK, bar(bars->kv_full), rg * 64, key0, bg);
+        tma_load_3d(sV + rg * kBwdRegion, &tmV, bar(bars->kv_full), rg * 64, key0, bg);
+      }
+      const uint32_t qbytes = Cfg::kRegions * 128 * a.G * a.TQ;
+      for (int i = 0; i < ntiles; ++i) {
+        const int st = i & 1;
+        const int t0 = (first_qt + i) * a.TQ;
+        if (i >= 2) mbar_wait(bar(bars->q_empty[st]), ((i >> 1) - 1) & 1, abort_flag);
+        mbar_expect_tx(bar(bars->q_full[st]), qbytes);
+        for (int rg = 0; rg < Cfg::kRegions; ++rg)
+          tma_load_4d(sQ(st) + rg * kBwdRegion, &tmQ, bar(bars->q_full[st]), rg * 64, 0, t0,
+                      bg);
+        if (i >= 2) mbar_wait(bar(bars->do_empty[st]), ((i >> 1) - 1) & 1, abort_flag);
+        mbar_expect_tx(bar(bars->do_full[st]), qbytes);
+        for (int rg = 0; rg < Cfg::kRegions; ++rg)
+          tma_load_4d(sDO(st) + rg * kBwdRegion, &tmDO, bar(bars->do_full[st]), rg * 64, 0,
+                      t0, bg);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ tcgen05 issuer
+    if (elect_one()) {
+      constexpr uint32_t idesc_t = make_idesc_bf16(128, 128, 0, 0);  // S^T, dP^T
+      constexpr uint32_t idesc_g = make_idesc_bf16(128, D, 0, 1);    // dV, dK (A in TMEM)
+      constexpr uint32_t idesc_q = make_idesc_bf16(128, D, 1, 1);    // dQ (A = dS, MN-major)
+      mbar_wait(bar(bars->kv_full), 0, abort_flag);
+      for (int i = 0; i < ntiles; ++i) {
+        const int st = i & 1;
+        const uint32_t par = (i >> 1) & 1;
+        mbar_wait(bar(bars->q_full[st]), par, abort_flag);
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t off = (ks / 4) * kBwdRegion + (ks % 4) * 32;
+          mma_ss(tS, make_sdesc_sw128(sK + off, 16, 1024), make_sdesc_sw128(sQ(st) + off, 16, 1024),
+                 idesc_t, ks > 0 ? 1u : 0u);
+        }
+        tc_commit(bar(bars->s_full));
+        mbar_wait(bar(bars->do_full[st]), par, abort_flag);
+        if (i > 0) mbar_wait(bar(bars->dq_free), (i - 1) & 1, abort_flag);
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t off = (ks / 4) * kBwdRegion + (ks % 4) * 32;
+          mma_ss(tDP, make_sdesc_sw128(sV + off, 16, 1024),
+                 make_sdesc_sw128(sDO(st) + off, 16, 1024), idesc_t, ks > 0 ? 1u : 0u);
+        }
+        tc_commit(bar(bars->dp_full));
+        mbar_wait(bar(bars->pds_full), i & 1, abort_flag);
+        tc_fence_after();
+        // dV += P^T dO : A = P^T (TMEM, keys x rows; hi then lo), B = dO (rows x D, MN-major).
+        // K-step ks covers rows 16ks..16ks+15: packed columns 32(ks/2) + 8(ks%2), lo +16.
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t col = (ks >> 1) * 32 + (ks & 1) * 8;
+          const uint64_t bd = make_sdesc_sw128(sDO(st) + ks * 2048, kBwdRegion, 1024);
+          mma_ts(tDV, tS + col, bd, idesc_g, (i > 0 || ks > 0) ? 1u : 0u);
+          mma_ts(tDV, tS + col + 16, bd, idesc_g, 1u);
+        }
+        tc_commit(bar(bars->do_empty[st]));
+        // dK += dS^T Q (hi then lo)
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t col = (ks >> 1) * 32 + (ks & 1) * 8;
+          const uint64_t bd = make_sdesc_sw128(sQ(st) + ks * 2048, kBwdRegion, 1024);
+          mma_ts(tDK, tDP + col, bd, idesc_g, (i > 0 || ks > 0) ? 1u : 0u);
+          mma_ts(tDK, tDP + col + 16, bd, idesc_g, 1u);
+        }
+        // dQ = dS K : A = dS (rows x keys, MN-major in shared memory), B = K (keys x D)
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          mma_ss(tDP, make_sdesc_sw128(sDS + ks * 2048, kBwdRegion, 1024),
+                 make_sdesc_sw128(sK + ks * 2048, kBwdRegion, 1024), idesc_q, ks > 0 ? 1u : 0u);
+        tc_commit(bar(bars->q_empty[st]));
+        tc_commit(bar(bars->dq_full));
+      }
+      tc_commit(bar(bars->kv_done));
+    }
+    __syncwarp();
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ P / dS warps
+    const int tid = threadIdx.x;  // TMEM lane = key key0 + tid
+    const int key = key0 + tid;
+    const uint32_t lane_base = uint32_t(warp * 32) << 16;
+    const int hl = tid % a.G, tok = tid / a.G;
+    for (int i = 0; i < ntiles; ++i) {
+      const int qt = first_qt + i;
+      const int b = i & 1;
+      {
+        const int t = qt * a.TQ + tok;
+        const bool valid = tok < a.TQ && t < a.T;
+        const long long idx = ((long long)bg * a.G + hl) * a.T + t;
+        ld_s[b * 256 + tid] = valid ? a.lse[idx] * kLog2eBwd : INFINITY;
+        ld_s[b * 256 + 128 + tid] = valid ? a.drow[idx] : 0.f;
+      }
+      named_bar_sync(1, 128);
+      // rows r < r_min hold tokens before this key (causal) -- their weight is zero
+      int r_min = 0;
+      if (key >= a.T)
+        r_min = 1 << 30;
+      else if (a.causal)
+        r_min = a.G * (key - qt * a.TQ);
+      const float* lse2 = ld_s + b * 256;
+      const float* dr = ld_s + b * 256 + 128;
+      mbar_wait(bar(bars->s_full), i & 1, abort_flag);
+      mbar_wait(bar(bars->dp_full), i & 1, abort_flag);
+      tc_fence_after();
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t s[32], dp[32];
+        tmem_ld32(tS + lane_base + c * 32, s);
+        tmem_ld32(tDP + lane_base + c * 32, dp);
+        tmem_wait_ld();
+        // P and dS as bf16 pairs hi + lo (lo = what bf16 rounding dropped): the dV and dK
+        // products use both, so their operands carry about 2^-17 relative error instead
+        // of 2^-9.  Chunk c writes its 32 columns back over the 32 it read: hi in the
+        // first 16, lo in the last 16.
+        uint32_t pp[16], pl[16], pd[16], dl[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const int r = c * 32 + e;
+          float P0 = ex2(__uint_as_float(s[e]) * a.scale_log2 - lse2[r]);
+          float P1 = ex2(__uint_as_float(s[e + 1]) * a.scale_log2 - lse2[r + 1]);
+          if (r < r_min) P0 = 0.f;
+          if (r + 1 < r_min) P1 = 0.f;
+          const float d0 = P0 * (__uint_as_float(dp[e]) - dr[r]) * a.scale;
+          const float d1 = P1 * (__uint_as_float(dp[e + 1]) - dr[r + 1]) * a.scale;
+          const uint32_t ph = pack_bf16x2(P0, P1), dh = pack_bf16x2(d0, d1);
+          pp[e / 2] = ph;
+          pl[e / 2] = pack_bf16x2(P0 - bf16lo(ph), P1 - bf16hi(ph));
+          pd[e / 2] = dh;
+          dl[e / 2] = pack_bf16x2(d0 - bf16lo(dh), d1 - bf16hi(dh));
+        }
+        tmem_st16(tS + lane_base + c * 32, pp);
+        tmem_st16(tS + lane_base + c * 32 + 16, pl);
+        tmem_st16(tDP + lane_base + c * 32, pd);
+        tmem_st16(tDP + lane_base + c * 32 + 16, dl);
+        // dS row-block for the dQ product: rows c*32..c*32+31 of this key's column
+        const uint32_t reg = sDS + (c >> 1) * kBwdRegion + uint32_t(tid) * 128;
+#pragma unroll
+        for (int qd = 0; qd < 4; ++qd) {
+          const uint32_t chunk = (c & 1) * 4 + qd;
+          sts128(reg + ((chunk ^ (tid & 7)) << 4),
+                 make_uint4(pd[qd * 4], pd[qd * 4 + 1], pd[qd * 4 + 2], pd[qd * 4 + 3]));
+        }
+      }
+      tmem_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar(bars->pds_full));
+    }
+    // epilogue: dV, dK rows of this key
+    mbar_wait(bar(bars->kv_done), 0, abort_flag);
+    tc_fence_after();
+    const bool kvalid = key < a.T;
+    const long long koff = ((long long)bg * a.T + (kvalid ? key : 0)) * D;
+#pragma unroll 1
+    for (int which = 0; which < 2; ++which) {
+      const uint32_t tsrc = (which ? tDK : tDV) + lane_base;
+      __nv_bfloat16* dst = (which ? a.dk : a.dv) + koff;
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t o[32];
+        tmem_ld32(tsrc + cc * 32, o);
+        tmem_wait_ld();
+        if (kvalid) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            float f[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(o[v * 8 + e]);
+            d4[v] = pack8(f, 1.f);
+          }
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ dQ warps 4-7
+    const int r = threadIdx.x - 128;  // TMEM lane = tile row
+    const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
+    const int hl = r % a.G, tok = r / a.G;
+    for (int i = 0; i < ntiles; ++i) {
+      const int t = (first_qt + i) * a.TQ + tok;
+      const bool valid = tok < a.TQ && t < a.T;
+      float* dst = a.dqacc + (((long long)bg * a.G + hl) * a.T + (valid ? t : 0)) * D;
+      mbar_wait(bar(bars->dq_full), i & 1, abort_flag);
+      tc_fence_after();
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t o[32];
+        tmem_ld32(tDP + lane_base + cc * 32, o);
+        tmem_wait_ld();
+        if (valid) {
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            red_add_v4(dst + cc * 32 + v * 4, __uint_as_float(o[v * 4]),
+                       __uint_as_float(o[v * 4 + 1]), __uint_as_float(o[v * 4 + 2]),
+                       __uint_as_float(o[v * 4 + 3]));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(bars->dq_free));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ============================================================ 3. dq convert
+__global__ void __launch_bounds__(256) moda_dq_convert_kernel(const float* __restrict__ acc,
+                                                              __nv_bfloat16* __restrict__ dq,
+                                                              long long n8) {
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n8;
+       i += (long long)gridDim.x * blockDim.x) {
+    const float4 x = reinterpret_cast<const float4*>(acc)[2 * i];
+    const float4 y = reinterpret_cast<const float4*>(acc)[2 * i + 1];
+    const float f[8] = {x.x, x.y, x.z, x.w, y.x, y.y, y.z, y.w};
+    reinterpret_cast<uint4*>(dq)[i] = pack8(f, 1.f);
+  }
+}
+
+// ============================================================ host side
+bool make_map_b(EncodeTiledFn encode, CUtensorMap* map, const void* base, int rank,
+                const cuuint64_t* dims, const cuuint64_t* strides_bytes, const cuuint32_t* box) {
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  return encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims,
+                strides_bytes, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+template <int D, int GM>
+cudaError_t launch_depth(const BwdDepthArgs& a, cudaStream_t stream, const char** why) {
+  const int tpb = kDepthThreads / (D / 8);
+  const size_t smem = size_t(tpb) * 2 * a.G * D * 2;
+  cudaError_t e = cudaFuncSetAttribute(moda_bwd_depth_kernel<D, GM>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) {
+    *why = "cudaFuncSetAttribute(depth backward) failed";
+    return e;
+  }
+  int per_sm = 1;
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, moda_bwd_depth_kernel<D, GM>,
+                                                kDepthThreads, smem);
+  if (per_sm < 1) per_sm = 1;
+  const long long need = (a.ntok + tpb - 1) / tpb;
+  const long long cap = (long long)sm_count() * per_sm;
+  const unsigned grid = unsigned(need < cap ? need : cap);
+  moda_bwd_depth_kernel<D, GM><<<grid, kDepthThreads, smem, stream>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) *why = "depth backward launch failed";
+  return e;
+}
+
+template <int D>
+cudaError_t launch_backward_d(const Problem& p, const void* q, const void* k, const void* v,
+                              const void* kd, const void* vd, const void* out,
+                              const float* lse, const void* dout, void* dq, void* dk,
+                              void* dv, void* dkd, void* dvd, void* workspace,
+                              EncodeTiledFn encode, cudaStream_t stream, const char** why) {
+  const TileGeom tg = tile_geom(p);
+  const long long rows = (long long)p.B * p.Hq * p.T;
+  float* dqacc = static_cast<float*>(workspace);
+  float* drow = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + rows * D * 4);
+
+  // 1. depth part, row terms, dq accumulator initialisation
+  BwdDepthArgs da;
+  da.q = static_cast<const __nv_bfloat16*>(q);
+  da.out = static_cast<const __nv_bfloat16*>(out);
+  da.dout = static_cast<const __nv_bfloat16*>(dout);
+  da.kd = static_cast<const __nv_bfloat16*>(kd);
+  da.vd = static_cast<const __nv_bfloat16*>(vd);
+  da.lse = lse;
+  da.dkd = static_cast<__nv_bfloat16*>(dkd);
+  da.dvd = static_cast<__nv_bfloat16*>(dvd);
+  da.dqacc = dqacc;
+  da.drow = drow;
+  da.ntok = (long long)p.B * p.Hkv * p.T;
+  da.T = p.T;
+  da.L = p.L;
+  da.G = p.G;
+  da.scale = p.scale;
+  da.scale_log2 = p.scale * kLog2eBwd;
+  cudaError_t e;
+  if (p.G <= 1)
+    e = launch_depth<D, 1>(da, stream, why);
+  else if (p.G <= 2)
+    e = launch_depth<D, 2>(da, stream, why);
+  else if (p.G <= 4)
+    e = launch_depth<D, 4>(da, stream, why);
+  else if (p.G <= 8)
+    e = launch_depth<D, 8>(da, stream, why);
+  else
+    e = launch_depth<D, 16>(da, stream, why);
+  if (e != cudaSuccess) return e;
+
+  // 2. sequence part
+  const cuuint64_t E = 2;
+  const cuuint64_t BG = cuuint64_t(p.B) * p.Hkv;
+  CUtensorMap mQ, mDO, mK, mV;
+  {
+    const cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(p.G), cuuint64_t(p.T), BG};
+    const cuuint64_t str[3] = {cuuint64_t(p.T) * D * E, cuuint64_t(D) * E,
+                               cuuint64_t(p.G) * p.T * D * E};
+    const cuuint32_t box[4] = {64, cuuint32_t(p.G), cuuint32_t(tg.TQ), 1};
+    if (!make_map_b(encode, &mQ, q, 4, dims, str, box) ||
+        !make_map_b(encode, &mDO, dout, 4, dims, str, box)) {
+      *why = "cuTensorMapEncodeTiled failed for q/dout";
+      return cudaErrorInvalidValue;
+    }
+  }
+  {
+    const cuuint64_t dims[3] = {cuuint64_t(D), cuuint64_t(p.T), BG};
+    const cuuint64_t str[2] = {cuuint64_t(D) * E, cuuint64_t(p.T) * D * E};
+    const cuuint32_t box[3] = {64, 128, 1};
+    if (!make_map_b(encode, &mK, k, 3, dims, str, box) ||
+        !make_map_b(encode, &mV, v, 3, dims, str, box)) {
+      *why = "cuTensorMapEncodeTiled failed for k/v";
+      return cudaErrorInvalidValue;
+    }
+  }
+  SeqArgs sa;
+  sa.dk = static_cast<__nv_bfloat16*>(dk);
+  sa.dv = static_cast<__nv_bfloat16*>(dv);
+  sa.dqacc = dqacc;
+  sa.lse = lse;
+  sa.drow = drow;
+  sa.Hkv = p.Hkv;
+  sa.T = p.T;
+  sa.G = p.G;
+  sa.TQ = tg.TQ;
+  sa.nqt = tg.nqt;
+  sa.BG = int(BG);
+  sa.causal = p.causal;
+  sa.scale = p.scale;
+  sa.scale_log2 = p.scale * kLog2eBwd;
+  e = cudaFuncSetAttribute(moda_bwd_seq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           SeqCfg<D>::kSmemBytes);
+  if (e != cudaSuccess) {
+    *why = "cudaFuncSetAttribute(sequence backward) failed";
+    return e;
+  }
+  const int nkb = (p.T + 127) / 128;
+  moda_bwd_seq_kernel<D><<<unsigned(BG) * nkb, kSeqThreads, SeqCfg<D>::kSmemBytes, stream>>>(
+      mQ, mDO, mK, mV, sa);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    *why = "sequence backward launch failed";
+    return e;
+  }
+
+  // 3. dq (bf16)
+  const long long n8 = rows * D / 8;
+  long long blocks = (n8 + 255) / 256;
+  if (blocks > 8LL * sm_count()) blocks = 8LL * sm_count();
+  moda_dq_convert_kernel<<<unsigned(blocks), 256, 0, stream>>>(
+      dqacc, static_cast<__nv_bfloat16*>(dq), n8);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) *why = "dq convert launch failed";
+  return e;
+}
+
+}  // namespace
 
 size_t backward_workspace_bytes(const Problem& p) {
   const size_t rows = size_t(p.B) * p.Hq * p.T;
   return rows * p.d * 4 + rows * 4 + 256;
 }
 
-cudaError_t launch_backward(const Problem&, const void*, const void*, const void*,
-                            const void*, const void*, const void*, const float*, const void*,
-                            void*, void*, void*, void*, void*, void*, EncodeTiledFn,
-                            cudaStream_t, const char** why) {
-  *why = "backward kernels are not built yet";
-  return cudaErrorNotSupported;
+cudaError_t launch_backward(const Problem& p, const void* q, const void* k, const void* v,
+                            const void* kd, const void* vd, const void* out, const float* lse,
+                            const void* dout, void* dq, void* dk, void* dv, void* dkd,
+                            void* dvd, void* workspace, EncodeTiledFn encode,
+                            cudaStream_t stream, const char** why) {
+  if (p.d == 128)
+    return launch_backward_d<128>(p, q, k, v, kd, vd, out, lse, dout, dq, dk, dv, dkd, dvd,
+                                  workspace, encode, stream, why);
+  return launch_backward_d<64>(p, q, k, v, kd, vd, out, lse, dout, dq, dk, dv, dkd, dvd,
+                               workspace, encode, stream, why);
 }
 
 }  // namespace moda

@@ -80,6 +80,8 @@ size_t moda_backward_workspace_size(int B, int Hq, int Hkv, int T, int L, int d)
  * D = <dout, out> per row and dS = P * (<dout, value> - D):
  *   dq = scale * sum dS * key,  dk/dkd = scale * sum dS * q,  dv/dvd = sum P * dout.
  * The pages give no backward design; this is the exact gradient of the definition.
+ * Supports Hq / Hkv <= 16 (MODA_ERR_UNSUPPORTED beyond).  dq is summed with fp32 atomics,
+ * so its last bits may differ between runs; dk, dv, dkd and dvd are deterministic.
  * `out` and `lse` must be the forward's outputs for the same inputs.  `workspace`
  * (device, >= moda_backward_workspace_size bytes, 256-byte aligned) is scratch owned
  * by the caller; its contents on entry do not matter.

@@ -2,8 +2,14 @@
 fp64 oracle on the same bf16 bits (whole problem or token windows), compare with the
 stated tolerances.
 
-Tolerances (bf16 outputs, fp32 accumulation on the GPU): max-abs error <= 1e-2 and
-mean-abs error <= 1e-3 against the fp64 oracle's unrounded result; lse within 1e-3.
+Tolerances (bf16 outputs, fp32 accumulation on the GPU), against the fp64 oracle's unrounded
+result: max-abs error <= 1e-2 and mean-abs error <= 1e-3; lse within 1e-3.
+
+The max-abs bound is applied beyond the output format's own rounding: element x may differ
+from the exact value by 1e-2 plus half a bf16 ULP of x.  No bf16 number lies within 1e-2 of
+some reals above 4 (bf16's spacing there is 1/32), so an exact kernel would otherwise fail
+on large gradient entries.  For |x| < 2 the extra term is at most 2^-8.  Gradients are also
+held to a relative RMS error of 1e-2 (bf16 operands carry 2^-9 relative rounding).
 """
 from __future__ import annotations
 
@@ -14,6 +20,18 @@ import oracle
 import workloads
 
 OUT_MAX, OUT_MEAN, LSE_MAX = 1e-2, 1e-3, 1e-3
+GRAD_REL_RMS = 1e-2
+
+
+def bf16_half_ulp(x):
+    """Half the spacing of bf16 numbers at |x| (8 significant bits)."""
+    a = np.maximum(np.abs(x), 2.0 ** -126)
+    return np.exp2(np.floor(np.log2(a)) - 8.0)
+
+
+def excess(err, ref):
+    """Error beyond the bf16 output rounding allowance (<= OUT_MAX passes)."""
+    return err - bf16_half_ulp(ref)
 
 
 def gpu_inputs(cfg, seed_base, with_dout=False, device="cuda"):
@@ -48,7 +66,8 @@ def compare_forward(out, lse, ref_out, ref_lse, what=""):
     err = np.abs(o - ref_out)
     lerr = np.abs(ls - ref_lse)
     assert np.isfinite(o).all(), f"{what}: non-finite output"
-    assert err.max() <= OUT_MAX, f"{what}: out max-abs {err.max():.3e}"
+    ex = excess(err, ref_out)
+    assert ex.max() <= OUT_MAX, f"{what}: out max-abs {err.max():.3e} (beyond rounding {ex.max():.3e})"
     assert err.mean() <= OUT_MEAN, f"{what}: out mean-abs {err.mean():.3e}"
     assert lerr.max() <= LSE_MAX, f"{what}: lse max-abs {lerr.max():.3e}"
     return float(err.max()), float(err.mean()), float(lerr.max())
@@ -58,6 +77,11 @@ def compare_grad(g, ref, what, max_tol=OUT_MAX, mean_tol=OUT_MEAN):
     a = g.detach().to("cpu", torch.float64).numpy()
     err = np.abs(a - ref)
     assert np.isfinite(a).all(), f"{what}: non-finite"
-    assert err.max() <= max_tol, f"{what}: max-abs {err.max():.3e}"
+    ex = excess(err, ref)
+    assert ex.max() <= max_tol, f"{what}: max-abs {err.max():.3e} (beyond rounding {ex.max():.3e})"
     assert err.mean() <= mean_tol, f"{what}: mean-abs {err.mean():.3e}"
+    rms = float(np.sqrt((ref ** 2).mean()))
+    if rms > 0:
+        rel = float(np.sqrt((err ** 2).mean())) / rms
+        assert rel <= GRAD_REL_RMS, f"{what}: relative RMS error {rel:.3e}"
     return float(err.max()), float(err.mean())

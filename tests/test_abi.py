@@ -98,6 +98,8 @@ def test_backward_rejects_small_workspace_and_aliasing():
     assert st == moda.MODA_ERR_INVALID_ARGUMENT
     st = moda.moda_backward(**args, **dict(base, workspace=A * 64 + 16))  # not 256-aligned
     assert st == moda.MODA_ERR_INVALID_ARGUMENT
+    st = moda.moda_backward(**args, **dict(base, Hq=64, Hkv=2))  # group of 32 heads
+    assert st == moda.MODA_ERR_UNSUPPORTED
 
 
 def test_binding_has_no_fallback():
