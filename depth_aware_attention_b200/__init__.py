@@ -29,7 +29,8 @@ BACKWARD_LAUNCHES = 3
 
 # Every symbol include/moda.h declares (checked by the ABI tests).
 EXPORTED = ("moda_forward", "moda_backward", "moda_backward_workspace_size",
-            "moda_check_device_errors", "moda_status_string", "moda_last_error_message")
+            "moda_backward_noalloc", "moda_check_device_errors", "moda_status_string",
+            "moda_last_error_message")
 
 
 class ModaError(RuntimeError):
@@ -51,6 +52,8 @@ def _load():
     lib.moda_backward_workspace_size.restype = S
     lib.moda_backward.argtypes = [P] * 14 + [S] + [I] * 6 + [F, I, P]
     lib.moda_backward.restype = I
+    lib.moda_backward_noalloc.argtypes = [P] * 13 + [I] * 6 + [F, I, P]
+    lib.moda_backward_noalloc.restype = I
     lib.moda_check_device_errors.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
     lib.moda_check_device_errors.restype = I
     lib.moda_status_string.argtypes = [I]
@@ -86,6 +89,13 @@ def moda_backward(q, k, v, kd, vd, out, lse, dout, dq, dk, dv, dkd, dvd, workspa
     return lib.moda_backward(q, k, v, kd, vd, out, lse, dout, dq, dk, dv, dkd, dvd,
                              workspace, workspace_bytes, B, Hq, Hkv, T, L, d, float(scale),
                              int(causal), stream)
+
+
+def moda_backward_noalloc(q, k, v, kd, vd, out, lse, dout, dq, dk, dv, dkd, dvd, B, Hq, Hkv,
+                          T, L, d, scale, causal, stream):
+    """The backward with library-owned static scratch (no workspace argument)."""
+    return lib.moda_backward_noalloc(q, k, v, kd, vd, out, lse, dout, dq, dk, dv, dkd, dvd, B,
+                                     Hq, Hkv, T, L, d, float(scale), int(causal), stream)
 
 
 def moda_backward_workspace_size(B, Hq, Hkv, T, L, d):

@@ -3,3 +3,4 @@
 #include "moda_api.cu"
 #include "moda_fwd.cu"
 #include "moda_bwd.cu"
+#include "moda_noalloc.cu"

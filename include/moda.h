@@ -94,6 +94,33 @@ moda_status_t moda_backward(const void *q, const void *k, const void *v, const v
                             moda_stream_t stream);
 
 /*
+ * The backward of moda_backward for callers that cannot allocate device memory: those
+ * whose device memory is owned by another allocator or by a fixed memory plan that hands
+ * out only the tensors it planned, and those calling through a plain C binding with no
+ * device allocation API.  (The paper has no counterpart; this is an interface addition.)
+ *
+ * Same arguments and results as moda_backward, without the workspace: the library takes
+ * it from a static device array of 64 MiB that every GPU loading the library holds until
+ * the process exits.  Neither the caller nor the library allocates anything.
+ *   - Sizes whose moda_backward_workspace_size() exceeds 64 MiB are rejected with
+ *     MODA_ERR_UNSUPPORTED (about B*Hq*T <= 130000 rows at d = 128).
+ *   - The first call on a device (the calling thread's current device) looks up the
+ *     array's device address with cudaGetSymbolAddress; make that first call before any
+ *     stream capture begins.
+ *   - Every call on a device shares the one array and leaves its contents behind.  The
+ *     backward writes every workspace element it reads before reading it, so nothing has
+ *     to be cleared between calls, but calls that may overlap on the GPU (different
+ *     streams, or concurrent host threads) race on the array and must be serialised by
+ *     the caller.
+ */
+moda_status_t moda_backward_noalloc(const void *q, const void *k, const void *v,
+                                    const void *kd, const void *vd, const void *out,
+                                    const float *lse, const void *dout, void *dq, void *dk,
+                                    void *dv, void *dkd, void *dvd, int B, int Hq, int Hkv,
+                                    int T, int L, int d, float scale, int causal,
+                                    moda_stream_t stream);
+
+/*
  * Synchronises `stream`, then reads and clears the calling device's kernel error word.
  * *flags (may be NULL) receives the raw bits: 1 = a bounded wait ran out, 2 = an
  * internal index/consistency check failed.  Returns MODA_ERR_TIMEOUT / MODA_ERR_INTERNAL
