@@ -10,7 +10,8 @@ point follows the definition of the operator on the hyper.ai summary of arXiv
 2603.15619, section "Mixture-of-Depths Attention (MoDA)": one softmax, jointly
 normalised, over the query's causal sequence keys and its own token's depth keys.
 
-Parity status: forward, backward and the row-weight view are pinned by the
+Parity status: forward, backward, the backward with a given output and the row-weight
+view are pinned by the
 ``-m "not gpu"`` tests in ``tests/test_oracle_pins.py`` (library special cases, closed
 forms, invariants, finite differences and hand-derived golden cases).
 """
@@ -46,6 +47,8 @@ def _load():
         lib.moda_oracle_forward.argtypes = [P] * 7 + [I] * 8 + [D, I, I]
         lib.moda_oracle_backward.argtypes = [P] * 13 + [I] * 8 + [D, I, I]
         lib.moda_oracle_row_weights.argtypes = [P] * 3 + [I] * 9 + [D, I, P, P]
+        lib.moda_oracle_backward_given_out.argtypes = [P] * 12 + [I] * 8 + [D, I, I]
+        lib.moda_oracle_backward_given_out.restype = I
         for f in (lib.moda_oracle_forward, lib.moda_oracle_backward,
                   lib.moda_oracle_row_weights):
             f.restype = I
@@ -129,6 +132,38 @@ def backward(q, k, v, kd, vd, dout, scale, causal=True, t0=0, nthreads=None):
     if rc != 0:
         raise ValueError("moda_oracle_backward rejected the sizes")
     return dict(dq=dq, dk=dk, dv=dv, dkd=dkd, dvd=dvd, out=out, lse=lse)
+
+
+def backward_given_out(q, k, v, kd, vd, dout, out, scale, causal=True, t0=0, nthreads=None):
+    """Oracle backward whose row terms D = <dO, out> use the given ``out`` (window-sized,
+    e.g. the forward's bf16 output widened) instead of the oracle's exact output.
+
+    Everything else is exactly moda's gradient: P comes from the exact logits and
+    log-sum-exp.  This is the exact result a backward can reach when it is handed only
+    the forward's rounded output.  Returns dict(dq, dk, dv, dkd, dvd), same windows as
+    ``backward``.
+    """
+    q, k, v, dout, out = _f64(q), _f64(k), _f64(v), _f64(dout), _f64(out)
+    B, Hq, nt, d = q.shape
+    Hkv, T = k.shape[1], k.shape[2]
+    if kd is None or kd.shape[3] == 0:
+        L = 0
+        kd = vd = np.zeros((1,), np.float64)
+    else:
+        kd, vd = _f64(kd), _f64(vd)
+        L = kd.shape[3]
+    dq = np.empty((B, Hq, nt, d), np.float64)
+    dk = np.empty((B, Hkv, T, d), np.float64)
+    dv = np.empty((B, Hkv, T, d), np.float64)
+    dkd = np.empty((B, Hkv, nt, L, d), np.float64)
+    dvd = np.empty((B, Hkv, nt, L, d), np.float64)
+    rc = _load().moda_oracle_backward_given_out(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(kd), _ptr(vd), _ptr(dout), _ptr(out), _ptr(dq),
+        _ptr(dk), _ptr(dv), _ptr(dkd), _ptr(dvd), B, Hq, Hkv, T, L, d, t0, nt, float(scale),
+        int(bool(causal)), nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("moda_oracle_backward_given_out rejected the arguments")
+    return dict(dq=dq, dk=dk, dv=dv, dkd=dkd, dvd=dvd)
 
 
 def row_weights(q, k, kd, b, h, t, scale, causal=True):

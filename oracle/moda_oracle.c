@@ -56,6 +56,7 @@
 
 typedef struct {
     const double *q, *k, *v, *kd, *vd, *dout;
+    const double *out_given; /* backward only: if set, D = <dO, out_given> (see below) */
     double *out, *lse, *dq, *dk, *dv, *dkd, *dvd;
     int64_t nunits;
     int B, Hq, Hkv, T, L, d, causal;
@@ -157,7 +158,7 @@ static void backward_unit(job_t *J, int b, int g, double *scratch, double *o_row
             double lse;
             forward_row(J, b, h, w, scratch, o_row, &lse);
             if (J->out) { memcpy(J->out + r * d, o_row, sizeof(double) * d); J->lse[r] = lse; }
-            const double D = dot(dor, o_row, d);
+            const double D = dot(dor, J->out_given ? J->out_given + r * d : o_row, d);
             /* sequence keys: logits are in scratch[0..ns) from forward_row */
             for (int s = 0; s < ns; ++s) {
                 const double P = exp(scratch[s] - lse);
@@ -238,6 +239,20 @@ int moda_oracle_forward(const double *q, const double *k, const double *v,
  *   with causal=1 and t0+nt=T, dk/dv of every key s >= t0 are exact (only rows of
  *   tokens t >= s see key s); the full backward is the window t0=0, nt=T.
  * If out/lse are non-NULL the oracle's own forward results are written there too. */
+/* Backward whose row terms D = <dO, out> use a caller-given `out` (window-sized, like q)
+ * instead of the oracle's own exact output; every other quantity (the logits, P from the
+ * exact log-sum-exp, the value products) is computed exactly as in moda_oracle_backward.
+ * A backward that receives only the forward's rounded output (the operator's backward
+ * interface takes `out` as an input) can at best compute D from it, and this mode is the
+ * exact result of that; with out_given = the oracle's own out it equals
+ * moda_oracle_backward. */
+int moda_oracle_backward_given_out(const double *q, const double *k, const double *v,
+                                   const double *kd, const double *vd, const double *dout,
+                                   const double *out_given, double *dq, double *dk,
+                                   double *dv, double *dkd, double *dvd, int B, int Hq,
+                                   int Hkv, int T, int L, int d, int t0, int nt,
+                                   double scale, int causal, int nthreads);
+
 int moda_oracle_backward(const double *q, const double *k, const double *v,
                          const double *kd, const double *vd, const double *dout,
                          double *dq, double *dk, double *dv, double *dkd, double *dvd,
@@ -253,6 +268,29 @@ int moda_oracle_backward(const double *q, const double *k, const double *v,
     job_t J = {0};
     J.q = q; J.k = k; J.v = v; J.kd = kd; J.vd = vd; J.dout = dout;
     J.dq = dq; J.dk = dk; J.dv = dv; J.dkd = dkd; J.dvd = dvd; J.out = out; J.lse = lse;
+    J.B = B; J.Hq = Hq; J.Hkv = Hkv; J.T = T; J.L = L; J.d = d; J.causal = causal;
+    J.t0 = t0; J.nt = nt; J.scale = scale;
+    J.nunits = (int64_t)B * Hkv;
+    run(&J, backward_worker, nthreads);
+    return 0;
+}
+
+int moda_oracle_backward_given_out(const double *q, const double *k, const double *v,
+                                   const double *kd, const double *vd, const double *dout,
+                                   const double *out_given, double *dq, double *dk,
+                                   double *dv, double *dkd, double *dvd, int B, int Hq,
+                                   int Hkv, int T, int L, int d, int t0, int nt,
+                                   double scale, int causal, int nthreads) {
+    if (bad_dims(B, Hq, Hkv, T, L, d, t0, nt) || !out_given) return 1;
+    const size_t nq = (size_t)B * Hq * nt * d, nk = (size_t)B * Hkv * T * d;
+    const size_t nd = (size_t)B * Hkv * nt * (size_t)L * d;
+    memset(dq, 0, nq * sizeof(double));
+    memset(dk, 0, nk * sizeof(double));
+    memset(dv, 0, nk * sizeof(double));
+    if (nd) { memset(dkd, 0, nd * sizeof(double)); memset(dvd, 0, nd * sizeof(double)); }
+    job_t J = {0};
+    J.q = q; J.k = k; J.v = v; J.kd = kd; J.vd = vd; J.dout = dout; J.out_given = out_given;
+    J.dq = dq; J.dk = dk; J.dv = dv; J.dkd = dkd; J.dvd = dvd;
     J.B = B; J.Hq = Hq; J.Hkv = Hkv; J.T = T; J.L = L; J.d = d; J.causal = causal;
     J.t0 = t0; J.nt = nt; J.scale = scale;
     J.nunits = (int64_t)B * Hkv;

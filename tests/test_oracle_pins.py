@@ -297,3 +297,38 @@ def test_seeded_inputs_are_reproducible_bf16():
     # N(0,1): sample mean/std sanity on the largest tensor
     assert abs(float(a["kd"].float().mean())) < 0.05
     assert abs(float(a["kd"].float().std()) - 1.0) < 0.05
+
+
+# ---------------------------------------------------------------- backward with a given out
+def test_backward_given_own_out_equals_backward():
+    x = rand_problem(B=1, T=11, Hq=4, Hkv=2, d=8, L=3, seed=41)
+    scale = 0.35
+    ref = oracle.backward(x["q"], x["k"], x["v"], x["kd"], x["vd"], x["dout"], scale, True)
+    got = oracle.backward_given_out(x["q"], x["k"], x["v"], x["kd"], x["vd"], x["dout"],
+                                    ref["out"], scale, True)
+    for n in ("dq", "dk", "dv", "dkd", "dvd"):
+        np.testing.assert_allclose(got[n], ref[n], rtol=0, atol=1e-13)
+
+
+def test_backward_given_out_shifts_only_the_row_terms():
+    """With out' = out + delta, D' = <dO, out'> replaces D.  The value gradients dv, dvd do
+    not involve D; and since a row's dS then sums to D - D' instead of zero, the sum over
+    all keys (sequence and depth) of dk + dkd equals scale * sum_r (D_r - D'_r) q_r per KV
+    group -- zero for the exact out."""
+    B, T, Hq, Hkv, d, L = 1, 9, 4, 2, 6, 2
+    x = rand_problem(B=B, T=T, Hq=Hq, Hkv=Hkv, d=d, L=L, seed=42)
+    scale = 0.4
+    ref = oracle.backward(x["q"], x["k"], x["v"], x["kd"], x["vd"], x["dout"], scale, True)
+    g = torch.Generator().manual_seed(43)
+    delta = 1e-3 * torch.randn(B, Hq, T, d, generator=g, dtype=torch.float64).numpy()
+    got = oracle.backward_given_out(x["q"], x["k"], x["v"], x["kd"], x["vd"], x["dout"],
+                                    ref["out"] + delta, scale, True)
+    np.testing.assert_allclose(got["dv"], ref["dv"], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(got["dvd"], ref["dvd"], rtol=0, atol=1e-13)
+    dO, q = x["dout"].numpy(), x["q"].numpy()
+    dD = -(dO * delta).sum(-1)                                   # D - D'  [B,Hq,T]
+    G = Hq // Hkv
+    expect = scale * np.einsum("bht,bhtc->bhc", dD, q).reshape(B, Hkv, G, d).sum(2)
+    total = got["dk"].sum(2) + got["dkd"].sum(axis=(2, 3))
+    np.testing.assert_allclose(total, expect, rtol=1e-9, atol=1e-13)
+    assert np.abs(ref["dk"].sum(2) + ref["dkd"].sum(axis=(2, 3))).max() < 1e-12
