@@ -47,7 +47,7 @@ KERNEL_SOURCES = [os.path.join(ROOT, "depth_aware_attention_b200", "csrc", f)
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["moda", "reference"], default="moda")
     ap.add_argument("--workload", default="long-64k", choices=sorted(workloads.CONFIGS))
@@ -120,6 +120,12 @@ class ClockSampler:
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
+    def wait_first(self, timeout=5.0):
+        """Block until the first sample arrived, so the timed region is covered."""
+        t0 = time.time()
+        while self.proc is not None and not self.lines and time.time() - t0 < timeout:
+            time.sleep(0.05)
+
     def __exit__(self, *exc):
         if self.proc is not None:
             self.proc.terminate()
@@ -172,16 +178,57 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """Max of a per-rank scalar over all ranks (the slowest rank's time sets the job's)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_value(step_flops_per_rank, world, ms_max):
+    """Whole-job throughput in TFLOP/s: every rank runs one replica of the step, so the
+    job does world x the step's FLOPs in the slowest rank's time."""
+    return step_flops_per_rank * world / (ms_max * 1e-3) / 1e12
 
 
 def step_flops(cfg, fwd_only):
     f = workloads.forward_flops(**cfg)
     return f if fwd_only else f * (1.0 + BWD_FLOP_FACTOR)
+
+
+def kernel_roofline(name, cfg, avg_ms, pk, workload):
+    """Roofline entry for one kernel: algorithmic work per launch over its average
+    CUDA-event duration, against the measured sustained peak (every kernel here runs
+    inside a step of back-to-back launches)."""
+    B, Hq, Hkv, T, L, d = (cfg[n] for n in ("B", "Hq", "Hkv", "T", "L", "d"))
+    rows = B * Hq * T
+    if name == "moda_fwd_kernel":
+        bound, work = "tensor", workloads.forward_flops(**cfg)
+        what = "4*B*Hq*d*(T^2/2 + T*L) FLOPs"
+    elif name == "moda_bwd_seq_kernel":
+        bound, work = "tensor", BWD_FLOP_FACTOR * 4.0 * B * Hq * d * T * T / 2.0
+        what = "2.5 x 4*B*Hq*d*T^2/2 FLOPs (sequence part of the backward)"
+    elif name == "moda_bwd_depth_kernel":
+        bound = "hbm"
+        work = (2 * workloads.depth_bytes(**cfg)           # kd, vd read; dkd, dvd written
+                + 3 * rows * d * 2 + rows * d * 4 + rows * 8)  # q, dout, out; dq acc; lse, D
+        what = "bytes: kd+vd read, dkd+dvd written, q/dout/out read, fp32 dq written, lse/D"
+    else:
+        bound, work = "hbm", rows * d * (4 + 2)
+        what = "bytes: fp32 dq read, bf16 dq written"
+    if bound == "tensor":
+        achieved, peak, unit = work / (avg_ms * 1e-3) / 1e12, pk["bf16_sustained"], "TFLOP/s"
+        peak_kind = f"{pk['source']} bf16 dense, sustained"
+    else:
+        achieved, peak, unit = work / (avg_ms * 1e-3) / 1e9, pk["hbm"], "GB/s"
+        peak_kind = f"{pk['source']} HBM copy bandwidth"
+    return {"kernel": name, "bound": bound, "achieved": round(achieved, 1), "peak": peak,
+            "unit": unit, "frac": round(achieved / peak, 4),
+            "traffic": recorded_traffic(name, workload), "peak_kind": peak_kind,
+            "algorithmic_work_per_launch": work, "work_counted": what,
+            "avg_launch_ms": round(avg_ms, 4)}
 
 
 # ----------------------------------------------------------------------------- GPU arm
@@ -205,19 +252,32 @@ def run_moda(args, world, rank, local):
                  dkd=torch.empty_like(kd) if L else None,
                  dvd=torch.empty_like(vd) if L else None)
     stream = torch.cuda.current_stream(dev)
-    fwd_events = []
+    # Every launch of the step is bracketed by CUDA events on the launching stream: the
+    # forward kernel, then the backward's three stages (row terms + depth part, sequence
+    # part, dq convert), each launched on its own through moda_backward_stages.
+    names = ["moda_fwd_kernel"] + ([] if args.fwd_only else
+                                   ["moda_bwd_depth_kernel", "moda_bwd_seq_kernel",
+                                    "moda_dq_convert_kernel"])
+    events = {n: [] for n in names}
+
+    def timed(name, fn, record):
+        if not record:
+            fn()
+            return
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        events[name].append((e0, e1))
 
     def step(record=False):
-        if record:
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-        moda.forward(q, k, v, kd, vd, scale, True, out=out, lse=lse)
-        if record:
-            e1.record(stream)
-            fwd_events.append((e0, e1))
+        timed("moda_fwd_kernel",
+              lambda: moda.forward(q, k, v, kd, vd, scale, True, out=out, lse=lse), record)
         if not args.fwd_only:
-            moda.backward(q, k, v, kd, vd, out, lse, dout, scale, True, workspace=ws,
-                          grads=grads)
+            for name, stage in zip(names[1:], (1, 2, 4)):
+                timed(name, lambda st=stage: moda.backward(
+                    q, k, v, kd, vd, out, lse, dout, scale, True, workspace=ws, grads=grads,
+                    stages=st), record)
 
     for _ in range(args.warmup):
         step()
@@ -228,6 +288,7 @@ def run_moda(args, world, rank, local):
     torch.cuda.synchronize(dev)
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clocks:
+        clocks.wait_first()
         t_start.record(stream)
         for _ in range(args.steps):
             step(record=True)
@@ -237,22 +298,14 @@ def run_moda(args, world, rank, local):
     moda.check_device_errors()
     ms_local = t_start.elapsed_time(t_end) / args.steps
     ms = max_over_ranks(ms_local, world)
-    flops = step_flops(cfg, args.fwd_only)
-    value = flops * world / (ms * 1e-3) / 1e12
-    fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in fwd_events)
-    launches_per_step = 1 if args.fwd_only else 1 + moda.BACKWARD_LAUNCHES
+    value = job_value(step_flops(cfg, args.fwd_only), world, ms)
+    launches_per_step = len(names)
+    kernel_ms = {n: statistics.mean(a.elapsed_time(b) for a, b in ev) for n, ev in events.items()}
 
     pk = peaks()
     fwd_flops = workloads.forward_flops(**cfg)
-    fwd_tflops = fwd_flops / (fwd_ms * 1e-3) / 1e12
-    traffic = recorded_traffic("moda_fwd_kernel", args.workload)
-    roofline = {"kernel": "moda_fwd_kernel", "bound": "tensor", "achieved": round(fwd_tflops, 1),
-                "peak": pk["bf16_sustained"], "unit": "TFLOP/s",
-                "frac": round(fwd_tflops / pk["bf16_sustained"], 4), "traffic": traffic,
-                "peak_kind": f"{pk['source']} bf16 dense, sustained (kernel timed inside a "
-                             "long step)",
-                "algorithmic_flops_per_launch": fwd_flops,
-                "avg_launch_ms": round(fwd_ms, 4)}
+    dominant = max(kernel_ms, key=kernel_ms.get)
+    roofline = kernel_roofline(dominant, cfg, kernel_ms[dominant], pk, args.workload)
 
     # Extras the metric names: the L=0 causal ratio and the depth stream's HBM rate.
     extras = {}
@@ -293,6 +346,7 @@ def run_moda(args, world, rank, local):
 
     del x, q, k, v, kd, vd, dout, out, lse, ws, grads
     torch.cuda.empty_cache()
+    extras["kernels_ms"] = {n: round(t, 4) for n, t in kernel_ms.items()}
     return dict(ms=ms, value=value, clocks=clocks.summary(), roofline=roofline,
                 launches=launches_per_step * args.steps, extras=extras, e2e=e2e)
 
@@ -342,7 +396,7 @@ def run_e2e(args, moda, cfg, x, scale, dev, stream, world):
     torch.cuda.synchronize(dev)
     barrier(world)
     ms = max_over_ranks(e0.elapsed_time(e1) / steps, world)
-    value = step_flops(cfg, args.fwd_only) * world / (ms * 1e-3) / 1e12
+    value = job_value(step_flops(cfg, args.fwd_only), world, ms)
     del host, dbuf, out_h, lse_h, res_h
     return {"value": round(value, 2), "unit": UNIT, "ms_per_step": round(ms, 3),
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}

@@ -24,12 +24,13 @@ MODA_ERR_CUDA = 3
 MODA_ERR_TIMEOUT = 4
 MODA_ERR_INTERNAL = 5
 
-# Kernel launches one moda_backward call makes (row terms + depth, sequence, dQ convert).
+# Kernel launches one moda_backward call makes (row terms + depth, sequence, dQ convert),
+# one per stage of moda_backward_stages.
 BACKWARD_LAUNCHES = 3
 
 # Every symbol include/moda.h declares (checked by the ABI tests).
 EXPORTED = ("moda_forward", "moda_backward", "moda_backward_workspace_size",
-            "moda_backward_noalloc", "moda_check_device_errors", "moda_status_string",
+            "moda_backward_stages", "moda_backward_noalloc", "moda_check_device_errors", "moda_status_string",
             "moda_last_error_message")
 
 
@@ -52,6 +53,8 @@ def _load():
     lib.moda_backward_workspace_size.restype = S
     lib.moda_backward.argtypes = [P] * 14 + [S] + [I] * 6 + [F, I, P]
     lib.moda_backward.restype = I
+    lib.moda_backward_stages.argtypes = [P] * 14 + [S] + [I] * 6 + [F, I, ctypes.c_uint, P]
+    lib.moda_backward_stages.restype = I
     lib.moda_backward_noalloc.argtypes = [P] * 13 + [I] * 6 + [F, I, P]
     lib.moda_backward_noalloc.restype = I
     lib.moda_check_device_errors.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
@@ -96,6 +99,13 @@ def moda_backward_noalloc(q, k, v, kd, vd, out, lse, dout, dq, dk, dv, dkd, dvd,
     """The backward with library-owned static scratch (no workspace argument)."""
     return lib.moda_backward_noalloc(q, k, v, kd, vd, out, lse, dout, dq, dk, dv, dkd, dvd, B,
                                      Hq, Hkv, T, L, d, float(scale), int(causal), stream)
+
+
+def moda_backward_stages(q, k, v, kd, vd, out, lse, dout, dq, dk, dv, dkd, dvd, workspace,
+                         workspace_bytes, B, Hq, Hkv, T, L, d, scale, causal, stages, stream):
+    return lib.moda_backward_stages(q, k, v, kd, vd, out, lse, dout, dq, dk, dv, dkd, dvd,
+                                    workspace, workspace_bytes, B, Hq, Hkv, T, L, d,
+                                    float(scale), int(causal), int(stages), stream)
 
 
 def moda_backward_workspace_size(B, Hq, Hkv, T, L, d):
@@ -152,12 +162,14 @@ def forward(q, k, v, kd=None, vd=None, scale=None, causal=True, out=None, lse=No
 
 
 def backward(q, k, v, kd, vd, out, lse, dout, scale=None, causal=True, workspace=None,
-             grads=None):
+             grads=None, stages=7):
     """MoDA backward on the current CUDA stream.  Returns dict(dq, dk, dv, dkd, dvd).
 
     ``out``/``lse`` are the forward's results for the same inputs.  ``workspace`` (uint8
     CUDA tensor of at least moda_backward_workspace_size bytes) and ``grads`` (a dict of
     preallocated gradient tensors) are optional; missing ones are allocated with torch.
+    ``stages`` (bit mask 1 | 2 | 4, see moda_backward_stages) runs part of the backward;
+    the default runs all of it (moda_backward).
     """
     import torch
     B, Hq, Hkv, T, L, d = _dims(q, k, kd)
@@ -179,13 +191,17 @@ def backward(q, k, v, kd, vd, out, lse, dout, scale=None, causal=True, workspace
         g["dvd"] = torch.empty_like(vd)
     if not L:
         g["dkd"] = g["dvd"] = None
-    st = lib.moda_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(kd) if L else None,
-                           _ptr(vd) if L else None, _ptr(out), _ptr(lse), _ptr(dout),
-                           _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dkd"]),
-                           _ptr(g["dvd"]), _ptr(workspace),
-                           workspace.numel() * workspace.element_size(), B, Hq, Hkv, T, L, d,
-                           float(scale), int(bool(causal)), _stream_handle(q.device))
-    _check(st, "moda_backward")
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(kd) if L else None, _ptr(vd) if L else None,
+            _ptr(out), _ptr(lse), _ptr(dout), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]),
+            _ptr(g["dkd"]), _ptr(g["dvd"]), _ptr(workspace),
+            workspace.numel() * workspace.element_size(), B, Hq, Hkv, T, L, d, float(scale),
+            int(bool(causal)))
+    if stages == 7:
+        st = lib.moda_backward(*args, _stream_handle(q.device))
+        _check(st, "moda_backward")
+    else:
+        st = lib.moda_backward_stages(*args, int(stages), _stream_handle(q.device))
+        _check(st, "moda_backward_stages")
     return g
 
 

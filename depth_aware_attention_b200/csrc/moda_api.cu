@@ -149,12 +149,16 @@ size_t moda_backward_workspace_size(int B, int Hq, int Hkv, int T, int L, int d)
   return moda::backward_workspace_bytes(p);
 }
 
-moda_status_t moda_backward(const void* q, const void* k, const void* v, const void* kd,
-                            const void* vd, const void* out, const float* lse,
-                            const void* dout, void* dq, void* dk, void* dv, void* dkd,
-                            void* dvd, void* workspace, size_t workspace_bytes, int B,
-                            int Hq, int Hkv, int T, int L, int d, float scale, int causal,
-                            moda_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+moda_status_t backward_entry(const void* q, const void* k, const void* v, const void* kd,
+                             const void* vd, const void* out, const float* lse,
+                             const void* dout, void* dq, void* dk, void* dv, void* dkd,
+                             void* dvd, void* workspace, size_t workspace_bytes, int B,
+                             int Hq, int Hkv, int T, int L, int d, float scale, int causal,
+                             unsigned stages, moda_stream_t stream) {
   g_msg[0] = 0;
   moda_status_t s = check_sizes(B, Hq, Hkv, T, L, d);
   if (s != MODA_OK) return s;
@@ -197,13 +201,43 @@ moda_status_t moda_backward(const void* q, const void* k, const void* v, const v
   if (!enc) return fail(MODA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
   const char* why = "";
   cudaError_t e = moda::launch_backward(p, q, k, v, kd, vd, out, lse, dout, dq, dk, dv, dkd,
-                                        dvd, workspace, enc,
+                                        dvd, workspace, stages, enc,
                                         static_cast<cudaStream_t>(stream), &why);
   if (e != cudaSuccess) {
     snprintf(g_msg, sizeof(g_msg), "%s: %s", why, cudaGetErrorString(e));
     return MODA_ERR_CUDA;
   }
   return MODA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+moda_status_t moda_backward(const void* q, const void* k, const void* v, const void* kd,
+                            const void* vd, const void* out, const float* lse,
+                            const void* dout, void* dq, void* dk, void* dv, void* dkd,
+                            void* dvd, void* workspace, size_t workspace_bytes, int B,
+                            int Hq, int Hkv, int T, int L, int d, float scale, int causal,
+                            moda_stream_t stream) {
+  return backward_entry(q, k, v, kd, vd, out, lse, dout, dq, dk, dv, dkd, dvd, workspace,
+                        workspace_bytes, B, Hq, Hkv, T, L, d, scale, causal, moda::kStagesAll,
+                        stream);
+}
+
+moda_status_t moda_backward_stages(const void* q, const void* k, const void* v,
+                                   const void* kd, const void* vd, const void* out,
+                                   const float* lse, const void* dout, void* dq, void* dk,
+                                   void* dv, void* dkd, void* dvd, void* workspace,
+                                   size_t workspace_bytes, int B, int Hq, int Hkv, int T,
+                                   int L, int d, float scale, int causal, unsigned stages,
+                                   moda_stream_t stream) {
+  if (stages == 0 || (stages & ~moda::kStagesAll)) {
+    g_msg[0] = 0;
+    return fail(MODA_ERR_INVALID_ARGUMENT, "stages must be a non-empty subset of {1, 2, 4}");
+  }
+  return backward_entry(q, k, v, kd, vd, out, lse, dout, dq, dk, dv, dkd, dvd, workspace,
+                        workspace_bytes, B, Hq, Hkv, T, L, d, scale, causal, stages, stream);
 }
 
 moda_status_t moda_check_device_errors(moda_stream_t stream, uint32_t* flags) {

@@ -574,7 +574,8 @@ cudaError_t launch_backward_d(const Problem& p, const void* q, const void* k, co
                               const void* kd, const void* vd, const void* out,
                               const float* lse, const void* dout, void* dq, void* dk,
                               void* dv, void* dkd, void* dvd, void* workspace,
-                              EncodeTiledFn encode, cudaStream_t stream, const char** why) {
+                              unsigned stages, EncodeTiledFn encode, cudaStream_t stream,
+                              const char** why) {
   const TileGeom tg = tile_geom(p);
   const long long rows = (long long)p.B * p.Hq * p.T;
   float* dqacc = static_cast<float*>(workspace);
@@ -598,18 +599,21 @@ cudaError_t launch_backward_d(const Problem& p, const void* q, const void* k, co
   da.G = p.G;
   da.scale = p.scale;
   da.scale_log2 = p.scale * kLog2eBwd;
-  cudaError_t e;
-  if (p.G <= 1)
-    e = launch_depth<D, 1>(da, stream, why);
-  else if (p.G <= 2)
-    e = launch_depth<D, 2>(da, stream, why);
-  else if (p.G <= 4)
-    e = launch_depth<D, 4>(da, stream, why);
-  else if (p.G <= 8)
-    e = launch_depth<D, 8>(da, stream, why);
-  else
-    e = launch_depth<D, 16>(da, stream, why);
-  if (e != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
+  if (stages & kStageDepth) {
+    if (p.G <= 1)
+      e = launch_depth<D, 1>(da, stream, why);
+    else if (p.G <= 2)
+      e = launch_depth<D, 2>(da, stream, why);
+    else if (p.G <= 4)
+      e = launch_depth<D, 4>(da, stream, why);
+    else if (p.G <= 8)
+      e = launch_depth<D, 8>(da, stream, why);
+    else
+      e = launch_depth<D, 16>(da, stream, why);
+    if (e != cudaSuccess) return e;
+  }
+  if (!(stages & (kStageSeq | kStageConvert))) return cudaSuccess;
 
   // 2. sequence part
   const cuuint64_t E = 2;
@@ -658,7 +662,8 @@ cudaError_t launch_backward_d(const Problem& p, const void* q, const void* k, co
     return e;
   }
   const int nkb = (p.T + 127) / 128;
-  moda_bwd_seq_kernel<D><<<unsigned(BG) * nkb, kSeqThreads, SeqCfg<D>::kSmemBytes, stream>>>(
+  if (stages & kStageSeq)
+    moda_bwd_seq_kernel<D><<<unsigned(BG) * nkb, kSeqThreads, SeqCfg<D>::kSmemBytes, stream>>>(
       mQ, mDO, mK, mV, sa);
   e = cudaGetLastError();
   if (e != cudaSuccess) {
@@ -667,6 +672,7 @@ cudaError_t launch_backward_d(const Problem& p, const void* q, const void* k, co
   }
 
   // 3. dq (bf16)
+  if (!(stages & kStageConvert)) return cudaSuccess;
   const long long n8 = rows * D / 8;
   long long blocks = (n8 + 255) / 256;
   if (blocks > 8LL * sm_count()) blocks = 8LL * sm_count();
@@ -687,13 +693,13 @@ size_t backward_workspace_bytes(const Problem& p) {
 cudaError_t launch_backward(const Problem& p, const void* q, const void* k, const void* v,
                             const void* kd, const void* vd, const void* out, const float* lse,
                             const void* dout, void* dq, void* dk, void* dv, void* dkd,
-                            void* dvd, void* workspace, EncodeTiledFn encode,
-                            cudaStream_t stream, const char** why) {
+                            void* dvd, void* workspace, unsigned stages,
+                            EncodeTiledFn encode, cudaStream_t stream, const char** why) {
   if (p.d == 128)
     return launch_backward_d<128>(p, q, k, v, kd, vd, out, lse, dout, dq, dk, dv, dkd, dvd,
-                                  workspace, encode, stream, why);
+                                  workspace, stages, encode, stream, why);
   return launch_backward_d<64>(p, q, k, v, kd, vd, out, lse, dout, dq, dk, dv, dkd, dvd,
-                               workspace, encode, stream, why);
+                               workspace, stages, encode, stream, why);
 }
 
 }  // namespace moda

@@ -6,25 +6,26 @@
 // logits of the row's own-token depth block and of every visible causal sequence block
 // before the single normalisation at the end.
 //
-// One CTA owns one query tile of 128 rows = TQ tokens x G heads of one KV group
-// (token-major), so each K/V block and each depth chunk it loads serves all G heads of
-// the group ("group-aware") and the tile touches only its own tokens' depth rows
-// (TQ x L of them -- "chunk-aware"), read once from HBM.
+// One CTA owns a PAIR of adjacent query tiles.  A tile is 128 rows = TQ tokens x the G
+// heads of one KV group (token-major), so each K/V block and depth chunk loaded serves all
+// G heads of the group ("group-aware"), and a tile reads only its own tokens' TQ x L depth
+// rows ("chunk-aware"), each byte once.  Both tiles consume every K/V block the CTA loads.
 //
-// Warp roles (224 threads):
-//   warps 0-3  softmax/depth/epilogue: thread r owns tile row r (TMEM lane r).
-//              1. depth fold: logits q.kd and the running sums over the tile's depth
-//                 chunks on CUDA cores, accumulator written into TMEM as O's start;
-//              2. per sequence block: S row from TMEM -> mask -> exp2 -> P (bf16) back
-//                 into TMEM over S; rescales O only when the row max grows by > 2^8;
-//              3. epilogue: O / l -> bf16 out, lse = ln(sum exp).
-//   warp 4     TMA producer: Q tile, then the K/V blocks through the K/V ring.
-//   warp 6     TMA producer: the tile's depth chunks (kd, vd) through the depth ring.
-//              Each ring has exactly one consumer (tensor cores / softmax warps), which
-//              waits on every stage use in order, so the parity waits are unambiguous.
-//   warp 5     tcgen05 issuer: S = Q K^T (both operands in shared memory) and
-//              O += P V (P from tensor memory, V in shared memory), fp32 in TMEM.
-// TMEM columns: S/P double buffer at [0,128) and [128,256), O at [256, 256+D).
+// Warp roles (320 threads):
+//   warps 0-3 / 4-7  tile 0 / tile 1 compute warps: thread r owns row r of its tile (TMEM
+//            lane r).  First the depth fold: logits q.kd on CUDA cores from the tile's
+//            depth chunks, folded into (m, l) with the P.vd sums accumulated in registers
+//            and stored into TMEM as O's starting value.  Then per sequence block: S row
+//            from TMEM -> mask -> exp2 -> P (bf16) back into TMEM over S; O is rescaled
+//            only when the row max grows by more than 2^8.  Last the epilogue.
+//   warp 8   TMA producer: lane 0 streams the Q tiles and the K/V blocks through the K/V
+//            ring; lanes 1 and 2 stream tile 0's and tile 1's depth chunks through their
+//            own depth rings.  Every ring has exactly one in-order consumer.
+//   warp 9   tcgen05 issuer, in the order S0(0) S1(0) { PV0(j) S0(j+1) PV1(j) S1(j+1) }:
+//            while one tile's warps turn S into P, the tensor cores work for the other
+//            tile.  Because S_t(j+1) is issued after PV_t(j), a tile's warps that have
+//            seen S_t(j+1) know PV_t(j) has finished, so rescaling O_t needs no extra wait.
+// TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -44,36 +45,37 @@ constexpr int kRegion = 16384;     // one 128-row x 128-byte swizzled region
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only past 256x
-constexpr int kFwdThreads = 224;           // 7 warps, roles below
+constexpr int kFwdThreads = 320;
 
 template <int D>
 struct FwdCfg {
-  static constexpr int kRegions = D / 64;                 // 64-column swizzled regions
-  static constexpr int kTileBytes = kRegions * kRegion;   // Q tile or one ring stage
-  static constexpr int kKV = (D == 128) ? 4 : 6;          // K/V ring stages
-  static constexpr int kDS = (D == 128) ? 2 : 4;          // depth ring stages
-  static constexpr int kBarOff = kTileBytes * (1 + kKV + kDS);
-  static constexpr int kSmemBytes = 1024 + kBarOff + 256;
+  static constexpr int kRegions = D / 64;                // 64-column swizzled regions
+  static constexpr int kTileBytes = kRegions * kRegion;  // one Q tile / one K or V block
+  static constexpr int kKV = (D == 128) ? 3 : 4;         // K/V ring stages
+  static constexpr int kDS = (D == 128) ? 2 : 3;         // stages per depth ring (16 KB each)
+  static constexpr int kOffQ = 0;                        // two Q tiles
+  static constexpr int kOffKV = 2 * kTileBytes;
+  static constexpr int kOffD = kOffKV + kKV * kTileBytes;  // two depth rings
+  static constexpr int kBarOff = kOffD + 2 * kDS * kRegion;
+  static constexpr int kSmemBytes = 1024 + kBarOff + 512;
 };
 
 struct FwdArgs {
   __nv_bfloat16* out;
   float* lse;
-  int B, Hq, Hkv, T, L, G, TQ, JC, nqt, causal;
+  int B, Hq, Hkv, T, L, G, TQ, JC, nqt, npairs, causal;
   float scale_log2;
 };
 
-// Shared-memory barrier block (after the tiles).
 struct Bars {
   uint64_t q_full;
-  uint64_t full[6];    // K/V ring: data landed
-  uint64_t empty[6];   // K/V ring: stage released by the tensor cores
-  uint64_t dfull[4];   // depth ring: data landed
-  uint64_t dempty[4];  // depth ring: stage released by the softmax warps
-  uint64_t s_full[2];
-  uint64_t p_full[2];
-  uint64_t o_done;
-  uint64_t o_final;
+  uint64_t full[4];       // K/V ring: data landed
+  uint64_t empty[4];      // K/V ring: stage released by the tensor cores
+  uint64_t dfull[2][3];   // depth ring of tile t: data landed
+  uint64_t dempty[2][3];  // depth ring of tile t: stage released by tile t's warps
+  uint64_t s_full[2];     // S_t(j) in TMEM
+  uint64_t p_full[2];     // P_t(j) in TMEM (and O_t rescaled)
+  uint64_t o_final[2];    // last PV_t done
   uint32_t tmem_base;
   int abort;
 };
@@ -103,25 +105,25 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const uint32_t sQ = smem_u32(smem);
-  const uint32_t sRing = sQ + Cfg::kTileBytes;               // K/V ring
-  const uint32_t sDRing = sRing + NKV * Cfg::kTileBytes;      // depth ring
+  const uint32_t s0 = smem_u32(smem);
+  auto sQ = [&](int t) { return s0 + Cfg::kOffQ + uint32_t(t) * Cfg::kTileBytes; };
+  auto sKV = [&](int s) { return s0 + Cfg::kOffKV + uint32_t(s) * Cfg::kTileBytes; };
+  auto sDS = [&](int t, int s) { return s0 + Cfg::kOffD + uint32_t(t * NDS + s) * kRegion; };
   Bars* bars = reinterpret_cast<Bars*>(smem + Cfg::kBarOff);
   volatile int* abort_flag = &bars->abort;
+  auto bar = [&](uint64_t& b) { return smem_u32(&b); };
 
   const int warp = threadIdx.x >> 5;
   const int nbg = a.B * a.Hkv;
   const int bg = blockIdx.x % nbg;
-  const int qt = a.nqt - 1 - blockIdx.x / nbg;  // heaviest (latest) tiles first
-  const int t0 = qt * a.TQ;
-  const int kv_end = a.causal ? min(a.T, t0 + a.TQ) : a.T;
-  const int NB = (kv_end + kBN - 1) / kBN;
+  const int pair = a.npairs - 1 - blockIdx.x / nbg;  // heaviest (latest) pairs first
+  const int tq0 = 2 * pair * a.TQ, tq1 = tq0 + a.TQ;  // first token of tile 0 / tile 1
+  const int NB0 = ((a.causal ? min(a.T, tq0 + a.TQ) : a.T) + kBN - 1) / kBN;
+  // NB0 <= NB1; a tile 1 past the end of the sequence is computed but never stored
+  const int NB1 = tq1 >= a.T ? NB0 : ((a.causal ? min(a.T, tq1 + a.TQ) : a.T) + kBN - 1) / kBN;
   const int NC = a.L > 0 ? (a.L + a.JC - 1) / a.JC : 0;
   const bool has_depth = NC > 0;
-
-  auto bar = [&](uint64_t& b) { return smem_u32(&b); };
-  auto stage_addr = [&](int s) { return sRing + uint32_t(s) * Cfg::kTileBytes; };
-  auto dstage_addr = [&](int s) { return sDRing + uint32_t(s) * Cfg::kTileBytes; };
+  constexpr int kDUses = 2 * Cfg::kRegions;   // depth stage uses per chunk: kd, vd regions
 
   if (threadIdx.x == 0) {
     mbar_init(bar(bars->q_full), 1);
@@ -129,29 +131,30 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_init(bar(bars->full[s]), 1);
       mbar_init(bar(bars->empty[s]), 1);
     }
-    for (int s = 0; s < NDS; ++s) {
-      mbar_init(bar(bars->dfull[s]), 1);
-      mbar_init(bar(bars->dempty[s]), 1);
+    for (int t = 0; t < 2; ++t) {
+      for (int s = 0; s < NDS; ++s) {
+        mbar_init(bar(bars->dfull[t][s]), 1);
+        mbar_init(bar(bars->dempty[t][s]), 1);
+      }
+      mbar_init(bar(bars->s_full[t]), 1);
+      mbar_init(bar(bars->p_full[t]), 1);
+      mbar_init(bar(bars->o_final[t]), 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(bar(bars->s_full[i]), 1);
-      mbar_init(bar(bars->p_full[i]), 1);
-    }
-    mbar_init(bar(bars->o_done), 1);
-    mbar_init(bar(bars->o_final), 1);
     bars->abort = 0;
     fence_barrier_init();
   }
-  // Rows past TQ*G (when G does not divide 128) never receive TMA data: zero them so the
-  // tensor cores see finite values there.
+  // Rows past TQ*G (when G does not divide 128) never receive TMA data: zero them in both
+  // Q tiles so the tensor cores see finite values there.
   if (threadIdx.x < kBM && threadIdx.x >= a.TQ * a.G) {
-    for (int rg = 0; rg < Cfg::kRegions; ++rg) {
-      uint4* row = reinterpret_cast<uint4*>(smem + rg * kRegion + threadIdx.x * 128);
-      for (int c = 0; c < 8; ++c) row[c] = make_uint4(0, 0, 0, 0);
-    }
+    for (int t = 0; t < 2; ++t)
+      for (int rg = 0; rg < Cfg::kRegions; ++rg) {
+        uint4* row = reinterpret_cast<uint4*>(smem + Cfg::kOffQ + t * Cfg::kTileBytes +
+                                              rg * kRegion + threadIdx.x * 128);
+        for (int c = 0; c < 8; ++c) row[c] = make_uint4(0, 0, 0, 0);
+      }
     fence_proxy_async_smem();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(smem_u32(&bars->tmem_base), 512);
     tmem_relinquish();
   }
@@ -160,99 +163,122 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
-  if (warp == 4) {
-    // ------------------------------------------------ TMA producer: Q tile, K/V blocks
-    if (elect_one()) {
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer lanes
+    const int lane = threadIdx.x & 31;
+    if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      mbar_expect_tx(bar(bars->q_full), Cfg::kRegions * 128 * a.G * a.TQ);
-      for (int rg = 0; rg < Cfg::kRegions; ++rg)
-        tma_load_4d(sQ + rg * kRegion, &tmQ, bar(bars->q_full), rg * 64, 0, t0, bg);
-      for (int idx = 0; idx < 2 * NB; ++idx) {
+      mbar_expect_tx(bar(bars->q_full), 2 * Cfg::kRegions * 128 * a.G * a.TQ);
+      for (int t = 0; t < 2; ++t)
+        for (int rg = 0; rg < Cfg::kRegions; ++rg)
+          tma_load_4d(sQ(t) + rg * kRegion, &tmQ, bar(bars->q_full), rg * 64, 0,
+                      t ? tq1 : tq0, bg);
+      for (int idx = 0; idx < 2 * NB1; ++idx) {
         const int s = idx % NKV;
         if (idx >= NKV) mbar_wait(bar(bars->empty[s]), ((idx / NKV) - 1) & 1, abort_flag);
         const CUtensorMap* map = (idx & 1) ? &tmV : &tmK;
         mbar_expect_tx(bar(bars->full[s]), Cfg::kTileBytes);
         for (int rg = 0; rg < Cfg::kRegions; ++rg)
-          tma_load_3d(stage_addr(s) + rg * kRegion, map, bar(bars->full[s]), rg * 64,
+          tma_load_3d(sKV(s) + rg * kRegion, map, bar(bars->full[s]), rg * 64,
                       (idx >> 1) * kBN, bg);
       }
-    }
-    __syncwarp();
-  } else if (warp == 6) {
-    // ------------------------------------------------ TMA producer: depth chunks
-    // Chunk ci holds entries [ci*JC, ci*JC+JC) of the tile's TQ tokens, rows
-    // (token, entry) with the entry fastest: each token's entries are one contiguous
-    // run of the [B,Hkv,T,L,d] cache.
-    if (has_depth && elect_one()) {
-      tma_prefetch_desc(&tmKD);
-      tma_prefetch_desc(&tmVD);
-      const uint32_t dbytes = Cfg::kRegions * 128 * a.TQ * a.JC;
-      for (int idx = 0; idx < 2 * NC; ++idx) {
+    } else if ((lane == 1 || lane == 2) && has_depth) {
+      // Depth chunk ci of tile t: entries [ci*JC, ci*JC+JC) of the tile's TQ tokens as
+      // rows (token, entry), one 64-column region per stage: kd regions, then vd regions.
+      const int t = lane - 1;
+      if (t == 0) {
+        tma_prefetch_desc(&tmKD);
+        tma_prefetch_desc(&tmVD);
+      }
+      const uint32_t dbytes = 128u * a.TQ * a.JC;
+      for (int idx = 0; idx < NC * kDUses; ++idx) {
         const int s = idx % NDS;
-        if (idx >= NDS) mbar_wait(bar(bars->dempty[s]), ((idx / NDS) - 1) & 1, abort_flag);
-        const CUtensorMap* map = (idx & 1) ? &tmVD : &tmKD;
-        mbar_expect_tx(bar(bars->dfull[s]), dbytes);
-        for (int rg = 0; rg < Cfg::kRegions; ++rg)
-          tma_load_4d(dstage_addr(s) + rg * kRegion, map, bar(bars->dfull[s]), rg * 64,
-                      (idx >> 1) * a.JC, t0, bg);
+        if (idx >= NDS)
+          mbar_wait(bar(bars->dempty[t][s]), ((idx / NDS) - 1) & 1, abort_flag);
+        const int u = idx % kDUses;
+        const CUtensorMap* map = (u < Cfg::kRegions) ? &tmKD : &tmVD;
+        const int rg = u % Cfg::kRegions;
+        mbar_expect_tx(bar(bars->dfull[t][s]), dbytes);
+        tma_load_4d(sDS(t, s), map, bar(bars->dfull[t][s]), rg * 64, (idx / kDUses) * a.JC,
+                    t ? tq1 : tq0, bg);
       }
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------ tcgen05 issuer
     if (elect_one()) {
       constexpr uint32_t idesc_s = make_idesc_bf16(kBM, kBN, 0, 0);
       constexpr uint32_t idesc_o = make_idesc_bf16(kBM, D, 0, 1);
-      const uint32_t tO = tmem + 256;
       mbar_wait(bar(bars->q_full), 0, abort_flag);
-      auto issue_pv = [&](int j) {
-        mbar_wait(bar(bars->p_full[j & 1]), (j >> 1) & 1, abort_flag);
-        const int vidx = 2 * j + 1;
-        const int vs = vidx % NKV;
-        mbar_wait(bar(bars->full[vs]), (vidx / NKV) & 1, abort_flag);
+      auto wait_kv = [&](int idx) {
+        mbar_wait(bar(bars->full[idx % NKV]), (idx / NKV) & 1, abort_flag);
         tc_fence_after();
-        const uint32_t vbase = stage_addr(vs);
-#pragma unroll
-        for (int ks = 0; ks < kBN / 16; ++ks) {
-          const uint64_t bdesc = make_sdesc_sw128(vbase + ks * 2048, kRegion, 1024);
-          mma_ts(tO, tmem + (j & 1) * 128 + ks * 8, bdesc, idesc_o,
-                 (ks > 0 || j > 0 || has_depth) ? 1u : 0u);
-        }
-        tc_commit(bar(bars->empty[vs]));
-        tc_commit(bar(bars->o_done));
-        if (j == NB - 1) tc_commit(bar(bars->o_final));
       };
-      for (int jb = 0; jb < NB; ++jb) {
-        const int kidx = 2 * jb;
-        const int ks_ = kidx % NKV;
-        mbar_wait(bar(bars->full[ks_]), (kidx / NKV) & 1, abort_flag);
-        tc_fence_after();
-        const uint32_t kbase = stage_addr(ks_);
+      auto issue_s = [&](int t, int j) {
+        const uint32_t kbase = sKV((2 * j) % NKV);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t off = (ks / 4) * kRegion + (ks % 4) * 32;
-          const uint64_t adesc = make_sdesc_sw128(sQ + off, 16, 1024);
-          const uint64_t bdesc = make_sdesc_sw128(kbase + off, 16, 1024);
-          mma_ss(tmem + (jb & 1) * 128, adesc, bdesc, idesc_s, ks > 0 ? 1u : 0u);
+          mma_ss(tmem + t * 128, make_sdesc_sw128(sQ(t) + off, 16, 1024),
+                 make_sdesc_sw128(kbase + off, 16, 1024), idesc_s, ks > 0 ? 1u : 0u);
         }
-        tc_commit(bar(bars->s_full[jb & 1]));
-        tc_commit(bar(bars->empty[ks_]));
-        if (jb >= 1) issue_pv(jb - 1);
+        tc_commit(bar(bars->s_full[t]));
+      };
+      auto issue_pv = [&](int t, int j) {
+        mbar_wait(bar(bars->p_full[t]), j & 1, abort_flag);
+        tc_fence_after();
+        const uint32_t vbase = sKV((2 * j + 1) % NKV);
+        const uint32_t tO = tmem + 256 + t * D;
+#pragma unroll
+        for (int ks = 0; ks < kBN / 16; ++ks)
+          mma_ts(tO, tmem + t * 128 + ks * 8,
+                 make_sdesc_sw128(vbase + ks * 2048, kRegion, 1024), idesc_o,
+                 (ks > 0 || j > 0 || has_depth) ? 1u : 0u);
+      };
+      wait_kv(0);
+      issue_s(0, 0);
+      issue_s(1, 0);
+      tc_commit(bar(bars->empty[0]));
+      for (int j = 0; j < NB1; ++j) {
+        wait_kv(2 * j + 1);
+        bool k_next_ready = false;
+        if (j < NB0) {
+          issue_pv(0, j);
+          if (j == NB0 - 1) tc_commit(bar(bars->o_final[0]));
+          if (j + 1 < NB0) {
+            wait_kv(2 * j + 2);
+            k_next_ready = true;
+            issue_s(0, j + 1);
+          }
+        }
+        issue_pv(1, j);
+        tc_commit(bar(bars->empty[(2 * j + 1) % NKV]));
+        if (j == NB1 - 1) tc_commit(bar(bars->o_final[1]));
+        if (j + 1 < NB1) {
+          if (!k_next_ready) wait_kv(2 * j + 2);
+          issue_s(1, j + 1);
+          tc_commit(bar(bars->empty[(2 * j + 2) % NKV]));
+        }
       }
-      issue_pv(NB - 1);
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ softmax warps 0-3
-    const int r = threadIdx.x;
+    // ------------------------------------------------------------ compute warps
+    const int tt = warp >> 2;                     // tile of this warpgroup
+    const int r = threadIdx.x & 127;              // tile row
     const int tok = r / a.G;
     const int hl = r - tok * a.G;
+    const int t0 = tt ? tq1 : tq0;
     const int t = t0 + tok;
     const bool valid = (tok < a.TQ) && (t < a.T);
-    const uint32_t lane_base = uint32_t(warp * 32) << 16;
-    const uint32_t tO = tmem + lane_base + 256;
+    const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_base + tt * 128;
+    const uint32_t tO = tmem + lane_base + 256 + tt * D;
+    const uint32_t q_base = sQ(tt);
+    const int NB = tt ? NB1 : NB0;
+    const uint32_t wg_bar = 1 + tt;               // named barrier of this warpgroup
     float m = -INFINITY, l = 0.f;
 
     mbar_wait(bar(bars->q_full), 0, abort_flag);
@@ -262,30 +288,34 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
       for (int c = 0; c < D; ++c) acc[c] = 0.f;
       const int tokc = tok < a.TQ ? tok : 0;  // padding rows read a valid row
+      int use = 0;
+      auto take = [&]() -> uint32_t {
+        const int s = use % NDS;
+        mbar_wait(bar(bars->dfull[tt][s]), (use / NDS) & 1, abort_flag);
+        return sDS(tt, s);
+      };
+      auto give = [&]() {
+        named_bar_sync(wg_bar, 128);
+        if (r == 0) mbar_arrive(bar(bars->dempty[tt][use % NDS]));
+        ++use;
+      };
       for (int ci = 0; ci < NC; ++ci) {
-        const int kidx = 2 * ci, vidx = 2 * ci + 1;
-        const int kst = kidx % NDS, vst = vidx % NDS;
         float y[kJCMax];
 #pragma unroll
         for (int jj = 0; jj < kJCMax; ++jj) y[jj] = 0.f;
-        mbar_wait(bar(bars->dfull[kst]), (kidx / NDS) & 1, abort_flag);
-        const uint32_t kb = dstage_addr(kst);
-#pragma unroll 2
-        for (int c8 = 0; c8 < D / 8; ++c8) {
-          const uint32_t reg = (c8 >> 3) * kRegion;
-          const uint4 qw = lds128(sQ + reg + sw128_off(r, c8 & 7));
-          float qf[8] = {bf16lo(qw.x), bf16hi(qw.x), bf16lo(qw.y), bf16hi(qw.y),
-                         bf16lo(qw.z), bf16hi(qw.z), bf16lo(qw.w), bf16hi(qw.w)};
 #pragma unroll
-          for (int jj = 0; jj < kJCMax; ++jj) {
-            if (jj < a.JC) {
-              const uint32_t row = tokc * a.JC + jj;
-              y[jj] += dot8(qf, lds128(kb + reg + sw128_off(row, c8 & 7)));
-            }
+        for (int rg = 0; rg < Cfg::kRegions; ++rg) {
+          const uint32_t kb = take();
+#pragma unroll 2
+          for (int c8 = 0; c8 < 8; ++c8) {
+            const uint4 qw = lds128(q_base + rg * kRegion + sw128_off(r, c8));
+#pragma unroll
+            for (int jj = 0; jj < kJCMax; ++jj)
+              if (jj < a.JC)
+                y[jj] = dot8_bf16(qw, lds128(kb + sw128_off(tokc * a.JC + jj, c8)), y[jj]);
           }
+          give();
         }
-        named_bar_sync(1, 128);
-        if (r == 0) mbar_arrive(bar(bars->dempty[kst]));
         // online update over this chunk's depth logits (log2 domain)
         float mx = -INFINITY;
 #pragma unroll
@@ -296,40 +326,32 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
         const float m_new = fmaxf(m, mx);
         const float alpha = ex2(m - m_new);
+        // The weights enter the P.vd sums as bf16, the same precision the sequence part's
+        // P takes into the tensor cores; l sums them unrounded, as for the sequence part.
         float ps = 0.f;
+        uint16_t pb[kJCMax];
 #pragma unroll
         for (int jj = 0; jj < kJCMax; ++jj) {
-          y[jj] = ex2(y[jj] - m_new);
-          ps += y[jj];
+          const float p = ex2(y[jj] - m_new);
+          pb[jj] = bf16_bits(p);
+          ps += p;
         }
         l = l * alpha + ps;
         m = m_new;
-        mbar_wait(bar(bars->dfull[vst]), (vidx / NDS) & 1, abort_flag);
-        const uint32_t vb = dstage_addr(vst);
 #pragma unroll
-        for (int c8 = 0; c8 < D / 8; ++c8) {
-          const uint32_t reg = (c8 >> 3) * kRegion;
+        for (int rg = 0; rg < Cfg::kRegions; ++rg) {
+          const uint32_t vb = take();
 #pragma unroll
-          for (int e = 0; e < 8; ++e) acc[c8 * 8 + e] *= alpha;
+          for (int c8 = 0; c8 < 8; ++c8) {
+            float(&ac)[8] = *reinterpret_cast<float(*)[8]>(acc + rg * 64 + c8 * 8);
 #pragma unroll
-          for (int jj = 0; jj < kJCMax; ++jj) {
-            if (jj < a.JC) {
-              const uint32_t row = tokc * a.JC + jj;
-              const uint4 w = lds128(vb + reg + sw128_off(row, c8 & 7));
-              const float p = y[jj];
-              acc[c8 * 8 + 0] = fmaf(p, bf16lo(w.x), acc[c8 * 8 + 0]);
-              acc[c8 * 8 + 1] = fmaf(p, bf16hi(w.x), acc[c8 * 8 + 1]);
-              acc[c8 * 8 + 2] = fmaf(p, bf16lo(w.y), acc[c8 * 8 + 2]);
-              acc[c8 * 8 + 3] = fmaf(p, bf16hi(w.y), acc[c8 * 8 + 3]);
-              acc[c8 * 8 + 4] = fmaf(p, bf16lo(w.z), acc[c8 * 8 + 4]);
-              acc[c8 * 8 + 5] = fmaf(p, bf16hi(w.z), acc[c8 * 8 + 5]);
-              acc[c8 * 8 + 6] = fmaf(p, bf16lo(w.w), acc[c8 * 8 + 6]);
-              acc[c8 * 8 + 7] = fmaf(p, bf16hi(w.w), acc[c8 * 8 + 7]);
-            }
+            for (int e = 0; e < 8; ++e) ac[e] *= alpha;
+#pragma unroll
+            for (int jj = 0; jj < kJCMax; ++jj)
+              if (jj < a.JC) axpy8_bf16(pb[jj], lds128(vb + sw128_off(tokc * a.JC + jj, c8)), ac);
           }
+          give();
         }
-        named_bar_sync(1, 128);
-        if (r == 0) mbar_arrive(bar(bars->dempty[vst]));
       }
       // depth accumulator becomes O's starting value
 #pragma unroll
@@ -345,9 +367,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     // ---- sequence blocks
     const int key_lim = a.causal ? t : a.T - 1;
     for (int jb = 0; jb < NB; ++jb) {
-      mbar_wait(bar(bars->s_full[jb & 1]), (jb >> 1) & 1, abort_flag);
+      mbar_wait(bar(bars->s_full[tt]), jb & 1, abort_flag);
       tc_fence_after();
-      const uint32_t tS = tmem + lane_base + (jb & 1) * 128;
       uint32_t s[kBN];
       tmem_ld32(tS + 0, &s[0]);
       tmem_ld32(tS + 32, &s[32]);
@@ -356,37 +377,44 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       tmem_wait_ld();
       const int kbase = jb * kBN;
       const bool need_mask = a.causal ? (kbase + kBN - 1 > t0) : (kbase + kBN > a.T);
-      float x[kBN];
+      // Row max on the raw scores (scale > 0 commutes with max); masked keys -> -inf.
       float mx = -INFINITY;
+      if (need_mask) {
 #pragma unroll
-      for (int c = 0; c < kBN; ++c) {
-        float v = __uint_as_float(s[c]) * a.scale_log2;
-        if (need_mask && kbase + c > key_lim) v = -INFINITY;
-        x[c] = v;
-        mx = fmaxf(mx, v);
+        for (int c = 0; c < kBN; ++c) {
+          if (kbase + c > key_lim) s[c] = __float_as_uint(-INFINITY);
+          mx = fmaxf(mx, __uint_as_float(s[c]));
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < kBN; ++c) mx = fmaxf(mx, __uint_as_float(s[c]));
       }
-      const float m_cand = fmaxf(m, mx);
+      const float m_cand = fmaxf(m, mx * a.scale_log2);
       const bool grow = m_cand > m + kRescaleThreshold;
       const float m_new = grow ? m_cand : m;
       const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
       const float alpha = ex2(m - m_use);
-      float ps = 0.f;
-      uint32_t pk[kBN / 2];
+      float ps0 = 0.f, ps1 = 0.f;
 #pragma unroll
-      for (int c = 0; c < kBN; c += 2) {
-        const float p0 = ex2(x[c] - m_use);
-        const float p1 = ex2(x[c + 1] - m_use);
-        ps += p0 + p1;
-        pk[c / 2] = pack_bf16x2(p0, p1);
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          // p = 2^(s*scale*log2e - m): one FFMA feeds each exp2
+          const float p0 = ex2(fmaf(__uint_as_float(s[half * 64 + c]), a.scale_log2, -m_use));
+          const float p1 = ex2(fmaf(__uint_as_float(s[half * 64 + c + 1]), a.scale_log2, -m_use));
+          ps0 += p0;
+          ps1 += p1;
+          pk[c / 2] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(tS + half * 32, pk);
       }
-      tmem_st32(tS + 0, &pk[0]);
-      tmem_st32(tS + 32, &pk[32]);
+      const float ps = ps0 + ps1;
       l = l * alpha + ps;
       m = m_new;
+      // O_t holds every PV_t issued so far (S_t(jb) was issued after PV_t(jb-1)).
       const bool has_o = has_depth || jb > 0;
       if (__any_sync(0xffffffffu, grow && has_o)) {
-        if (jb > 0) mbar_wait(bar(bars->o_done), (jb - 1) & 1, abort_flag);
-        tc_fence_after();
         const float f = grow ? alpha : 1.f;
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
@@ -400,12 +428,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       tmem_wait_st();
       tc_fence_before();
-      named_bar_sync(1, 128);
-      if (r == 0) mbar_arrive(bar(bars->p_full[jb & 1]));
+      named_bar_sync(wg_bar, 128);
+      if (r == 0) mbar_arrive(bar(bars->p_full[tt]));
     }
 
     // ---- epilogue
-    mbar_wait(bar(bars->o_final), 0, abort_flag);
+    mbar_wait(bar(bars->o_final[tt]), 0, abort_flag);
     tc_fence_after();
     const float inv_l = 1.f / l;
     const int h = (bg % a.Hkv) * a.G + hl;
@@ -438,13 +466,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
 }
 
-// Host-side tensor map helpers.
+// Host-side tensor map helper.
 bool make_map(EncodeTiledFn encode, CUtensorMap* map, const void* base, int rank,
               const cuuint64_t* dims, const cuuint64_t* strides_bytes,
               const cuuint32_t* box) {
@@ -514,6 +542,7 @@ cudaError_t launch_forward_d(const Problem& p, const void* q, const void* k, con
   args.TQ = tg.TQ;
   args.JC = tg.JC;
   args.nqt = tg.nqt;
+  args.npairs = (tg.nqt + 1) / 2;
   args.causal = p.causal;
   args.scale_log2 = p.scale * kLog2e;
 
@@ -526,8 +555,9 @@ cudaError_t launch_forward_d(const Problem& p, const void* q, const void* k, con
       return e;
     }
   }
-  const unsigned grid = unsigned(BG) * unsigned(tg.nqt);
-  moda_fwd_kernel<D><<<grid, kFwdThreads, Cfg::kSmemBytes, stream>>>(mQ, mK, mV, mKD, mVD, args);
+  const unsigned grid = unsigned(BG) * unsigned(args.npairs);
+  moda_fwd_kernel<D><<<grid, kFwdThreads, Cfg::kSmemBytes, stream>>>(mQ, mK, mV, mKD, mVD,
+                                                                      args);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) *why = "forward kernel launch failed";
   return e;

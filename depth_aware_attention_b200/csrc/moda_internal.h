@@ -49,7 +49,12 @@ cudaError_t launch_backward(const Problem& p, const void* q, const void* k, cons
                             const void* kd, const void* vd, const void* out,
                             const float* lse, const void* dout, void* dq, void* dk,
                             void* dv, void* dkd, void* dvd, void* workspace,
-                            EncodeTiledFn encode, cudaStream_t stream, const char** why);
+                            unsigned stages, EncodeTiledFn encode, cudaStream_t stream,
+                            const char** why);
+
+// Backward stages (bit mask): 1 row terms + depth part + dq accumulator initialisation,
+// 2 sequence part (adds to the dq accumulator), 4 dq conversion to bf16.
+constexpr unsigned kStageDepth = 1u, kStageSeq = 2u, kStageConvert = 4u, kStagesAll = 7u;
 
 size_t backward_workspace_bytes(const Problem& p);
 

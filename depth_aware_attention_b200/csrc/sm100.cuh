@@ -328,6 +328,43 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
       : "memory");
 }
 
+// acc + <a, b> over 8 bf16 pairs (a, b: 8 packed bf16 each) with the mixed-precision
+// fma.rn.f32.bf16 (bf16 sources, fp32 accumulate): the products of two bf16 are exact in
+// fp32, so this equals widening both to fp32 and using fp32 FMAs, without the unpacking.
+__device__ __forceinline__ float dot8_bf16(uint4 a, uint4 b, float acc) {
+  asm("{\n\t.reg .b16 a0,a1,a2,a3,a4,a5,a6,a7,b0,b1,b2,b3,b4,b5,b6,b7;\n\t"
+      "mov.b32 {a0,a1}, %1;\n\tmov.b32 {a2,a3}, %2;\n\t"
+      "mov.b32 {a4,a5}, %3;\n\tmov.b32 {a6,a7}, %4;\n\t"
+      "mov.b32 {b0,b1}, %5;\n\tmov.b32 {b2,b3}, %6;\n\t"
+      "mov.b32 {b4,b5}, %7;\n\tmov.b32 {b6,b7}, %8;\n\t"
+      "fma.rn.f32.bf16 %0, a0, b0, %0;\n\tfma.rn.f32.bf16 %0, a1, b1, %0;\n\t"
+      "fma.rn.f32.bf16 %0, a2, b2, %0;\n\tfma.rn.f32.bf16 %0, a3, b3, %0;\n\t"
+      "fma.rn.f32.bf16 %0, a4, b4, %0;\n\tfma.rn.f32.bf16 %0, a5, b5, %0;\n\t"
+      "fma.rn.f32.bf16 %0, a6, b6, %0;\n\tfma.rn.f32.bf16 %0, a7, b7, %0;\n\t}"
+      : "+f"(acc)
+      : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w));
+  return acc;
+}
+
+// acc[0..8) += p * v[0..8) with p (bf16 bits) and v (8 packed bf16) as bf16 sources and
+// fp32 accumulation (fma.rn.f32.bf16).
+__device__ __forceinline__ void axpy8_bf16(uint16_t p, uint4 v, float (&acc)[8]) {
+  asm("{\n\t.reg .b16 v0,v1,v2,v3,v4,v5,v6,v7;\n\t"
+      "mov.b32 {v0,v1}, %9;\n\tmov.b32 {v2,v3}, %10;\n\t"
+      "mov.b32 {v4,v5}, %11;\n\tmov.b32 {v6,v7}, %12;\n\t"
+      "fma.rn.f32.bf16 %0, v0, %8, %0;\n\tfma.rn.f32.bf16 %1, v1, %8, %1;\n\t"
+      "fma.rn.f32.bf16 %2, v2, %8, %2;\n\tfma.rn.f32.bf16 %3, v3, %8, %3;\n\t"
+      "fma.rn.f32.bf16 %4, v4, %8, %4;\n\tfma.rn.f32.bf16 %5, v5, %8, %5;\n\t"
+      "fma.rn.f32.bf16 %6, v6, %8, %6;\n\tfma.rn.f32.bf16 %7, v7, %8, %7;\n\t}"
+      : "+f"(acc[0]), "+f"(acc[1]), "+f"(acc[2]), "+f"(acc[3]), "+f"(acc[4]), "+f"(acc[5]),
+        "+f"(acc[6]), "+f"(acc[7])
+      : "h"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w));
+}
+
+__device__ __forceinline__ uint16_t bf16_bits(float x) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
+
 // Byte offset of 16-byte chunk `c` (0..7) of row `r` inside a 128B-swizzled region.
 __device__ __forceinline__ uint32_t sw128_off(uint32_t r, uint32_t c) {
   return r * 128u + ((c ^ (r & 7u)) << 4);

@@ -94,6 +94,26 @@ moda_status_t moda_backward(const void *q, const void *k, const void *v, const v
                             moda_stream_t stream);
 
 /*
+ * moda_backward split into its three launches, for callers that schedule or time them
+ * separately.  `stages` is a non-empty bit mask:
+ *   1  row terms D = <dout, out> (into the workspace), the depth gradients dkd and dvd,
+ *      and the depth share of dq, which initialises the workspace's fp32 dq accumulator;
+ *   2  the sequence part: dk and dv, plus the sequence share of dq added to the
+ *      accumulator (needs stage 1's workspace contents);
+ *   4  dq (bf16) from the accumulator (needs stages 1 and 2).
+ * Running 1, 2 and 4 in that order on one stream (with the same arguments and workspace)
+ * equals one moda_backward call; moda_backward is stages = 7.  Arguments, checks and
+ * errors are moda_backward's; an invalid mask gives MODA_ERR_INVALID_ARGUMENT.
+ */
+moda_status_t moda_backward_stages(const void *q, const void *k, const void *v,
+                                   const void *kd, const void *vd, const void *out,
+                                   const float *lse, const void *dout, void *dq, void *dk,
+                                   void *dv, void *dkd, void *dvd, void *workspace,
+                                   size_t workspace_bytes, int B, int Hq, int Hkv, int T,
+                                   int L, int d, float scale, int causal, unsigned stages,
+                                   moda_stream_t stream);
+
+/*
  * The backward of moda_backward for callers that cannot allocate device memory: those
  * whose device memory is owned by another allocator or by a fixed memory plan that hands
  * out only the tensors it planned, and those calling through a plain C binding with no

@@ -102,6 +102,13 @@ def test_backward_rejects_small_workspace_and_aliasing():
     assert st == moda.MODA_ERR_UNSUPPORTED
 
 
+@pytest.mark.parametrize("stages", [0, 8, 15])
+def test_backward_stages_rejects_bad_masks(stages):
+    args = [A * (i + 1) for i in range(13)] + [A * 64, 1 << 20, 1, 4, 2, 16, 2, 64, 0.125, 1,
+                                               stages, None]
+    assert moda.moda_backward_stages(*args) == moda.MODA_ERR_INVALID_ARGUMENT
+
+
 def test_binding_has_no_fallback():
     src = open(os.path.join(ROOT, "depth_aware_attention_b200", "__init__.py")).read()
     assert "oracle" not in src.lower().replace("no cpu", "")

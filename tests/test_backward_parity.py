@@ -4,9 +4,10 @@ The GPU backward takes the GPU forward's out (bf16) and lse (fp32); the oracle d
 its own fp64 forward.  Tolerances are those of parity_util: max-abs 1e-2 beyond the bf16 output's own rounding,
 mean-abs 1e-3, relative RMS 1e-2.
 
-Small problems are compared in full (all of dq, dk, dv, dkd, dvd).  The 16K-token
-forward+backward workload, in the launch configuration the benchmark times, is compared on
-token windows: for a window [t0, t0+nt) the oracle's dq, dkd and dvd are exact, and for the
+Small problems are compared in full (all of dq, dk, dv, dkd, dvd) against the oracle's
+backward given the GPU forward's bf16 out (the only out a backward receives).  The 16K-token
+forward+backward workload, in the launch configuration the benchmark times, is compared with
+the oracle's exact gradient on token windows: for a window [t0, t0+nt) the oracle's dq, dkd and dvd are exact, and for the
 window that ends at T its dk and dv are exact for every key s >= t0 (only tokens t >= s see
 key s under the causal mask).
 """
@@ -40,21 +41,29 @@ SMALL = [
 NAMES = ("dq", "dk", "dv", "dkd", "dvd")
 
 
-def run_gpu(x, scale, causal):
+def run_gpu(x, scale, causal, keep_out=False):
     out, lse = moda.forward(x["q"], x["k"], x["v"], x["kd"], x["vd"], scale, causal)
     g = moda.backward(x["q"], x["k"], x["v"], x["kd"], x["vd"], out, lse, x["dout"], scale,
                       causal)
     moda.check_device_errors()
+    if keep_out:
+        g["out"] = out
     return g
 
 
 @pytest.mark.parametrize("name,cfg,causal", SMALL, ids=[s[0] for s in SMALL])
 def test_backward_small_full(name, cfg, causal):
+    """All five gradients in full against the oracle's exact backward given the same inputs
+    as the GPU backward, including the forward's bf16 out: the backward's row terms
+    D = <dO, out> can only use that out (oracle.backward_given_out).  On these short
+    sequences a key collects gradient from up to G*T rows, entries reach 7, and the bf16
+    rounding of out alone moves them by up to 1e-2 through D."""
     x = gpu_inputs(cfg, seed_base=200 + SMALL.index((name, cfg, causal)), with_dout=True)
     scale = 1.0 / math.sqrt(cfg["d"])
-    g = run_gpu(x, scale, causal)
+    g = run_gpu(x, scale, causal, keep_out=True)
     w = window(x, 0, cfg["T"])
-    ref = oracle.backward(w["q"], w["k"], w["v"], w["kd"], w["vd"], w["dout"], scale, causal)
+    ref = oracle.backward_given_out(w["q"], w["k"], w["v"], w["kd"], w["vd"], w["dout"],
+                                    g["out"].cpu(), scale, causal)
     for n in NAMES:
         if cfg["L"] == 0 and n in ("dkd", "dvd"):
             assert g[n] is None
@@ -74,6 +83,25 @@ def test_backward_is_deterministic_in_dk_dv_and_leaves_inputs_intact():
     assert (a["dq"].float() - b["dq"].float()).abs().max().item() < 1e-3
     for k, v in before.items():
         assert torch.equal(v, x[k]), k
+
+
+def test_backward_stages_in_order_equal_one_backward_call():
+    """moda_backward_stages 1, 2, 4 on one stream give moda_backward's results."""
+    cfg = dict(B=1, T=400, Hq=8, Hkv=2, d=128, L=5)
+    x = gpu_inputs(cfg, seed_base=252, with_dout=True)
+    scale = 1 / math.sqrt(128)
+    out, lse = moda.forward(x["q"], x["k"], x["v"], x["kd"], x["vd"], scale, True)
+    ref = moda.backward(x["q"], x["k"], x["v"], x["kd"], x["vd"], out, lse, x["dout"], scale)
+    ws = torch.empty(moda.moda_backward_workspace_size(1, 8, 2, 400, 5, 128), device="cuda",
+                     dtype=torch.uint8)
+    g = {n: torch.empty_like(ref[n]) for n in NAMES}
+    for st in (1, 2, 4):
+        moda.backward(x["q"], x["k"], x["v"], x["kd"], x["vd"], out, lse, x["dout"], scale,
+                      workspace=ws, grads=g, stages=st)
+    moda.check_device_errors()
+    for n in ("dk", "dv", "dkd", "dvd"):
+        assert torch.equal(g[n], ref[n]), n
+    assert (g["dq"].float() - ref["dq"].float()).abs().max().item() < 1e-3
 
 
 def test_L0_backward_matches_torch_autograd():

@@ -24,11 +24,14 @@ CONFIGS = {
     "long-64k-L0": dict(B=1, T=65536, Hq=16, Hkv=4, d=128, L=0),
     "deep-stack": dict(B=4, T=8192, Hq=32, Hkv=8, d=128, L=128),
     "fwd-bwd-16k": dict(B=1, T=16384, Hq=16, Hkv=4, d=128, L=48),
+    # deep-stack head layout at 4K tokens: small enough (2.2 GB of depth cache) for an
+    # ncu capture of the depth-dominated regime
+    "deep-4k": dict(B=1, T=4096, Hq=32, Hkv=8, d=128, L=128),
 }
 
 # seed base per workload (inputs use base*1000 + index, index 0..5 = q,k,v,kd,vd,dout)
 SEED_BASE = {"tiny": 0, "layer-4k": 1, "long-64k": 2, "long-64k-L0": 2, "deep-stack": 3,
-             "fwd-bwd-16k": 4}
+             "fwd-bwd-16k": 4, "deep-4k": 5}
 
 NAMES = ("q", "k", "v", "kd", "vd", "dout")
 
