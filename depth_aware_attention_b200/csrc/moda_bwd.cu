@@ -19,7 +19,8 @@
 //     compute S^T = K Q^T and dP^T = V dO^T into TMEM; the softmax warps turn them into
 //     P^T and dS^T (bf16, back into TMEM, and dS into shared memory); the tensor cores
 //     accumulate dV += P^T dO and dK += dS^T Q in TMEM for the whole walk and compute
-//     dQ = dS K, which the dQ warps add to the fp32 accumulator with vector atomics.
+//     dQ = dS K, which the dQ warps stage in shared memory and the TMA unit adds to the
+//     fp32 accumulator (bulk tensor reduce-add).
 //  3. moda_dq_convert_kernel: dq (bf16) from the fp32 accumulator.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -37,7 +38,7 @@ constexpr int kBwdRegion = 16384;  // one 128-row x 128-byte swizzled region
 constexpr float kLog2eBwd = 1.4426950408889634f;
 
 // ============================================================ 1. depth + row terms
-constexpr int kDepthThreads = 256;
+constexpr int kDepthThreads = 128;
 
 struct BwdDepthArgs {
   const __nv_bfloat16 *q, *out, *dout, *kd, *vd;
@@ -110,15 +111,24 @@ __global__ void __launch_bounds__(kDepthThreads) moda_bwd_depth_kernel(const Bwd
       for (int e = 0; e < 8; ++e) dq[h][e] = 0.f;
 
     const long long tok_off = (bg * a.T + t) * L * D + cs * 8;
-    for (long long j = 0; j < L; ++j) {
-      uint4 kw = make_uint4(0, 0, 0, 0), vw = make_uint4(0, 0, 0, 0);
-      if (valid) {
-        kw = ldg_nc_v4(a.kd + tok_off + j * D);
-        vw = ldg_nc_v4(a.vd + tok_off + j * D);
+    constexpr int kU = 4;  // depth entries whose loads are in flight together
+    for (long long j0 = 0; j0 < L; j0 += kU) {
+      uint4 kwu[kU], vwu[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        kwu[u] = vwu[u] = make_uint4(0, 0, 0, 0);
+        if (valid && j0 + u < L) {
+          kwu[u] = ldg_nc_v4(a.kd + tok_off + (j0 + u) * D);
+          vwu[u] = ldg_nc_v4(a.vd + tok_off + (j0 + u) * D);
+        }
       }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+      if (j0 + u >= L) break;
+      const long long j = j0 + u;
       float kf[8], vf[8];
-      unpack8(kw, kf);
-      unpack8(vw, vf);
+      unpack8(kwu[u], kf);
+      unpack8(vwu[u], vf);
       float y[GM], p[GM];
 #pragma unroll
       for (int h = 0; h < GM; ++h) {
@@ -167,6 +177,7 @@ __global__ void __launch_bounds__(kDepthThreads) moda_bwd_depth_kernel(const Bwd
       if (valid) {
         *reinterpret_cast<uint4*>(a.dvd + tok_off + j * D) = pack8(dv, 1.f);
         *reinterpret_cast<uint4*>(a.dkd + tok_off + j * D) = pack8(dk, a.scale);
+      }
       }
     }
     if (valid) {
@@ -225,7 +236,8 @@ __global__ void __launch_bounds__(kSeqThreads, 1)
     moda_bwd_seq_kernel(const __grid_constant__ CUtensorMap tmQ,
                         const __grid_constant__ CUtensorMap tmDO,
                         const __grid_constant__ CUtensorMap tmK,
-                        const __grid_constant__ CUtensorMap tmV, const SeqArgs a) {
+                        const __grid_constant__ CUtensorMap tmV,
+                        const __grid_constant__ CUtensorMap tmDQ, const SeqArgs a) {
   using Cfg = SeqCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
   // The swizzled operand layouts need a 1024-byte aligned base, and there is no room
@@ -287,7 +299,7 @@ __global__ void __launch_bounds__(kSeqThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
-  // TMEM columns: S^T/P^T [0,128), dP^T/dS^T and then dQ [128,256), dV [256,256+D),
+  // TMEM columns: S^T/P^T and then dQ [0,128), dP^T/dS^T [128,256), dV [256,256+D),
   // dK [256+D, 256+2D).  P^T and dS^T are stored as bf16 hi/lo pairs: each 32-row chunk
   // occupies 32 columns, 16 of packed hi values then 16 of packed lo values.
   const uint32_t tS = tmem, tDP = tmem + 128, tDV = tmem + 256, tDK = tmem + 256 + D;
@@ -328,28 +340,36 @@ __global__ void __launch_bounds__(kSeqThreads, 1)
       constexpr uint32_t idesc_g = make_idesc_bf16(128, D, 0, 1);    // dV, dK (A in TMEM)
       constexpr uint32_t idesc_q = make_idesc_bf16(128, D, 1, 1);    // dQ (A = dS, MN-major)
       mbar_wait(bar(bars->kv_full), 0, abort_flag);
-      for (int i = 0; i < ntiles; ++i) {
-        const int st = i & 1;
-        const uint32_t par = (i >> 1) & 1;
-        mbar_wait(bar(bars->q_full[st]), par, abort_flag);
+      // S^T(i) = K Q(i)^T and dP^T(i) = V dO(i)^T
+      auto issue_s = [&](int i) {
+        mbar_wait(bar(bars->q_full[i & 1]), (i >> 1) & 1, abort_flag);
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t off = (ks / 4) * kBwdRegion + (ks % 4) * 32;
-          mma_ss(tS, make_sdesc_sw128(sK + off, 16, 1024), make_sdesc_sw128(sQ(st) + off, 16, 1024),
-                 idesc_t, ks > 0 ? 1u : 0u);
+          mma_ss(tS, make_sdesc_sw128(sK + off, 16, 1024),
+                 make_sdesc_sw128(sQ(i & 1) + off, 16, 1024), idesc_t, ks > 0 ? 1u : 0u);
         }
         tc_commit(bar(bars->s_full));
-        mbar_wait(bar(bars->do_full[st]), par, abort_flag);
-        if (i > 0) mbar_wait(bar(bars->dq_free), (i - 1) & 1, abort_flag);
+      };
+      auto issue_dp = [&](int i) {
+        mbar_wait(bar(bars->do_full[i & 1]), (i >> 1) & 1, abort_flag);
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t off = (ks / 4) * kBwdRegion + (ks % 4) * 32;
           mma_ss(tDP, make_sdesc_sw128(sV + off, 16, 1024),
-                 make_sdesc_sw128(sDO(st) + off, 16, 1024), idesc_t, ks > 0 ? 1u : 0u);
+                 make_sdesc_sw128(sDO(i & 1) + off, 16, 1024), idesc_t, ks > 0 ? 1u : 0u);
         }
         tc_commit(bar(bars->dp_full));
+      };
+      // Per tile: dV, then dQ into the S^T columns (free once dV has read P^T), then dK,
+      // then the next tile's dP^T (its columns are free once dK has read dS^T).  Only
+      // the next S^T waits for the dQ readout, which overlaps dK and the next dP^T.
+      issue_s(0);
+      issue_dp(0);
+      for (int i = 0; i < ntiles; ++i) {
+        const int st = i & 1;
         mbar_wait(bar(bars->pds_full), i & 1, abort_flag);
         tc_fence_after();
         // dV += P^T dO : A = P^T (TMEM, keys x rows; hi then lo), B = dO (rows x D, MN-major).
@@ -362,6 +382,13 @@ __global__ void __launch_bounds__(kSeqThreads, 1)
           mma_ts(tDV, tS + col + 16, bd, idesc_g, 1u);
         }
         tc_commit(bar(bars->do_empty[st]));
+        // dQ = dS K into the S^T columns : A = dS (rows x keys, MN-major in shared memory),
+        // B = K (keys x D)
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          mma_ss(tS, make_sdesc_sw128(sDS + ks * 2048, kBwdRegion, 1024),
+                 make_sdesc_sw128(sK + ks * 2048, kBwdRegion, 1024), idesc_q, ks > 0 ? 1u : 0u);
+        tc_commit(bar(bars->dq_full));
         // dK += dS^T Q (hi then lo)
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
@@ -370,13 +397,12 @@ __global__ void __launch_bounds__(kSeqThreads, 1)
           mma_ts(tDK, tDP + col, bd, idesc_g, (i > 0 || ks > 0) ? 1u : 0u);
           mma_ts(tDK, tDP + col + 16, bd, idesc_g, 1u);
         }
-        // dQ = dS K : A = dS (rows x keys, MN-major in shared memory), B = K (keys x D)
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-          mma_ss(tDP, make_sdesc_sw128(sDS + ks * 2048, kBwdRegion, 1024),
-                 make_sdesc_sw128(sK + ks * 2048, kBwdRegion, 1024), idesc_q, ks > 0 ? 1u : 0u);
         tc_commit(bar(bars->q_empty[st]));
-        tc_commit(bar(bars->dq_full));
+        if (i + 1 < ntiles) {
+          issue_dp(i + 1);
+          mbar_wait(bar(bars->dq_free), i & 1, abort_flag);
+          issue_s(i + 1);
+        }
       }
       tc_commit(bar(bars->kv_done));
     }
@@ -387,25 +413,32 @@ __global__ void __launch_bounds__(kSeqThreads, 1)
     const int key = key0 + tid;
     const uint32_t lane_base = uint32_t(warp * 32) << 16;
     const int hl = tid % a.G, tok = tid / a.G;
+    // lse and D of row `tid` of tile i, loaded one tile ahead so the global-load latency
+    // stays off the per-tile critical path
+    auto load_rowterms = [&](int i, float& lse2v, float& dv_) {
+      const int t = (first_qt + i) * a.TQ + tok;
+      const bool valid = i < ntiles && tok < a.TQ && t < a.T;
+      const long long idx = ((long long)bg * a.G + hl) * a.T + (valid ? t : 0);
+      lse2v = valid ? -a.lse[idx] * kLog2eBwd : -INFINITY;  // stored negated
+      dv_ = valid ? -a.drow[idx] : 0.f;                      // stored negated
+    };
+    float nxt_lse, nxt_d;
+    load_rowterms(0, nxt_lse, nxt_d);
     for (int i = 0; i < ntiles; ++i) {
       const int qt = first_qt + i;
       const int b = i & 1;
-      {
-        const int t = qt * a.TQ + tok;
-        const bool valid = tok < a.TQ && t < a.T;
-        const long long idx = ((long long)bg * a.G + hl) * a.T + t;
-        ld_s[b * 256 + tid] = valid ? a.lse[idx] * kLog2eBwd : INFINITY;
-        ld_s[b * 256 + 128 + tid] = valid ? a.drow[idx] : 0.f;
-      }
+      ld_s[b * 256 + tid] = nxt_lse;
+      ld_s[b * 256 + 128 + tid] = nxt_d;
       named_bar_sync(1, 128);
+      load_rowterms(i + 1, nxt_lse, nxt_d);
       // rows r < r_min hold tokens before this key (causal) -- their weight is zero
       int r_min = 0;
       if (key >= a.T)
         r_min = 1 << 30;
       else if (a.causal)
         r_min = a.G * (key - qt * a.TQ);
-      const float* lse2 = ld_s + b * 256;
-      const float* dr = ld_s + b * 256 + 128;
+      const float* nlse2 = ld_s + b * 256;      // -lse * log2e per row
+      const float* ndr = ld_s + b * 256 + 128;  // -D per row
       mbar_wait(bar(bars->s_full), i & 1, abort_flag);
       mbar_wait(bar(bars->dp_full), i & 1, abort_flag);
       tc_fence_after();
@@ -420,20 +453,33 @@ __global__ void __launch_bounds__(kSeqThreads, 1)
         // of 2^-9.  Chunk c writes its 32 columns back over the 32 it read: hi in the
         // first 16, lo in the last 16.
         uint32_t pp[16], pl[16], pd[16], dl[16];
+        const bool masked = r_min > c * 32;  // some row of this chunk precedes the key
+        const float2 sl2 = make_float2(a.scale_log2, a.scale_log2);
+        const float2 sc2 = make_float2(a.scale, a.scale);
+        const float2 neg1 = make_float2(-1.f, -1.f);
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
           const int r = c * 32 + e;
-          float P0 = ex2(__uint_as_float(s[e]) * a.scale_log2 - lse2[r]);
-          float P1 = ex2(__uint_as_float(s[e + 1]) * a.scale_log2 - lse2[r + 1]);
-          if (r < r_min) P0 = 0.f;
-          if (r + 1 < r_min) P1 = 0.f;
-          const float d0 = P0 * (__uint_as_float(dp[e]) - dr[r]) * a.scale;
-          const float d1 = P1 * (__uint_as_float(dp[e + 1]) - dr[r + 1]) * a.scale;
-          const uint32_t ph = pack_bf16x2(P0, P1), dh = pack_bf16x2(d0, d1);
+          // P = 2^(s*scale*log2e - lse*log2e); the row terms are stored negated
+          const float2 arg = ffma2(make_float2(__uint_as_float(s[e]), __uint_as_float(s[e + 1])),
+                                   sl2, make_float2(nlse2[r], nlse2[r + 1]));
+          float P0 = ex2(arg.x), P1 = ex2(arg.y);
+          if (masked) {
+            if (r < r_min) P0 = 0.f;
+            if (r + 1 < r_min) P1 = 0.f;
+          }
+          // dS = P * scale * (dP - D)
+          const float2 Ps = fmul2(make_float2(P0, P1), sc2);
+          const float2 dd = fadd2(make_float2(__uint_as_float(dp[e]), __uint_as_float(dp[e + 1])),
+                                  make_float2(ndr[r], ndr[r + 1]));
+          const float2 dS = fmul2(Ps, dd);
+          const uint32_t ph = pack_bf16x2(P0, P1), dh = pack_bf16x2(dS.x, dS.y);
+          const float2 plo = ffma2(make_float2(bf16lo(ph), bf16hi(ph)), neg1, make_float2(P0, P1));
+          const float2 dlo = ffma2(make_float2(bf16lo(dh), bf16hi(dh)), neg1, dS);
           pp[e / 2] = ph;
-          pl[e / 2] = pack_bf16x2(P0 - bf16lo(ph), P1 - bf16hi(ph));
+          pl[e / 2] = pack_bf16x2(plo.x, plo.y);
           pd[e / 2] = dh;
-          dl[e / 2] = pack_bf16x2(d0 - bf16lo(dh), d1 - bf16hi(dh));
+          dl[e / 2] = pack_bf16x2(dlo.x, dlo.y);
         }
         tmem_st16(tS + lane_base + c * 32, pp);
         tmem_st16(tS + lane_base + c * 32 + 16, pl);
@@ -481,31 +527,43 @@ __global__ void __launch_bounds__(kSeqThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ dQ warps 4-7
+    // dQ of each tile is added to the fp32 accumulator by the TMA unit: the warps stage
+    // it, 64 columns at a time, as two 128B-swizzled fp32 regions in the dS buffer (idle
+    // from the dQ product's completion until the next tile's P/dS) and one thread issues
+    // the bulk tensor reduce-adds.
     const int r = threadIdx.x - 128;  // TMEM lane = tile row
     const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
-    const int hl = r % a.G, tok = r / a.G;
     for (int i = 0; i < ntiles; ++i) {
-      const int t = (first_qt + i) * a.TQ + tok;
-      const bool valid = tok < a.TQ && t < a.T;
-      float* dst = a.dqacc + (((long long)bg * a.G + hl) * a.T + (valid ? t : 0)) * D;
+      const int t0q = (first_qt + i) * a.TQ;
       mbar_wait(bar(bars->dq_full), i & 1, abort_flag);
       tc_fence_after();
+#pragma unroll 1
+      for (int half = 0; half < D / 64; ++half) {
 #pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t o[32];
-        tmem_ld32(tDP + lane_base + cc * 32, o);
-        tmem_wait_ld();
-        if (valid) {
+        for (int q = 0; q < 2; ++q) {
+          uint32_t o[32];
+          tmem_ld32(tS + lane_base + half * 64 + q * 32, o);
+          tmem_wait_ld();
+          const uint32_t reg = sDS + q * kBwdRegion + uint32_t(r) * 128;
 #pragma unroll
-          for (int v = 0; v < 8; ++v)
-            red_add_v4(dst + cc * 32 + v * 4, __uint_as_float(o[v * 4]),
-                       __uint_as_float(o[v * 4 + 1]), __uint_as_float(o[v * 4 + 2]),
-                       __uint_as_float(o[v * 4 + 3]));
+          for (int c = 0; c < 8; ++c)
+            sts128(reg + ((uint32_t(c) ^ (uint32_t(r) & 7u)) << 4),
+                   make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]));
         }
+        fence_proxy_async_smem();
+        named_bar_sync(2, 128);
+        if (r == 0) {
+          tma_reduce_add_4d(&tmDQ, sDS, half * 64, 0, t0q, bg);
+          tma_reduce_add_4d(&tmDQ, sDS + kBwdRegion, half * 64 + 32, 0, t0q, bg);
+          bulk_commit_group();
+          bulk_wait_read_all();
+        }
+        named_bar_sync(2, 128);
       }
       tc_fence_before();
       mbar_arrive(bar(bars->dq_free));
     }
+    if (r == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -640,6 +698,23 @@ cudaError_t launch_backward_d(const Problem& p, const void* q, const void* k, co
       return cudaErrorInvalidValue;
     }
   }
+  CUtensorMap mDQ;
+  {
+    // fp32 dq accumulator viewed like q: [bg][t][head-in-group][c]; a box is 32 columns
+    // (128 bytes) of one tile's rows (token, head), 128B-swizzled.
+    const cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(p.G), cuuint64_t(p.T), BG};
+    const cuuint64_t str[3] = {cuuint64_t(p.T) * D * 4, cuuint64_t(D) * 4,
+                               cuuint64_t(p.G) * p.T * D * 4};
+    const cuuint32_t box[4] = {32, cuuint32_t(p.G), cuuint32_t(tg.TQ), 1};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    if (encode(&mDQ, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dqacc, dims, str, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
+      *why = "cuTensorMapEncodeTiled failed for the dq accumulator";
+      return cudaErrorInvalidValue;
+    }
+  }
   SeqArgs sa;
   sa.dk = static_cast<__nv_bfloat16*>(dk);
   sa.dv = static_cast<__nv_bfloat16*>(dv);
@@ -664,7 +739,7 @@ cudaError_t launch_backward_d(const Problem& p, const void* q, const void* k, co
   const int nkb = (p.T + 127) / 128;
   if (stages & kStageSeq)
     moda_bwd_seq_kernel<D><<<unsigned(BG) * nkb, kSeqThreads, SeqCfg<D>::kSmemBytes, stream>>>(
-      mQ, mDO, mK, mV, sa);
+      mQ, mDO, mK, mV, mDQ, sa);
   e = cudaGetLastError();
   if (e != cudaSuccess) {
     *why = "sequence backward launch failed";

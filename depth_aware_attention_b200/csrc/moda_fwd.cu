@@ -193,7 +193,27 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         tma_prefetch_desc(&tmVD);
       }
       const uint32_t dbytes = 128u * a.TQ * a.JC;
-      for (int idx = 0; idx < NC * kDUses; ++idx) {
+      // Each use is also pulled into L2 kDPrefetch uses ahead of its load, so the ring's
+      // few shared-memory stages refill from L2 rather than from DRAM.
+      constexpr int kDPrefetch = 6;
+      const int nuse = NC * kDUses;
+      auto box = [&](int idx, const CUtensorMap*& map, int& x, int& y) {
+        const int u = idx % kDUses;
+        map = (u < Cfg::kRegions) ? &tmKD : &tmVD;
+        x = (u % Cfg::kRegions) * 64;
+        y = (idx / kDUses) * a.JC;
+      };
+      for (int idx = 0; idx < kDPrefetch && idx < nuse; ++idx) {
+        const CUtensorMap* map; int x, y;
+        box(idx, map, x, y);
+        tma_prefetch_l2_4d(map, x, y, t ? tq1 : tq0, bg);
+      }
+      for (int idx = 0; idx < nuse; ++idx) {
+        if (idx + kDPrefetch < nuse) {
+          const CUtensorMap* pmap; int px, py;
+          box(idx + kDPrefetch, pmap, px, py);
+          tma_prefetch_l2_4d(pmap, px, py, t ? tq1 : tq0, bg);
+        }
         const int s = idx % NDS;
         if (idx >= NDS)
           mbar_wait(bar(bars->dempty[t][s]), ((idx / NDS) - 1) & 1, abort_flag);
