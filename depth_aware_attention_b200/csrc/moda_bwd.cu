@@ -228,6 +228,7 @@ struct SeqArgs {
   float* dqacc;
   const float *lse, *drow;
   int Hkv, T, G, TQ, nqt, BG, causal;
+  int half_box;  // 64 % G == 0: a 64-row half of a query tile is whole tokens
   float scale, scale_log2;
 };
 
@@ -574,6 +575,398 @@ __global__ void __launch_bounds__(kSeqThreads, 1)
   }
 }
 
+// ============================================================ 2b. sequence part, d = 128,
+// query tiles processed as two 64-row halves
+//
+// Same algorithm as moda_bwd_seq_kernel, software-pipelined over the two 64-row halves h
+// of each query tile so that one half's P/dS math and dQ readout overlap the other
+// half's tensor-core products.  TMEM: region A_h = columns [64h, 64h+64) holds S^T_h,
+// then P^T_h (bf16 hi/lo), then dQ^T_h; region B_h = [128+64h, 128+64h+64) holds dP^T_h,
+// then dS^T_h (hi/lo); dV [256,384), dK [384,512).  dQ^T_h = K^T dS_h^T is an M = 128
+// (head-dimension lanes) product, so every tensor-core result keeps the 128-lane layout.
+// The dQ warps stage dQ_h through the half's own dS region (free once dQ^T_h has read
+// it) as row-major fp32 and hand each row to a 1-D bulk reduce-add into the accumulator.
+//
+// Tensor-core issue order per tile i (primes: tile i+1):
+//   [pds0] dV0 dK0 dQ0 dP0'   [pds1] dV1 dK1 [dqfree0] S0' dQ1 dP1'   [dqfree1] S1'
+struct SeqHBars {
+  uint64_t kv_full;
+  uint64_t q_full[2], q_empty[2];
+  uint64_t do_full[2], do_empty[2];
+  uint64_t s_full[2], dp_full[2], pds_full[2], dq_full[2], dq_free[2];
+  uint64_t kv_done;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__global__ void __launch_bounds__(kSeqThreads, 1)
+    moda_bwd_seq_h_kernel(const __grid_constant__ CUtensorMap tmQ,
+                          const __grid_constant__ CUtensorMap tmDO,
+                          const __grid_constant__ CUtensorMap tmK,
+                          const __grid_constant__ CUtensorMap tmV,
+                          const __grid_constant__ CUtensorMap tmDQh, const SeqArgs a) {
+  constexpr int D = 128;
+  using Cfg = SeqCfg<D>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if (smem_u32(smem) & 1023u) {
+    if (threadIdx.x == 0) atomicOr(&g_error_word, kErrInternal);
+    return;
+  }
+  const uint32_t s0 = smem_u32(smem);
+  const uint32_t sK = s0 + Cfg::kOffK, sV = s0 + Cfg::kOffV, sDS = s0 + Cfg::kOffDS;
+  auto sQ = [&](int st) { return s0 + Cfg::kOffQ + uint32_t(st) * Cfg::kTile; };
+  auto sDO = [&](int st) { return s0 + Cfg::kOffDO + uint32_t(st) * Cfg::kTile; };
+  float* ld_s = reinterpret_cast<float*>(smem + Cfg::kOffLD);
+  SeqHBars* bars = reinterpret_cast<SeqHBars*>(smem + Cfg::kOffBar);
+  volatile int* abort_flag = &bars->abort;
+  auto bar = [&](uint64_t& b) { return smem_u32(&b); };
+
+  const int warp = threadIdx.x >> 5;
+  const int bg = blockIdx.x % a.BG;
+  const int kb = blockIdx.x / a.BG;
+  const int key0 = kb * 128;
+  const int first_qt = a.causal ? key0 / a.TQ : 0;
+  const int ntiles = a.nqt - first_qt;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(bars->kv_full), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(bars->q_full[i]), 1);
+      mbar_init(bar(bars->q_empty[i]), 1);
+      mbar_init(bar(bars->do_full[i]), 1);
+      mbar_init(bar(bars->do_empty[i]), 1);
+      mbar_init(bar(bars->s_full[i]), 1);
+      mbar_init(bar(bars->dp_full[i]), 1);
+      mbar_init(bar(bars->pds_full[i]), 128);
+      mbar_init(bar(bars->dq_full[i]), 1);
+      mbar_init(bar(bars->dq_free[i]), 128);
+    }
+    mbar_init(bar(bars->kv_done), 1);
+    bars->abort = 0;
+    fence_barrier_init();
+  }
+  // Q/dO rows past TQ*G (G not dividing 128) never receive TMA data: zero them once.
+  if (threadIdx.x < 128 && threadIdx.x >= a.TQ * a.G) {
+    for (int st = 0; st < 2; ++st)
+      for (int rg = 0; rg < Cfg::kRegions; ++rg) {
+        uint4* rq = reinterpret_cast<uint4*>(smem + Cfg::kOffQ + st * Cfg::kTile +
+                                             rg * kBwdRegion + threadIdx.x * 128);
+        uint4* rd = reinterpret_cast<uint4*>(smem + Cfg::kOffDO + st * Cfg::kTile +
+                                             rg * kBwdRegion + threadIdx.x * 128);
+        for (int c = 0; c < 8; ++c) rq[c] = rd[c] = make_uint4(0, 0, 0, 0);
+      }
+    fence_proxy_async_smem();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(&bars->tmem_base), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  auto tA = [&](int h) { return tmem + uint32_t(64 * h); };
+  auto tB = [&](int h) { return tmem + uint32_t(128 + 64 * h); };
+  const uint32_t tDV = tmem + 256, tDK = tmem + 384;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
+    if (elect_one()) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmDO);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      mbar_expect_tx(bar(bars->kv_full), 2 * Cfg::kTile);
+      for (int rg = 0; rg < Cfg::kRegions; ++rg) {
+        tma_load_3d(sK + rg * kBwdRegion, &tmK, bar(bars->kv_full), rg * 64, key0, bg);
+        tma_load_3d(sV + rg * kBwdRegion, &tmV, bar(bars->kv_full), rg * 64, key0, bg);
+      }
+      const uint32_t qbytes = Cfg::kRegions * 128 * a.G * a.TQ;
+      for (int i = 0; i < ntiles; ++i) {
+        const int st = i & 1;
+        const int t0 = (first_qt + i) * a.TQ;
+        if (i >= 2) mbar_wait(bar(bars->q_empty[st]), ((i >> 1) - 1) & 1, abort_flag);
+        mbar_expect_tx(bar(bars->q_full[st]), qbytes);
+        for (int rg = 0; rg < Cfg::kRegions; ++rg)
+          tma_load_4d(sQ(st) + rg * kBwdRegion, &tmQ, bar(bars->q_full[st]), rg * 64, 0, t0,
+                      bg);
+        if (i >= 2) mbar_wait(bar(bars->do_empty[st]), ((i >> 1) - 1) & 1, abort_flag);
+        mbar_expect_tx(bar(bars->do_full[st]), qbytes);
+        for (int rg = 0; rg < Cfg::kRegions; ++rg)
+          tma_load_4d(sDO(st) + rg * kBwdRegion, &tmDO, bar(bars->do_full[st]), rg * 64, 0,
+                      t0, bg);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ tcgen05 issuer
+    if (elect_one()) {
+      constexpr uint32_t idesc_t = make_idesc_bf16(128, 64, 0, 0);  // S^T_h, dP^T_h
+      constexpr uint32_t idesc_g = make_idesc_bf16(128, D, 0, 1);   // dV, dK (A in TMEM)
+      constexpr uint32_t idesc_q = make_idesc_bf16(128, 64, 1, 1);  // dQ^T_h = K^T dS_h^T
+      mbar_wait(bar(bars->kv_full), 0, abort_flag);
+      // S^T_h(i) = K Q_h(i)^T, dP^T_h(i) = V dO_h(i)^T : B = the half's 64 rows, K-major
+      auto issue_s = [&](int i, int h) {
+        if (h == 0) {
+          mbar_wait(bar(bars->q_full[i & 1]), (i >> 1) & 1, abort_flag);
+          tc_fence_after();
+        }
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t off = (ks / 4) * kBwdRegion + (ks % 4) * 32;
+          mma_ss(tA(h), make_sdesc_sw128(sK + off, 16, 1024),
+                 make_sdesc_sw128(sQ(i & 1) + off + 8192 * h, 16, 1024), idesc_t,
+                 ks > 0 ? 1u : 0u);
+        }
+        tc_commit(bar(bars->s_full[h]));
+      };
+      auto issue_dp = [&](int i, int h) {
+        if (h == 0) {
+          mbar_wait(bar(bars->do_full[i & 1]), (i >> 1) & 1, abort_flag);
+          tc_fence_after();
+        }
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t off = (ks / 4) * kBwdRegion + (ks % 4) * 32;
+          mma_ss(tB(h), make_sdesc_sw128(sV + off, 16, 1024),
+                 make_sdesc_sw128(sDO(i & 1) + off + 8192 * h, 16, 1024), idesc_t,
+                 ks > 0 ? 1u : 0u);
+        }
+        tc_commit(bar(bars->dp_full[h]));
+      };
+      // dV += P_h^T dO_h, dK += dS_h^T Q_h (hi then lo; K-step ks covers the half's rows
+      // 16ks..16ks+15: packed columns 32(ks/2) + 8(ks%2) of the region, lo +16), then
+      // dQ^T_h = K^T dS_h^T into region A_h.
+      auto issue_grads = [&](int i, int h) {
+        mbar_wait(bar(bars->pds_full[h]), i & 1, abort_flag);
+        tc_fence_after();
+        const int st = i & 1;
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint32_t col = (ks >> 1) * 32 + (ks & 1) * 8;
+          const uint64_t bd = make_sdesc_sw128(sDO(st) + (4 * h + ks) * 2048, kBwdRegion, 1024);
+          mma_ts(tDV, tA(h) + col, bd, idesc_g, (i > 0 || h > 0 || ks > 0) ? 1u : 0u);
+          mma_ts(tDV, tA(h) + col + 16, bd, idesc_g, 1u);
+        }
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint32_t col = (ks >> 1) * 32 + (ks & 1) * 8;
+          const uint64_t bd = make_sdesc_sw128(sQ(st) + (4 * h + ks) * 2048, kBwdRegion, 1024);
+          mma_ts(tDK, tB(h) + col, bd, idesc_g, (i > 0 || h > 0 || ks > 0) ? 1u : 0u);
+          mma_ts(tDK, tB(h) + col + 16, bd, idesc_g, 1u);
+        }
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          mma_ss(tA(h), make_sdesc_sw128(sK + ks * 2048, kBwdRegion, 1024),
+                 make_sdesc_sw128(sDS + h * kBwdRegion + ks * 2048, kBwdRegion, 1024), idesc_q,
+                 ks > 0 ? 1u : 0u);
+        tc_commit(bar(bars->dq_full[h]));
+      };
+      issue_s(0, 0);
+      issue_dp(0, 0);
+      issue_s(0, 1);
+      issue_dp(0, 1);
+      for (int i = 0; i < ntiles; ++i) {
+        const bool more = i + 1 < ntiles;
+        issue_grads(i, 0);
+        if (more) issue_dp(i + 1, 0);
+        issue_grads(i, 1);
+        tc_commit(bar(bars->do_empty[i & 1]));
+        tc_commit(bar(bars->q_empty[i & 1]));
+        if (more) {
+          mbar_wait(bar(bars->dq_free[0]), i & 1, abort_flag);
+          issue_s(i + 1, 0);
+          issue_dp(i + 1, 1);
+          mbar_wait(bar(bars->dq_free[1]), i & 1, abort_flag);
+          issue_s(i + 1, 1);
+        }
+      }
+      tc_commit(bar(bars->kv_done));
+    }
+    __syncwarp();
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ P / dS warps
+    const int tid = threadIdx.x;  // TMEM lane = key key0 + tid
+    const int key = key0 + tid;
+    const uint32_t lane_base = uint32_t(warp * 32) << 16;
+    const int hl = tid % a.G, tok = tid / a.G;
+    auto load_rowterms = [&](int i, float& nl, float& nd) {
+      const int t = (first_qt + i) * a.TQ + tok;
+      const bool valid = i < ntiles && tok < a.TQ && t < a.T;
+      const long long idx = ((long long)bg * a.G + hl) * a.T + (valid ? t : 0);
+      nl = valid ? -a.lse[idx] * kLog2eBwd : -INFINITY;  // stored negated
+      nd = valid ? -a.drow[idx] : 0.f;                   // stored negated
+    };
+    float nxt_lse, nxt_d;
+    load_rowterms(0, nxt_lse, nxt_d);
+    const float2 sl2 = make_float2(a.scale_log2, a.scale_log2);
+    const float2 sc2 = make_float2(a.scale, a.scale);
+    const float2 neg1 = make_float2(-1.f, -1.f);
+    for (int i = 0; i < ntiles; ++i) {
+      const int qt = first_qt + i;
+      const int b = i & 1;
+      ld_s[b * 256 + tid] = nxt_lse;
+      ld_s[b * 256 + 128 + tid] = nxt_d;
+      named_bar_sync(1, 128);
+      load_rowterms(i + 1, nxt_lse, nxt_d);
+      int r_min = 0;
+      if (key >= a.T)
+        r_min = 1 << 30;
+      else if (a.causal)
+        r_min = a.G * (key - qt * a.TQ);
+      const float* nlse2 = ld_s + b * 256;
+      const float* ndr = ld_s + b * 256 + 128;
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        mbar_wait(bar(bars->s_full[h]), i & 1, abort_flag);
+        mbar_wait(bar(bars->dp_full[h]), i & 1, abort_flag);
+        tc_fence_after();
+#pragma unroll 1
+        for (int cl = 0; cl < 2; ++cl) {
+          const int c = 2 * h + cl;  // 32-row chunk of the tile
+          uint32_t s[32], dp[32];
+          tmem_ld32(tA(h) + lane_base + cl * 32, s);
+          tmem_ld32(tB(h) + lane_base + cl * 32, dp);
+          tmem_wait_ld();
+          uint32_t pp[16], pl[16], pd[16], dl[16];
+          const bool masked = r_min > c * 32;
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const int r = c * 32 + e;
+            const float2 arg = ffma2(
+                make_float2(__uint_as_float(s[e]), __uint_as_float(s[e + 1])), sl2,
+                make_float2(nlse2[r], nlse2[r + 1]));
+            float P0 = ex2(arg.x), P1 = ex2(arg.y);
+            if (masked) {
+              if (r < r_min) P0 = 0.f;
+              if (r + 1 < r_min) P1 = 0.f;
+            }
+            const float2 Ps = fmul2(make_float2(P0, P1), sc2);
+            const float2 dd = fadd2(
+                make_float2(__uint_as_float(dp[e]), __uint_as_float(dp[e + 1])),
+                make_float2(ndr[r], ndr[r + 1]));
+            const float2 dS = fmul2(Ps, dd);
+            const uint32_t ph = pack_bf16x2(P0, P1), dh = pack_bf16x2(dS.x, dS.y);
+            const float2 plo =
+                ffma2(make_float2(bf16lo(ph), bf16hi(ph)), neg1, make_float2(P0, P1));
+            const float2 dlo = ffma2(make_float2(bf16lo(dh), bf16hi(dh)), neg1, dS);
+            pp[e / 2] = ph;
+            pl[e / 2] = pack_bf16x2(plo.x, plo.y);
+            pd[e / 2] = dh;
+            dl[e / 2] = pack_bf16x2(dlo.x, dlo.y);
+          }
+          tmem_st16(tA(h) + lane_base + cl * 32, pp);
+          tmem_st16(tA(h) + lane_base + cl * 32 + 16, pl);
+          tmem_st16(tB(h) + lane_base + cl * 32, pd);
+          tmem_st16(tB(h) + lane_base + cl * 32 + 16, dl);
+          // dS for the dQ^T product: region h, this key's row, rows 32cl..32cl+31 of the half
+          const uint32_t reg = sDS + h * kBwdRegion + uint32_t(tid) * 128;
+#pragma unroll
+          for (int qd = 0; qd < 4; ++qd) {
+            const uint32_t chunk = cl * 4 + qd;
+            sts128(reg + ((chunk ^ (tid & 7)) << 4),
+                   make_uint4(pd[qd * 4], pd[qd * 4 + 1], pd[qd * 4 + 2], pd[qd * 4 + 3]));
+          }
+        }
+        tmem_wait_st();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(bar(bars->pds_full[h]));
+      }
+    }
+    // epilogue: dV, dK rows of this key
+    mbar_wait(bar(bars->kv_done), 0, abort_flag);
+    tc_fence_after();
+    const bool kvalid = key < a.T;
+    const long long koff = ((long long)bg * a.T + (kvalid ? key : 0)) * D;
+#pragma unroll 1
+    for (int which = 0; which < 2; ++which) {
+      const uint32_t tsrc = (which ? tDK : tDV) + lane_base;
+      __nv_bfloat16* dst = (which ? a.dk : a.dv) + koff;
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t o[32];
+        tmem_ld32(tsrc + cc * 32, o);
+        tmem_wait_ld();
+        if (kvalid) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            float f[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(o[v * 8 + e]);
+            d4[v] = pack8(f, 1.f);
+          }
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ dQ warps 4-7
+    // Thread = TMEM lane = head-dimension index c of dQ^T_h.  Two rounds per half: the
+    // threads of columns [64rd, 64rd+64) write their 64 row values into the half's dS
+    // region as row-major fp32 [64 rows][64 columns]; then 64 threads each hand one row
+    // (256 bytes) to a bulk reduce-add.
+    const int c = threadIdx.x - 128;
+    const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
+    for (int i = 0; i < ntiles; ++i) {
+      const int t0q = (first_qt + i) * a.TQ;
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        mbar_wait(bar(bars->dq_full[h]), i & 1, abort_flag);
+        tc_fence_after();
+        uint32_t o[64];
+        tmem_ld32(tA(h) + lane_base, o);
+        tmem_ld32(tA(h) + lane_base + 32, o + 32);
+        tmem_wait_ld();
+        const uint32_t stage = sDS + h * kBwdRegion;
+#pragma unroll 1
+        for (int rd = 0; rd < 2; ++rd) {
+          if ((c >> 6) == rd) {
+            const uint32_t col = uint32_t(c & 63) * 4;
+#pragma unroll
+            for (int row = 0; row < 64; ++row)
+              asm volatile("st.shared.b32 [%0], %1;" ::"r"(stage + row * 256 + col),
+                           "r"(o[row])
+                           : "memory");
+          }
+          fence_proxy_async_smem();
+          named_bar_sync(2, 128);
+          if (a.half_box) {
+            // the half's 64 rows are whole tokens: one tensor box (64 columns x G heads x
+            // 64/G tokens) covers the staged rows
+            if (c == 0) {
+              tma_reduce_add_4d(&tmDQh, stage, 64 * rd, 0, t0q + (64 * h) / a.G, bg);
+              bulk_commit_group();
+              bulk_wait_read_all();
+            }
+          } else if (c < 64) {
+            const int R = 64 * h + c;  // tile row
+            const int tok = R / a.G, hl = R - (R / a.G) * a.G;
+            const int t = t0q + tok;
+            if (tok < a.TQ && t < a.T) {
+              float* dst = a.dqacc + (((long long)bg * a.G + hl) * a.T + t) * D + 64 * rd;
+              bulk_reduce_add_f32(dst, stage + c * 256, 256);
+            }
+            bulk_commit_group();
+            bulk_wait_read_all();
+          }
+          named_bar_sync(2, 128);
+        }
+        tc_fence_before();
+        mbar_arrive(bar(bars->dq_free[h]));
+      }
+    }
+    if (c < 64) bulk_wait_all();  // (thread 0 also covers the tensor-box path)
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 // ============================================================ 3. dq convert
 __global__ void __launch_bounds__(256) moda_dq_convert_kernel(const float* __restrict__ acc,
                                                               __nv_bfloat16* __restrict__ dq,
@@ -737,9 +1130,37 @@ cudaError_t launch_backward_d(const Problem& p, const void* q, const void* k, co
     return e;
   }
   const int nkb = (p.T + 127) / 128;
-  if (stages & kStageSeq)
+  sa.half_box = (64 % p.G) == 0;
+  CUtensorMap mDQh = mDQ;
+  if (sa.half_box) {
+    // fp32 dq accumulator as [bg][t][head-in-group][c]: one box = 64 columns (256 bytes,
+    // no swizzle) of the 64/G tokens x G heads of a half tile, row-major like the staging
+    const cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(p.G), cuuint64_t(p.T), BG};
+    const cuuint64_t str[3] = {cuuint64_t(p.T) * D * 4, cuuint64_t(D) * 4,
+                               cuuint64_t(p.G) * p.T * D * 4};
+    const cuuint32_t box[4] = {64, cuuint32_t(p.G), cuuint32_t(64 / p.G), 1};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    if (encode(&mDQh, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dqacc, dims, str, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
+      *why = "cuTensorMapEncodeTiled failed for the dq accumulator (half tiles)";
+      return cudaErrorInvalidValue;
+    }
+  }
+  if ((stages & kStageSeq) && D == 128) {
+    e = cudaFuncSetAttribute(moda_bwd_seq_h_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SeqCfg<128>::kSmemBytes);
+    if (e != cudaSuccess) {
+      *why = "cudaFuncSetAttribute(sequence backward, halves) failed";
+      return e;
+    }
+    moda_bwd_seq_h_kernel<<<unsigned(BG) * nkb, kSeqThreads, SeqCfg<128>::kSmemBytes,
+                            stream>>>(mQ, mDO, mK, mV, mDQh, sa);
+  } else if (stages & kStageSeq) {
     moda_bwd_seq_kernel<D><<<unsigned(BG) * nkb, kSeqThreads, SeqCfg<D>::kSmemBytes, stream>>>(
       mQ, mDO, mK, mV, mDQ, sa);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) {
     *why = "sequence backward launch failed";
