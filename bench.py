@@ -57,6 +57,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle sample")
+    ap.add_argument("--sweep", action="store_true",
+                    help="forward efficiency sweep over T x L (not the headline step)")
     return ap.parse_args()
 
 
@@ -198,6 +200,15 @@ def step_flops(cfg, fwd_only):
     return f if fwd_only else f * (1.0 + BWD_FLOP_FACTOR)
 
 
+def forward_bytes(cfg):
+    """Algorithmic bytes of one forward: every input read once, every output written once."""
+    B, Hq, Hkv, T, L, d = (cfg[n] for n in ("B", "Hq", "Hkv", "T", "L", "d"))
+    return (2 * B * Hq * T * d * 2              # q read, out written (bf16)
+            + 2 * B * Hkv * T * d * 2           # k, v
+            + workloads.depth_bytes(**cfg)      # kd, vd
+            + B * Hq * T * 4)                   # lse
+
+
 def kernel_roofline(name, cfg, avg_ms, pk, workload):
     """Roofline entry for one kernel: algorithmic work per launch over its average
     CUDA-event duration, against the measured sustained peak (every kernel here runs
@@ -205,8 +216,17 @@ def kernel_roofline(name, cfg, avg_ms, pk, workload):
     B, Hq, Hkv, T, L, d = (cfg[n] for n in ("B", "Hq", "Hkv", "T", "L", "d"))
     rows = B * Hq * T
     if name == "moda_fwd_kernel":
-        bound, work = "tensor", workloads.forward_flops(**cfg)
-        what = "4*B*Hq*d*(T^2/2 + T*L) FLOPs"
+        # the bound is whichever side takes longer at the measured peaks: the FLOPs at
+        # tensor speed, or the algorithmic bytes (inputs read once, outputs written once)
+        # at HBM speed -- the depth cache dominates the bytes when L is large
+        flops = workloads.forward_flops(**cfg)
+        fbytes = forward_bytes(cfg)
+        if fbytes / (pk["hbm"] * 1e9) > flops / (pk["bf16_sustained"] * 1e12):
+            bound, work = "hbm", fbytes
+            what = "bytes: q, k, v, kd, vd read once; out, lse written once"
+        else:
+            bound, work = "tensor", flops
+            what = "4*B*Hq*d*(T^2/2 + T*L) FLOPs"
     elif name == "moda_bwd_seq_kernel":
         bound, work = "tensor", BWD_FLOP_FACTOR * 4.0 * B * Hq * d * T * T / 2.0
         what = "2.5 x 4*B*Hq*d*T^2/2 FLOPs (sequence part of the backward)"
@@ -471,8 +491,60 @@ def run_reference(args, world, rank):
     return dict(value=value, ms=flops / (value * 1e12) * 1e3, cpu=dict(last, value=value))
 
 
+def run_sweep(args):
+    """Forward time over T in {4K..64K} x L in {0, 8, 32, 128} at the 1.5B-layer head shape
+    (B=1, Hq=16, Hkv=4, d=128): TFLOP/s and the ratio time(L=0)/time(L) per point, the
+    shape of the pages' efficiency-scaling experiment (the depth overhead shrinks as T
+    grows).  Prints one JSON line per point, then a markdown table."""
+    import depth_aware_attention_b200 as moda
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+    rows = []
+    for T in (4096, 8192, 16384, 32768, 65536):
+        ms0 = None
+        for L in (0, 8, 32, 128):
+            cfg = dict(B=1, T=T, Hq=16, Hkv=4, d=128, L=L)
+            x = workloads.make_inputs(cfg, 900 + T // 4096, dev)
+            out = torch.empty_like(x["q"])
+            lse = torch.empty(x["q"].shape[:3], device=dev, dtype=torch.float32)
+            f = lambda: moda.forward(x["q"], x["k"], x["v"], x["kd"], x["vd"], None, True,
+                                     out=out, lse=lse)
+            for _ in range(3):
+                f()
+            torch.cuda.synchronize(dev)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            n = 3 if T >= 32768 else 10
+            e0.record(stream)
+            for _ in range(n):
+                f()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            ms = e0.elapsed_time(e1) / n
+            moda.check_device_errors()
+            if L == 0:
+                ms0 = ms
+            tf = workloads.forward_flops(**cfg) / (ms * 1e-3) / 1e12
+            row = {"T": T, "L": L, "ms": round(ms, 4), "tflops": round(tf, 1),
+                   "time_ratio_L0_over_L": round(ms0 / ms, 4),
+                   "depth_gbs_from_difference": (round(workloads.depth_bytes(**cfg) /
+                                                       ((ms - ms0) * 1e-3) / 1e9, 1)
+                                                 if L and ms > ms0 * 1.02 else None)}
+            print(json.dumps(row), flush=True)
+            rows.append(row)
+            del x, out, lse
+            torch.cuda.empty_cache()
+    print("| T | L | ms | TFLOP/s | time(L=0)/time(L) |")
+    print("|---|---|---|---|---|")
+    for r in rows:
+        print(f"| {r['T']} | {r['L']} | {r['ms']:.3f} | {r['tflops']:.0f} | "
+              f"{r['time_ratio_L0_over_L']:.3f} |")
+
+
 def main():
     args = parse()
+    if args.sweep:
+        run_sweep(args)
+        return
     world, rank, local = dist_setup(args.gpus)
     cfg = workloads.CONFIGS[args.workload]
     config = {"workload": args.workload, **{k: cfg[k] for k in ("B", "T", "Hq", "Hkv", "d", "L")},

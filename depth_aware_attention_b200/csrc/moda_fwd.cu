@@ -134,7 +134,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     for (int t = 0; t < 2; ++t) {
       for (int s = 0; s < NDS; ++s) {
         mbar_init(bar(bars->dfull[t][s]), 1);
-        mbar_init(bar(bars->dempty[t][s]), 1);
+        mbar_init(bar(bars->dempty[t][s]), 128);
       }
       mbar_init(bar(bars->s_full[t]), 1);
       mbar_init(bar(bars->p_full[t]), 1);
@@ -314,9 +314,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         mbar_wait(bar(bars->dfull[tt][s]), (use / NDS) & 1, abort_flag);
         return sDS(tt, s);
       };
+      // every thread releases the stage itself (the empty barrier counts 128 arrivals),
+      // so a fast thread never waits at a barrier for the slow ones of the warpgroup
       auto give = [&]() {
-        named_bar_sync(wg_bar, 128);
-        if (r == 0) mbar_arrive(bar(bars->dempty[tt][use % NDS]));
+        mbar_arrive(bar(bars->dempty[tt][use % NDS]));
         ++use;
       };
       for (int ci = 0; ci < NC; ++ci) {
