@@ -19,8 +19,9 @@
 //     compute S^T = K Q^T and dP^T = V dO^T into TMEM; the softmax warps turn them into
 //     P^T and dS^T (bf16, back into TMEM, and dS into shared memory); the tensor cores
 //     accumulate dV += P^T dO and dK += dS^T Q in TMEM for the whole walk and compute
-//     dQ = dS K, which the dQ warps stage in shared memory and the TMA unit adds to the
-//     fp32 accumulator (bulk tensor reduce-add).
+//     dQ = dS K, which the dQ warps add to the fp32 accumulator: for d = 64 staged in
+//     shared memory and added by the TMA unit (bulk tensor reduce-add), for d = 128 (the
+//     half-tile variant, 2b) straight from registers with global reductions.
 //  3. moda_dq_convert_kernel: dq (bf16) from the fp32 accumulator.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -228,7 +229,6 @@ struct SeqArgs {
   float* dqacc;
   const float *lse, *drow;
   int Hkv, T, G, TQ, nqt, BG, causal;
-  int half_box;  // 64 % G == 0: a 64-row half of a query tile is whole tokens
   float scale, scale_log2;
 };
 
@@ -584,11 +584,19 @@ __global__ void __launch_bounds__(kSeqThreads, 1)
 // then P^T_h (bf16 hi/lo), then dQ^T_h; region B_h = [128+64h, 128+64h+64) holds dP^T_h,
 // then dS^T_h (hi/lo); dV [256,384), dK [384,512).  dQ^T_h = K^T dS_h^T is an M = 128
 // (head-dimension lanes) product, so every tensor-core result keeps the 128-lane layout.
-// The dQ warps stage dQ_h through the half's own dS region (free once dQ^T_h has read
-// it) as row-major fp32 and hand each row to a 1-D bulk reduce-add into the accumulator.
+// The dQ warps read dQ^T_h out of TMEM (thread = head-dimension column), release the
+// region at once and add the values to the fp32 accumulator with global reductions, a
+// warp covering 128 consecutive bytes of one row.  An SM moves about 40 GB/s into L2
+// either way (TMA bulk reduce-add or per-thread reductions), so the readout is bound by
+// that outbound rate; reductions from registers keep it off the tensor pipe's critical
+// path: no shared-memory staging, no wait for the TMA unit before TMEM is released.
 //
 // Tensor-core issue order per tile i (primes: tile i+1):
-//   [pds0] dV0 dK0 dQ0 dP0'   [pds1] dV1 dK1 [dqfree0] S0' dQ1 dP1'   [dqfree1] S1'
+//   [pds0] dV0 dK0 dQ0 dP0' [dqfree0] S0'   [pds1] dV1 dK1 dQ1 dP1' [dqfree1] S1'
+// so that the softmax warps work on half 0 of tile i+1 while the tensor cores run the
+// products of half 1 of tile i (and the reverse), instead of waiting on each other.
+constexpr int kSeqHThreads = 448;  // warps 0-7 P/dS, 8-11 dQ, 12 TMA, 13 tcgen05
+
 struct SeqHBars {
   uint64_t kv_full;
   uint64_t q_full[2], q_empty[2];
@@ -599,12 +607,71 @@ struct SeqHBars {
   int abort;
 };
 
-__global__ void __launch_bounds__(kSeqThreads, 1)
+// dQ warps of moda_bwd_seq_h_kernel.  Thread = TMEM lane = head-dimension index c of
+// dQ^T_h: per half it reads its 64 row values, frees the TMEM region at once and adds
+// the values to the fp32 accumulator with global reductions (a warp covers 32
+// consecutive columns of one row: 128 bytes).  Half row r is tile row R = 64h + r, i.e.
+// token R / G and head R % G.  GT = G for a power of two up to 16, so that each row's
+// offset from its head's base pointer is a compile-time constant; GT = 0 handles any G.
+template <int GT>
+__device__ __forceinline__ void dq_readout(const SeqArgs& a, SeqHBars* bars, uint32_t tmem,
+                                           uint32_t lane_base, int c, int bg, int first_qt,
+                                           int ntiles) {
+  constexpr int D = 128;
+  volatile int* abort_flag = &bars->abort;
+  const long long hs = (long long)a.T * D;
+  for (int i = 0; i < ntiles; ++i) {
+    const int t0q = (first_qt + i) * a.TQ;
+    const int ntok = min(a.TQ, a.T - t0q);  // valid tokens of this tile
+#pragma unroll 1
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t tA = tmem + uint32_t(64 * h);
+      mbar_wait(smem_u32(&bars->dq_full[h]), i & 1, abort_flag);
+      tc_fence_after();
+      uint32_t o[64];
+      tmem_ld32(tA + lane_base, o);
+      tmem_ld32(tA + lane_base + 32, o + 32);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&bars->dq_free[h]));
+      if constexpr (GT > 0) {
+        const int tok0 = (64 * h) / GT;
+        const int nv = ntok - tok0;
+        float* const base = a.dqacc + ((long long)bg * GT * a.T + t0q + tok0) * D + c;
+        // rows in order (heads cycling fastest), in blocks of up to four heads so that at
+        // most four base pointers are live; issuing the rows in order measured faster
+        // than head by head
+        constexpr int HB = GT < 4 ? GT : 4;
+#pragma unroll
+        for (int hb = 0; hb < GT / HB; ++hb) {
+          float* ph[HB];
+#pragma unroll
+          for (int j = 0; j < HB; ++j) ph[j] = base + (hb * HB + j) * hs;
+#pragma unroll
+          for (int tk = 0; tk < 64 / GT; ++tk)
+#pragma unroll
+            for (int j = 0; j < HB; ++j)
+              if (tk < nv) red_add_f32(ph[j] + tk * D, __uint_as_float(o[tk * GT + hb * HB + j]));
+        }
+      } else {
+        float* const base = a.dqacc + ((long long)bg * a.G * a.T + t0q) * D + c;
+#pragma unroll
+        for (int r = 0; r < 64; ++r) {
+          const int R = 64 * h + r;
+          const int tok = R / a.G;
+          if (tok < ntok)
+            red_add_f32(base + (R - tok * a.G) * hs + tok * D, __uint_as_float(o[r]));
+        }
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kSeqHThreads, 1)
     moda_bwd_seq_h_kernel(const __grid_constant__ CUtensorMap tmQ,
                           const __grid_constant__ CUtensorMap tmDO,
                           const __grid_constant__ CUtensorMap tmK,
-                          const __grid_constant__ CUtensorMap tmV,
-                          const __grid_constant__ CUtensorMap tmDQh, const SeqArgs a) {
+                          const __grid_constant__ CUtensorMap tmV, const SeqArgs a) {
   constexpr int D = 128;
   using Cfg = SeqCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -637,7 +704,7 @@ __global__ void __launch_bounds__(kSeqThreads, 1)
       mbar_init(bar(bars->do_empty[i]), 1);
       mbar_init(bar(bars->s_full[i]), 1);
       mbar_init(bar(bars->dp_full[i]), 1);
-      mbar_init(bar(bars->pds_full[i]), 128);
+      mbar_init(bar(bars->pds_full[i]), 256);
       mbar_init(bar(bars->dq_full[i]), 1);
       mbar_init(bar(bars->dq_free[i]), 128);
     }
@@ -657,7 +724,7 @@ __global__ void __launch_bounds__(kSeqThreads, 1)
       }
     fence_proxy_async_smem();
   }
-  if (warp == 9) {
+  if (warp == 13) {
     tmem_alloc(smem_u32(&bars->tmem_base), 512);
     tmem_relinquish();
   }
@@ -669,7 +736,7 @@ __global__ void __launch_bounds__(kSeqThreads, 1)
   auto tB = [&](int h) { return tmem + uint32_t(128 + 64 * h); };
   const uint32_t tDV = tmem + 256, tDK = tmem + 384;
 
-  if (warp == 8) {
+  if (warp == 12) {
     // ------------------------------------------------------------ TMA producer
     if (elect_one()) {
       tma_prefetch_desc(&tmQ);
@@ -698,7 +765,7 @@ __global__ void __launch_bounds__(kSeqThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 9) {
+  } else if (warp == 13) {
     // ------------------------------------------------------------ tcgen05 issuer
     if (elect_one()) {
       constexpr uint32_t idesc_t = make_idesc_bf16(128, 64, 0, 0);  // S^T_h, dP^T_h
@@ -769,13 +836,15 @@ __global__ void __launch_bounds__(kSeqThreads, 1)
       for (int i = 0; i < ntiles; ++i) {
         const bool more = i + 1 < ntiles;
         issue_grads(i, 0);
-        if (more) issue_dp(i + 1, 0);
+        if (more) {
+          issue_dp(i + 1, 0);
+          mbar_wait(bar(bars->dq_free[0]), i & 1, abort_flag);
+          issue_s(i + 1, 0);
+        }
         issue_grads(i, 1);
         tc_commit(bar(bars->do_empty[i & 1]));
         tc_commit(bar(bars->q_empty[i & 1]));
         if (more) {
-          mbar_wait(bar(bars->dq_free[0]), i & 1, abort_flag);
-          issue_s(i + 1, 0);
           issue_dp(i + 1, 1);
           mbar_wait(bar(bars->dq_free[1]), i & 1, abort_flag);
           issue_s(i + 1, 1);
@@ -784,31 +853,39 @@ __global__ void __launch_bounds__(kSeqThreads, 1)
       tc_commit(bar(bars->kv_done));
     }
     __syncwarp();
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     // ------------------------------------------------------------ P / dS warps
-    const int tid = threadIdx.x;  // TMEM lane = key key0 + tid
-    const int key = key0 + tid;
-    const uint32_t lane_base = uint32_t(warp * 32) << 16;
-    const int hl = tid % a.G, tok = tid / a.G;
-    auto load_rowterms = [&](int i, float& nl, float& nd) {
+    // Two warps per TMEM sub-partition: warp w owns key lanes 32(w%4)..32(w%4)+31 and, in
+    // each 64-row half, the 32-row chunk g = w/4.
+    const int g = warp >> 2;
+    const int kt = threadIdx.x & 127;  // TMEM lane = key key0 + kt
+    const int key = key0 + kt;
+    const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
+    // Row terms (lse, D) of the next tile, loaded by group 0 (row = kt) one tile ahead and
+    // transformed only when stored, so that the loads' latency stays hidden.
+    const int hl = kt % a.G, tok = kt / a.G;
+    float raw_l = 0.f, raw_d = 0.f;
+    bool raw_valid = false;
+    auto load_rowterms = [&](int i) {
       const int t = (first_qt + i) * a.TQ + tok;
-      const bool valid = i < ntiles && tok < a.TQ && t < a.T;
-      const long long idx = ((long long)bg * a.G + hl) * a.T + (valid ? t : 0);
-      nl = valid ? -a.lse[idx] * kLog2eBwd : -INFINITY;  // stored negated
-      nd = valid ? -a.drow[idx] : 0.f;                   // stored negated
+      raw_valid = i < ntiles && tok < a.TQ && t < a.T;
+      const long long idx = ((long long)bg * a.G + hl) * a.T + (raw_valid ? t : 0);
+      raw_l = a.lse[idx];
+      raw_d = a.drow[idx];
     };
-    float nxt_lse, nxt_d;
-    load_rowterms(0, nxt_lse, nxt_d);
+    if (g == 0) load_rowterms(0);
     const float2 sl2 = make_float2(a.scale_log2, a.scale_log2);
     const float2 sc2 = make_float2(a.scale, a.scale);
     const float2 neg1 = make_float2(-1.f, -1.f);
     for (int i = 0; i < ntiles; ++i) {
       const int qt = first_qt + i;
       const int b = i & 1;
-      ld_s[b * 256 + tid] = nxt_lse;
-      ld_s[b * 256 + 128 + tid] = nxt_d;
-      named_bar_sync(1, 128);
-      load_rowterms(i + 1, nxt_lse, nxt_d);
+      if (g == 0) {
+        ld_s[b * 256 + kt] = raw_valid ? -raw_l * kLog2eBwd : -INFINITY;  // stored negated
+        ld_s[b * 256 + 128 + kt] = raw_valid ? -raw_d : 0.f;              // stored negated
+      }
+      named_bar_sync(1, 256);
+      if (g == 0) load_rowterms(i + 1);
       int r_min = 0;
       if (key >= a.T)
         r_min = 1 << 30;
@@ -821,17 +898,21 @@ __global__ void __launch_bounds__(kSeqThreads, 1)
         mbar_wait(bar(bars->s_full[h]), i & 1, abort_flag);
         mbar_wait(bar(bars->dp_full[h]), i & 1, abort_flag);
         tc_fence_after();
-#pragma unroll 1
-        for (int cl = 0; cl < 2; ++cl) {
-          const int c = 2 * h + cl;  // 32-row chunk of the tile
-          uint32_t s[32], dp[32];
-          tmem_ld32(tA(h) + lane_base + cl * 32, s);
-          tmem_ld32(tB(h) + lane_base + cl * 32, dp);
-          tmem_wait_ld();
-          uint32_t pp[16], pl[16], pd[16], dl[16];
-          const bool masked = r_min > c * 32;
+        const int c = 2 * h + g;  // 32-row chunk of the tile
+        // the packed results overwrite these columns: load all 32 before storing any
+        uint32_t s[32], dp[32];
+        tmem_ld32(tA(h) + lane_base + g * 32, s);
+        tmem_ld32(tB(h) + lane_base + g * 32, dp);
+        tmem_wait_ld();
+        const bool masked = r_min > c * 32;
+        // dS for the dQ^T product: region h, this key's row, rows 32g..32g+31 of the half
+        const uint32_t reg = sDS + h * kBwdRegion + uint32_t(kt) * 128;
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
+        for (int k = 0; k < 2; ++k) {  // 16-row sub-chunks
+          uint32_t pp[8], pl[8], pd[8], dl[8];
+#pragma unroll
+          for (int e2 = 0; e2 < 16; e2 += 2) {
+            const int e = 16 * k + e2;
             const int r = c * 32 + e;
             const float2 arg = ffma2(
                 make_float2(__uint_as_float(s[e]), __uint_as_float(s[e + 1])), sl2,
@@ -850,21 +931,20 @@ __global__ void __launch_bounds__(kSeqThreads, 1)
             const float2 plo =
                 ffma2(make_float2(bf16lo(ph), bf16hi(ph)), neg1, make_float2(P0, P1));
             const float2 dlo = ffma2(make_float2(bf16lo(dh), bf16hi(dh)), neg1, dS);
-            pp[e / 2] = ph;
-            pl[e / 2] = pack_bf16x2(plo.x, plo.y);
-            pd[e / 2] = dh;
-            dl[e / 2] = pack_bf16x2(dlo.x, dlo.y);
+            pp[e2 / 2] = ph;
+            pl[e2 / 2] = pack_bf16x2(plo.x, plo.y);
+            pd[e2 / 2] = dh;
+            dl[e2 / 2] = pack_bf16x2(dlo.x, dlo.y);
           }
-          tmem_st16(tA(h) + lane_base + cl * 32, pp);
-          tmem_st16(tA(h) + lane_base + cl * 32 + 16, pl);
-          tmem_st16(tB(h) + lane_base + cl * 32, pd);
-          tmem_st16(tB(h) + lane_base + cl * 32 + 16, dl);
-          // dS for the dQ^T product: region h, this key's row, rows 32cl..32cl+31 of the half
-          const uint32_t reg = sDS + h * kBwdRegion + uint32_t(tid) * 128;
+          // packed P^T / dS^T words: hi at chunk column 8k.., lo 16 columns further
+          tmem_st8(tA(h) + lane_base + g * 32 + 8 * k, pp);
+          tmem_st8(tA(h) + lane_base + g * 32 + 16 + 8 * k, pl);
+          tmem_st8(tB(h) + lane_base + g * 32 + 8 * k, pd);
+          tmem_st8(tB(h) + lane_base + g * 32 + 16 + 8 * k, dl);
 #pragma unroll
-          for (int qd = 0; qd < 4; ++qd) {
-            const uint32_t chunk = cl * 4 + qd;
-            sts128(reg + ((chunk ^ (tid & 7)) << 4),
+          for (int qd = 0; qd < 2; ++qd) {
+            const uint32_t chunk = g * 4 + 2 * k + qd;
+            sts128(reg + ((chunk ^ (uint32_t(kt) & 7u)) << 4),
                    make_uint4(pd[qd * 4], pd[qd * 4 + 1], pd[qd * 4 + 2], pd[qd * 4 + 3]));
           }
         }
@@ -874,15 +954,14 @@ __global__ void __launch_bounds__(kSeqThreads, 1)
         mbar_arrive(bar(bars->pds_full[h]));
       }
     }
-    // epilogue: dV, dK rows of this key
+    // epilogue: group 0 writes this key's dV row, group 1 its dK row
     mbar_wait(bar(bars->kv_done), 0, abort_flag);
     tc_fence_after();
     const bool kvalid = key < a.T;
     const long long koff = ((long long)bg * a.T + (kvalid ? key : 0)) * D;
-#pragma unroll 1
-    for (int which = 0; which < 2; ++which) {
-      const uint32_t tsrc = (which ? tDK : tDV) + lane_base;
-      __nv_bfloat16* dst = (which ? a.dk : a.dv) + koff;
+    {
+      const uint32_t tsrc = (g ? tDK : tDV) + lane_base;
+      __nv_bfloat16* dst = (g ? a.dk : a.dv) + koff;
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t o[32];
@@ -901,67 +980,25 @@ __global__ void __launch_bounds__(kSeqThreads, 1)
       }
     }
   } else {
-    // ------------------------------------------------------------ dQ warps 4-7
-    // Thread = TMEM lane = head-dimension index c of dQ^T_h.  Two rounds per half: the
-    // threads of columns [64rd, 64rd+64) write their 64 row values into the half's dS
-    // region as row-major fp32 [64 rows][64 columns]; then 64 threads each hand one row
-    // (256 bytes) to a bulk reduce-add.
-    const int c = threadIdx.x - 128;
+    // ------------------------------------------------------------ dQ warps 8-11
+    // Thread = TMEM lane = head-dimension index c of dQ^T_h: it reads its 64 row values,
+    // frees the TMEM region, and adds them to the fp32 accumulator with global
+    // reductions (a warp covers 32 consecutive columns of one row: 128 bytes).
+    const int c = threadIdx.x - 256;
     const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
-    for (int i = 0; i < ntiles; ++i) {
-      const int t0q = (first_qt + i) * a.TQ;
-#pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-        mbar_wait(bar(bars->dq_full[h]), i & 1, abort_flag);
-        tc_fence_after();
-        uint32_t o[64];
-        tmem_ld32(tA(h) + lane_base, o);
-        tmem_ld32(tA(h) + lane_base + 32, o + 32);
-        tmem_wait_ld();
-        const uint32_t stage = sDS + h * kBwdRegion;
-#pragma unroll 1
-        for (int rd = 0; rd < 2; ++rd) {
-          if ((c >> 6) == rd) {
-            const uint32_t col = uint32_t(c & 63) * 4;
-#pragma unroll
-            for (int row = 0; row < 64; ++row)
-              asm volatile("st.shared.b32 [%0], %1;" ::"r"(stage + row * 256 + col),
-                           "r"(o[row])
-                           : "memory");
-          }
-          fence_proxy_async_smem();
-          named_bar_sync(2, 128);
-          if (a.half_box) {
-            // the half's 64 rows are whole tokens: one tensor box (64 columns x G heads x
-            // 64/G tokens) covers the staged rows
-            if (c == 0) {
-              tma_reduce_add_4d(&tmDQh, stage, 64 * rd, 0, t0q + (64 * h) / a.G, bg);
-              bulk_commit_group();
-              bulk_wait_read_all();
-            }
-          } else if (c < 64) {
-            const int R = 64 * h + c;  // tile row
-            const int tok = R / a.G, hl = R - (R / a.G) * a.G;
-            const int t = t0q + tok;
-            if (tok < a.TQ && t < a.T) {
-              float* dst = a.dqacc + (((long long)bg * a.G + hl) * a.T + t) * D + 64 * rd;
-              bulk_reduce_add_f32(dst, stage + c * 256, 256);
-            }
-            bulk_commit_group();
-            bulk_wait_read_all();
-          }
-          named_bar_sync(2, 128);
-        }
-        tc_fence_before();
-        mbar_arrive(bar(bars->dq_free[h]));
-      }
+    switch (a.G) {
+      case 1: dq_readout<1>(a, bars, tmem, lane_base, c, bg, first_qt, ntiles); break;
+      case 2: dq_readout<2>(a, bars, tmem, lane_base, c, bg, first_qt, ntiles); break;
+      case 4: dq_readout<4>(a, bars, tmem, lane_base, c, bg, first_qt, ntiles); break;
+      case 8: dq_readout<8>(a, bars, tmem, lane_base, c, bg, first_qt, ntiles); break;
+      case 16: dq_readout<16>(a, bars, tmem, lane_base, c, bg, first_qt, ntiles); break;
+      default: dq_readout<0>(a, bars, tmem, lane_base, c, bg, first_qt, ntiles); break;
     }
-    if (c < 64) bulk_wait_all();  // (thread 0 also covers the tensor-box path)
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 13) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -1130,24 +1167,6 @@ cudaError_t launch_backward_d(const Problem& p, const void* q, const void* k, co
     return e;
   }
   const int nkb = (p.T + 127) / 128;
-  sa.half_box = (64 % p.G) == 0;
-  CUtensorMap mDQh = mDQ;
-  if (sa.half_box) {
-    // fp32 dq accumulator as [bg][t][head-in-group][c]: one box = 64 columns (256 bytes,
-    // no swizzle) of the 64/G tokens x G heads of a half tile, row-major like the staging
-    const cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(p.G), cuuint64_t(p.T), BG};
-    const cuuint64_t str[3] = {cuuint64_t(p.T) * D * 4, cuuint64_t(D) * 4,
-                               cuuint64_t(p.G) * p.T * D * 4};
-    const cuuint32_t box[4] = {64, cuuint32_t(p.G), cuuint32_t(64 / p.G), 1};
-    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-    if (encode(&mDQh, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dqacc, dims, str, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
-      *why = "cuTensorMapEncodeTiled failed for the dq accumulator (half tiles)";
-      return cudaErrorInvalidValue;
-    }
-  }
   if ((stages & kStageSeq) && D == 128) {
     e = cudaFuncSetAttribute(moda_bwd_seq_h_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              SeqCfg<128>::kSmemBytes);
@@ -1155,8 +1174,8 @@ cudaError_t launch_backward_d(const Problem& p, const void* q, const void* k, co
       *why = "cudaFuncSetAttribute(sequence backward, halves) failed";
       return e;
     }
-    moda_bwd_seq_h_kernel<<<unsigned(BG) * nkb, kSeqThreads, SeqCfg<128>::kSmemBytes,
-                            stream>>>(mQ, mDO, mK, mV, mDQh, sa);
+    moda_bwd_seq_h_kernel<<<unsigned(BG) * nkb, kSeqHThreads, SeqCfg<128>::kSmemBytes,
+                            stream>>>(mQ, mDO, mK, mV, sa);
   } else if (stages & kStageSeq) {
     moda_bwd_seq_kernel<D><<<unsigned(BG) * nkb, kSeqThreads, SeqCfg<D>::kSmemBytes, stream>>>(
       mQ, mDO, mK, mV, mDQ, sa);
