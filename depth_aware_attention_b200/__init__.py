@@ -29,7 +29,7 @@ MODA_ERR_INTERNAL = 5
 BACKWARD_LAUNCHES = 3
 
 # Every symbol include/moda.h declares (checked by the ABI tests).
-EXPORTED = ("moda_forward", "moda_backward", "moda_backward_workspace_size",
+EXPORTED = ("moda_forward", "moda_forward_depth_path", "moda_backward", "moda_backward_workspace_size",
             "moda_backward_stages", "moda_backward_noalloc", "moda_check_device_errors", "moda_status_string",
             "moda_last_error_message")
 
@@ -49,6 +49,8 @@ def _load():
     P, I, F, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     lib.moda_forward.argtypes = [P] * 7 + [I] * 6 + [F, I, P]
     lib.moda_forward.restype = I
+    lib.moda_forward_depth_path.argtypes = [P] * 7 + [I] * 6 + [F, I, I, P]
+    lib.moda_forward_depth_path.restype = I
     lib.moda_backward_workspace_size.argtypes = [I] * 6
     lib.moda_backward_workspace_size.restype = S
     lib.moda_backward.argtypes = [P] * 14 + [S] + [I] * 6 + [F, I, P]
@@ -85,6 +87,13 @@ def moda_forward(q, k, v, kd, vd, out, lse, B, Hq, Hkv, T, L, d, scale, causal, 
     """Direct call of the C entry point with raw pointers (ints) and a stream handle."""
     return lib.moda_forward(q, k, v, kd, vd, out, lse, B, Hq, Hkv, T, L, d, float(scale),
                             int(causal), stream)
+
+
+def moda_forward_depth_path(q, k, v, kd, vd, out, lse, B, Hq, Hkv, T, L, d, scale, causal,
+                            depth_path, stream):
+    """Direct call of moda_forward_depth_path with raw pointers (ints) and a stream handle."""
+    return lib.moda_forward_depth_path(q, k, v, kd, vd, out, lse, B, Hq, Hkv, T, L, d,
+                                       float(scale), int(causal), int(depth_path), stream)
 
 
 def moda_backward(q, k, v, kd, vd, out, lse, dout, dq, dk, dv, dkd, dvd, workspace,
@@ -140,11 +149,14 @@ def _dims(q, k, kd):
     return B, Hq, Hkv, T, L, d
 
 
-def forward(q, k, v, kd=None, vd=None, scale=None, causal=True, out=None, lse=None):
+def forward(q, k, v, kd=None, vd=None, scale=None, causal=True, out=None, lse=None,
+            depth_path=0):
     """MoDA forward on the current CUDA stream.  Returns (out bf16, lse fp32).
 
     q [B,Hq,T,d], k/v [B,Hkv,T,d], kd/vd [B,Hkv,T,L,d] (or None for L = 0): contiguous
-    bf16 CUDA tensors.  scale defaults to 1/sqrt(d).
+    bf16 CUDA tensors.  scale defaults to 1/sqrt(d).  ``depth_path`` 0 lets the library
+    choose; 1 forces the CUDA-core depth fold, 2 dense depth blocks on the tensor cores
+    (moda_forward_depth_path).
     """
     import torch
     B, Hq, Hkv, T, L, d = _dims(q, k, kd)
@@ -154,10 +166,14 @@ def forward(q, k, v, kd=None, vd=None, scale=None, causal=True, out=None, lse=No
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, Hq, T), device=q.device, dtype=torch.float32)
-    st = lib.moda_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(kd) if L else None,
-                          _ptr(vd) if L else None, _ptr(out), _ptr(lse), B, Hq, Hkv, T, L,
-                          d, float(scale), int(bool(causal)), _stream_handle(q.device))
-    _check(st, "moda_forward")
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(kd) if L else None, _ptr(vd) if L else None,
+            _ptr(out), _ptr(lse), B, Hq, Hkv, T, L, d, float(scale), int(bool(causal)))
+    if depth_path == 0:
+        st = lib.moda_forward(*args, _stream_handle(q.device))
+        _check(st, "moda_forward")
+    else:
+        st = lib.moda_forward_depth_path(*args, int(depth_path), _stream_handle(q.device))
+        _check(st, "moda_forward_depth_path")
     return out, lse
 
 

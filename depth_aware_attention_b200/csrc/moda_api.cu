@@ -103,13 +103,15 @@ const char* moda_status_string(moda_status_t status) {
 
 const char* moda_last_error_message(void) { return g_msg; }
 
-moda_status_t moda_forward(const void* q, const void* k, const void* v, const void* kd,
-                           const void* vd, void* out, float* lse, int B, int Hq, int Hkv,
-                           int T, int L, int d, float scale, int causal,
-                           moda_stream_t stream) {
+static moda_status_t forward_entry(const void* q, const void* k, const void* v,
+                                   const void* kd, const void* vd, void* out, float* lse,
+                                   int B, int Hq, int Hkv, int T, int L, int d, float scale,
+                                   int causal, int depth_path, moda_stream_t stream) {
   g_msg[0] = 0;
   moda_status_t s = check_sizes(B, Hq, Hkv, T, L, d);
   if (s != MODA_OK) return s;
+  if (depth_path < moda::kDepthPathAuto || depth_path > moda::kDepthPathDense)
+    return fail(MODA_ERR_INVALID_ARGUMENT, "depth_path must be 0, 1 or 2");
   if (!q || !k || !v || !out || !lse)
     return fail(MODA_ERR_INVALID_ARGUMENT, "q, k, v, out and lse must be non-NULL");
   if (L > 0 && (!kd || !vd))
@@ -128,19 +130,38 @@ moda_status_t moda_forward(const void* q, const void* k, const void* v, const vo
       return fail(MODA_ERR_INVALID_ARGUMENT, "out/lse must not overlap an input");
   if (overlaps(out, nq, lse, nl))
     return fail(MODA_ERR_INVALID_ARGUMENT, "out and lse must not overlap");
+  moda::Problem p{B, Hq, Hkv, T, L, d, Hq / Hkv, causal ? 1 : 0, scale};
+  if (depth_path == moda::kDepthPathDense && !moda::dense_depth_supported(p))
+    return fail(MODA_ERR_UNSUPPORTED, "dense depth blocks need Hq/Hkv to divide 128");
   s = check_device();
   if (s != MODA_OK) return s;
   moda::EncodeTiledFn enc = get_encoder();
   if (!enc) return fail(MODA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
-  moda::Problem p{B, Hq, Hkv, T, L, d, Hq / Hkv, causal ? 1 : 0, scale};
   const char* why = "";
-  cudaError_t e = moda::launch_forward(p, q, k, v, kd, vd, out, lse, enc,
+  cudaError_t e = moda::launch_forward(p, q, k, v, kd, vd, out, lse, depth_path, enc,
                                        static_cast<cudaStream_t>(stream), &why);
   if (e != cudaSuccess) {
     snprintf(g_msg, sizeof(g_msg), "%s: %s", why, cudaGetErrorString(e));
     return MODA_ERR_CUDA;
   }
   return MODA_OK;
+}
+
+moda_status_t moda_forward(const void* q, const void* k, const void* v, const void* kd,
+                           const void* vd, void* out, float* lse, int B, int Hq, int Hkv,
+                           int T, int L, int d, float scale, int causal,
+                           moda_stream_t stream) {
+  return forward_entry(q, k, v, kd, vd, out, lse, B, Hq, Hkv, T, L, d, scale, causal,
+                       moda::kDepthPathAuto, stream);
+}
+
+moda_status_t moda_forward_depth_path(const void* q, const void* k, const void* v,
+                                      const void* kd, const void* vd, void* out, float* lse,
+                                      int B, int Hq, int Hkv, int T, int L, int d,
+                                      float scale, int causal, int depth_path,
+                                      moda_stream_t stream) {
+  return forward_entry(q, k, v, kd, vd, out, lse, B, Hq, Hkv, T, L, d, scale, causal,
+                       depth_path, stream);
 }
 
 size_t moda_backward_workspace_size(int B, int Hq, int Hkv, int T, int L, int d) {

@@ -11,16 +11,27 @@
 // G heads of the group ("group-aware"), and a tile reads only its own tokens' TQ x L depth
 // rows ("chunk-aware"), each byte once.  Both tiles consume every K/V block the CTA loads.
 //
+// Two depth paths (template flag kDense), the same operator:
+//   dense (default when G divides 128): a tile's depth rows go through the tensor-core
+//            pipeline ahead of its sequence blocks, as extra 128-key blocks of G entries
+//            of each of the tile's 128/G tokens (token-major).  Row r only sees its own
+//            token's G keys, so most of each depth block's products are masked away; the
+//            tensor cores have the FLOPs to spare, and the depth rows then stream through
+//            the same TMA ring as K/V at the rate HBM delivers them.
+//   fold:    the depth logits q.kd are computed on CUDA cores from the tile's depth
+//            chunks, folded into (m, l) with the P.vd sums accumulated in registers and
+//            stored into TMEM as O's starting value, before the sequence blocks.
+//
 // Warp roles (320 threads):
 //   warps 0-3 / 4-7  tile 0 / tile 1 compute warps: thread r owns row r of its tile (TMEM
-//            lane r).  First the depth fold: logits q.kd on CUDA cores from the tile's
-//            depth chunks, folded into (m, l) with the P.vd sums accumulated in registers
-//            and stored into TMEM as O's starting value.  Then per sequence block: S row
-//            from TMEM -> mask -> exp2 -> P (bf16) back into TMEM over S; O is rescaled
-//            only when the row max grows by more than 2^8.  Last the epilogue.
-//   warp 8   TMA producer: lane 0 streams the Q tiles and the K/V blocks through the K/V
-//            ring; lanes 1 and 2 stream tile 0's and tile 1's depth chunks through their
-//            own depth rings.  Every ring has exactly one in-order consumer.
+//            lane r).  Fold path: the depth fold first.  Then per block (depth blocks of
+//            the dense path, then sequence blocks): S row from TMEM -> mask -> exp2 -> P
+//            (bf16) back into TMEM over S; O is rescaled only when the row max grows by
+//            more than 2^8.  Last the epilogue.
+//   warp 8   TMA producer: lane 0 streams the Q tiles and the K/V blocks (dense path:
+//            preceded by each depth step's kd/vd blocks of both tiles) through the K/V
+//            ring; fold path: lanes 1 and 2 stream tile 0's and tile 1's depth chunks
+//            through their own depth rings.  Every ring has exactly one in-order consumer.
 //   warp 9   tcgen05 issuer, in the order S0(0) S1(0) { PV0(j) S0(j+1) PV1(j) S1(j+1) }:
 //            while one tile's warps turn S into P, the tensor cores work for the other
 //            tile.  Because S_t(j+1) is issued after PV_t(j), a tile's warps that have
@@ -47,12 +58,15 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only past 256x
 constexpr int kFwdThreads = 320;
 
-template <int D>
+// kDense selects the depth path: false = CUDA-core fold from two depth rings, true =
+// depth blocks through the K/V ring on the tensor cores (see the kernel comment).
+template <int D, bool kDense>
 struct FwdCfg {
   static constexpr int kRegions = D / 64;                // 64-column swizzled regions
   static constexpr int kTileBytes = kRegions * kRegion;  // one Q tile / one K or V block
-  static constexpr int kKV = (D == 128) ? 3 : 4;         // K/V ring stages
-  static constexpr int kDS = (D == 128) ? 2 : 3;         // stages per depth ring (16 KB each)
+  // K/V ring stages; the dense path has no depth rings and spends their room here
+  static constexpr int kKV = kDense ? ((D == 128) ? 5 : 8) : ((D == 128) ? 3 : 4);
+  static constexpr int kDS = kDense ? 0 : ((D == 128) ? 2 : 3);  // stages per depth ring
   static constexpr int kOffQ = 0;                        // two Q tiles
   static constexpr int kOffKV = 2 * kTileBytes;
   static constexpr int kOffD = kOffKV + kKV * kTileBytes;  // two depth rings
@@ -69,8 +83,8 @@ struct FwdArgs {
 
 struct Bars {
   uint64_t q_full;
-  uint64_t full[4];       // K/V ring: data landed
-  uint64_t empty[4];      // K/V ring: stage released by the tensor cores
+  uint64_t full[8];       // K/V ring: data landed
+  uint64_t empty[8];      // K/V ring: stage released by the tensor cores
   uint64_t dfull[2][3];   // depth ring of tile t: data landed
   uint64_t dempty[2][3];  // depth ring of tile t: stage released by tile t's warps
   uint64_t s_full[2];     // S_t(j) in TMEM
@@ -92,14 +106,14 @@ __device__ __forceinline__ float dot8(const float (&a)[8], uint4 w) {
   return s;
 }
 
-template <int D>
+template <int D, bool kDense>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     moda_fwd_kernel(const __grid_constant__ CUtensorMap tmQ,
                     const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV,
                     const __grid_constant__ CUtensorMap tmKD,
                     const __grid_constant__ CUtensorMap tmVD, const FwdArgs a) {
-  using Cfg = FwdCfg<D>;
+  using Cfg = FwdCfg<D, kDense>;
   constexpr int NKV = Cfg::kKV;
   constexpr int NDS = Cfg::kDS;
   extern __shared__ uint8_t smem_raw[];
@@ -121,9 +135,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const int NB0 = ((a.causal ? min(a.T, tq0 + a.TQ) : a.T) + kBN - 1) / kBN;
   // NB0 <= NB1; a tile 1 past the end of the sequence is computed but never stored
   const int NB1 = tq1 >= a.T ? NB0 : ((a.causal ? min(a.T, tq1 + a.TQ) : a.T) + kBN - 1) / kBN;
-  const int NC = a.L > 0 ? (a.L + a.JC - 1) / a.JC : 0;
-  const bool has_depth = NC > 0;
+  const bool has_depth = a.L > 0;
+  const int nchunk = has_depth ? (a.L + a.JC - 1) / a.JC : 0;
+  const int NC = kDense ? 0 : nchunk;  // CUDA-core fold chunks
+  const int ND = kDense ? nchunk : 0;  // tensor-core depth steps (ahead of the sequence)
+  const int N0 = ND + NB0, N1 = ND + NB1;  // steps of tile 0 / tile 1
   constexpr int kDUses = 2 * Cfg::kRegions;   // depth stage uses per chunk: kd, vd regions
+  // Ring entries in load order.  Depth step j: kd of tile 0, kd of tile 1, vd of tile 0,
+  // vd of tile 1; sequence block j: K then V, shared by both tiles.
+  auto kidx = [&](int t, int j) { return j < ND ? 4 * j + t : 4 * ND + 2 * (j - ND); };
+  auto vidx = [&](int t, int j) { return j < ND ? 4 * j + 2 + t : 4 * ND + 2 * (j - ND) + 1; };
 
   if (threadIdx.x == 0) {
     mbar_init(bar(bars->q_full), 1);
@@ -175,16 +196,33 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int rg = 0; rg < Cfg::kRegions; ++rg)
           tma_load_4d(sQ(t) + rg * kRegion, &tmQ, bar(bars->q_full), rg * 64, 0,
                       t ? tq1 : tq0, bg);
+      int e = 0;  // ring entry
+      auto acquire = [&](int bytes) {
+        const int s = e % NKV;
+        if (e >= NKV) mbar_wait(bar(bars->empty[s]), ((e / NKV) - 1) & 1, abort_flag);
+        mbar_expect_tx(bar(bars->full[s]), uint32_t(bytes));
+        ++e;
+        return s;
+      };
+      if constexpr (kDense) {
+        // depth chunk j of a tile: entries [j*JC, j*JC+JC) of its TQ tokens, token-major
+        for (int j = 0; j < ND; ++j)
+          for (int u = 0; u < 4; ++u) {
+            const int s = acquire(Cfg::kTileBytes);
+            const CUtensorMap* map = (u < 2) ? &tmKD : &tmVD;
+            for (int rg = 0; rg < Cfg::kRegions; ++rg)
+              tma_load_4d(sKV(s) + rg * kRegion, map, bar(bars->full[s]), rg * 64, j * a.JC,
+                          (u & 1) ? tq1 : tq0, bg);
+          }
+      }
       for (int idx = 0; idx < 2 * NB1; ++idx) {
-        const int s = idx % NKV;
-        if (idx >= NKV) mbar_wait(bar(bars->empty[s]), ((idx / NKV) - 1) & 1, abort_flag);
+        const int s = acquire(Cfg::kTileBytes);
         const CUtensorMap* map = (idx & 1) ? &tmV : &tmK;
-        mbar_expect_tx(bar(bars->full[s]), Cfg::kTileBytes);
         for (int rg = 0; rg < Cfg::kRegions; ++rg)
           tma_load_3d(sKV(s) + rg * kRegion, map, bar(bars->full[s]), rg * 64,
                       (idx >> 1) * kBN, bg);
       }
-    } else if ((lane == 1 || lane == 2) && has_depth) {
+    } else if constexpr (!kDense) if ((lane == 1 || lane == 2) && NC > 0) {
       // Depth chunk ci of tile t: entries [ci*JC, ci*JC+JC) of the tile's TQ tokens as
       // rows (token, entry), one 64-column region per stage: kd regions, then vd regions.
       const int t = lane - 1;
@@ -232,12 +270,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       constexpr uint32_t idesc_s = make_idesc_bf16(kBM, kBN, 0, 0);
       constexpr uint32_t idesc_o = make_idesc_bf16(kBM, D, 0, 1);
       mbar_wait(bar(bars->q_full), 0, abort_flag);
-      auto wait_kv = [&](int idx) {
-        mbar_wait(bar(bars->full[idx % NKV]), (idx / NKV) & 1, abort_flag);
+      auto wait_entry = [&](int e) {
+        mbar_wait(bar(bars->full[e % NKV]), (e / NKV) & 1, abort_flag);
         tc_fence_after();
       };
+      auto release = [&](int e) { tc_commit(bar(bars->empty[e % NKV])); };
+      // A sequence block's K and V are released after tile 1 (the last user) has read
+      // them; a depth block is its tile's own.
       auto issue_s = [&](int t, int j) {
-        const uint32_t kbase = sKV((2 * j) % NKV);
+        const int e = kidx(t, j);
+        wait_entry(e);
+        const uint32_t kbase = sKV(e % NKV);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t off = (ks / 4) * kRegion + (ks % 4) * 32;
@@ -245,42 +288,32 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                  make_sdesc_sw128(kbase + off, 16, 1024), idesc_s, ks > 0 ? 1u : 0u);
         }
         tc_commit(bar(bars->s_full[t]));
+        if (j < ND || t == 1) release(e);
       };
       auto issue_pv = [&](int t, int j) {
         mbar_wait(bar(bars->p_full[t]), j & 1, abort_flag);
-        tc_fence_after();
-        const uint32_t vbase = sKV((2 * j + 1) % NKV);
+        const int e = vidx(t, j);
+        wait_entry(e);
+        const uint32_t vbase = sKV(e % NKV);
         const uint32_t tO = tmem + 256 + t * D;
 #pragma unroll
         for (int ks = 0; ks < kBN / 16; ++ks)
           mma_ts(tO, tmem + t * 128 + ks * 8,
                  make_sdesc_sw128(vbase + ks * 2048, kRegion, 1024), idesc_o,
-                 (ks > 0 || j > 0 || has_depth) ? 1u : 0u);
+                 (ks > 0 || j > 0 || NC > 0) ? 1u : 0u);
+        if (j < ND || t == 1) release(e);
       };
-      wait_kv(0);
       issue_s(0, 0);
       issue_s(1, 0);
-      tc_commit(bar(bars->empty[0]));
-      for (int j = 0; j < NB1; ++j) {
-        wait_kv(2 * j + 1);
-        bool k_next_ready = false;
-        if (j < NB0) {
+      for (int j = 0; j < N1; ++j) {
+        if (j < N0) {
           issue_pv(0, j);
-          if (j == NB0 - 1) tc_commit(bar(bars->o_final[0]));
-          if (j + 1 < NB0) {
-            wait_kv(2 * j + 2);
-            k_next_ready = true;
-            issue_s(0, j + 1);
-          }
+          if (j == N0 - 1) tc_commit(bar(bars->o_final[0]));
+          if (j + 1 < N0) issue_s(0, j + 1);
         }
         issue_pv(1, j);
-        tc_commit(bar(bars->empty[(2 * j + 1) % NKV]));
-        if (j == NB1 - 1) tc_commit(bar(bars->o_final[1]));
-        if (j + 1 < NB1) {
-          if (!k_next_ready) wait_kv(2 * j + 2);
-          issue_s(1, j + 1);
-          tc_commit(bar(bars->empty[(2 * j + 2) % NKV]));
-        }
+        if (j == N1 - 1) tc_commit(bar(bars->o_final[1]));
+        if (j + 1 < N1) issue_s(1, j + 1);
       }
     }
     __syncwarp();
@@ -297,13 +330,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const uint32_t tS = tmem + lane_base + tt * 128;
     const uint32_t tO = tmem + lane_base + 256 + tt * D;
     const uint32_t q_base = sQ(tt);
-    const int NB = tt ? NB1 : NB0;
+    const int NS = tt ? N1 : N0;  // steps of this tile
     const uint32_t wg_bar = 1 + tt;               // named barrier of this warpgroup
     float m = -INFINITY, l = 0.f;
 
     mbar_wait(bar(bars->q_full), 0, abort_flag);
 
-    if (has_depth) {
+    if constexpr (!kDense) if (NC > 0) {
       float acc[D];
 #pragma unroll
       for (int c = 0; c < D; ++c) acc[c] = 0.f;
@@ -385,30 +418,45 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       tmem_wait_st();
     }
 
-    // ---- sequence blocks
+    // ---- depth steps (dense path), then sequence blocks
+    // A depth step's 128 keys are JC = G entries of each of the tile's TQ tokens,
+    // token-major, so row r (token r / G) owns keys [r - hl, r - hl + G): all inside the
+    // 32 keys of its warp's rows.  Only those 32 columns are read; P is zero elsewhere.
     const int key_lim = a.causal ? t : a.T - 1;
-    for (int jb = 0; jb < NB; ++jb) {
+    for (int jb = 0; jb < NS; ++jb) {
       mbar_wait(bar(bars->s_full[tt]), jb & 1, abort_flag);
       tc_fence_after();
+      const bool dstep = kDense && jb < ND;
       uint32_t s[kBN];
-      tmem_ld32(tS + 0, &s[0]);
-      tmem_ld32(tS + 32, &s[32]);
-      tmem_ld32(tS + 64, &s[64]);
-      tmem_ld32(tS + 96, &s[96]);
-      tmem_wait_ld();
-      const int kbase = jb * kBN;
-      const bool need_mask = a.causal ? (kbase + kBN - 1 > t0) : (kbase + kBN > a.T);
-      // Row max on the raw scores (scale > 0 commutes with max); masked keys -> -inf.
-      float mx = -INFINITY;
-      if (need_mask) {
+      float mx = -INFINITY;  // row max on the raw scores (scale > 0); masked keys -> -inf
+      if (dstep) {
+        tmem_ld32(tS + 32 * (warp & 3), &s[0]);
+        tmem_wait_ld();
+        const int lo = (r & 31) - hl;
+        const int nval = min(a.JC, a.L - jb * a.JC);
 #pragma unroll
-        for (int c = 0; c < kBN; ++c) {
-          if (kbase + c > key_lim) s[c] = __float_as_uint(-INFINITY);
+        for (int c = 0; c < 32; ++c) {
+          if (c < lo || c >= lo + nval) s[c] = __float_as_uint(-INFINITY);
           mx = fmaxf(mx, __uint_as_float(s[c]));
         }
       } else {
+        tmem_ld32(tS + 0, &s[0]);
+        tmem_ld32(tS + 32, &s[32]);
+        tmem_ld32(tS + 64, &s[64]);
+        tmem_ld32(tS + 96, &s[96]);
+        tmem_wait_ld();
+        const int kbase = (jb - ND) * kBN;
+        const bool need_mask = a.causal ? (kbase + kBN - 1 > t0) : (kbase + kBN > a.T);
+        if (need_mask) {
 #pragma unroll
-        for (int c = 0; c < kBN; ++c) mx = fmaxf(mx, __uint_as_float(s[c]));
+          for (int c = 0; c < kBN; ++c) {
+            if (kbase + c > key_lim) s[c] = __float_as_uint(-INFINITY);
+            mx = fmaxf(mx, __uint_as_float(s[c]));
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < kBN; ++c) mx = fmaxf(mx, __uint_as_float(s[c]));
+        }
       }
       const float m_cand = fmaxf(m, mx * a.scale_log2);
       const bool grow = m_cand > m + kRescaleThreshold;
@@ -416,25 +464,50 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
       const float alpha = ex2(m - m_use);
       float ps0 = 0.f, ps1 = 0.f;
+      if (dstep) {
+        uint32_t pk[16];
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          // p = 2^(s*scale*log2e - m): one FFMA feeds each exp2
-          const float p0 = ex2(fmaf(__uint_as_float(s[half * 64 + c]), a.scale_log2, -m_use));
-          const float p1 = ex2(fmaf(__uint_as_float(s[half * 64 + c + 1]), a.scale_log2, -m_use));
+        for (int c = 0; c < 32; c += 2) {
+          const float p0 = ex2(fmaf(__uint_as_float(s[c]), a.scale_log2, -m_use));
+          const float p1 = ex2(fmaf(__uint_as_float(s[c + 1]), a.scale_log2, -m_use));
           ps0 += p0;
           ps1 += p1;
           pk[c / 2] = pack_bf16x2(p0, p1);
         }
-        tmem_st32(tS + half * 32, pk);
+        uint32_t zero[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) zero[c] = 0u;
+        // packed P columns [16q, 16q+16) hold keys [32q, 32q+32): this warp's are pk
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          if (q == (warp & 3))
+            tmem_st16(tS + 16 * q, pk);
+          else
+            tmem_st16(tS + 16 * q, zero);
+        }
+      } else {
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int c = 0; c < 64; c += 2) {
+            // p = 2^(s*scale*log2e - m): one FFMA feeds each exp2
+            const float p0 =
+                ex2(fmaf(__uint_as_float(s[half * 64 + c]), a.scale_log2, -m_use));
+            const float p1 =
+                ex2(fmaf(__uint_as_float(s[half * 64 + c + 1]), a.scale_log2, -m_use));
+            ps0 += p0;
+            ps1 += p1;
+            pk[c / 2] = pack_bf16x2(p0, p1);
+          }
+          tmem_st32(tS + half * 32, pk);
+        }
       }
       const float ps = ps0 + ps1;
       l = l * alpha + ps;
       m = m_new;
       // O_t holds every PV_t issued so far (S_t(jb) was issued after PV_t(jb-1)).
-      const bool has_o = has_depth || jb > 0;
+      const bool has_o = NC > 0 || jb > 0;
       if (__any_sync(0xffffffffu, grow && has_o)) {
         const float f = grow ? alpha : 1.f;
 #pragma unroll
@@ -505,12 +578,14 @@ bool make_map(EncodeTiledFn encode, CUtensorMap* map, const void* base, int rank
   return r == CUDA_SUCCESS;
 }
 
-template <int D>
+template <int D, bool kDense>
 cudaError_t launch_forward_d(const Problem& p, const void* q, const void* k, const void* v,
                              const void* kd, const void* vd, void* out, float* lse,
                              EncodeTiledFn encode, cudaStream_t stream, const char** why) {
-  using Cfg = FwdCfg<D>;
-  const TileGeom tg = tile_geom(p);
+  using Cfg = FwdCfg<D, kDense>;
+  TileGeom tg = tile_geom(p);
+  // a dense depth block is JC entries of each of the tile's TQ tokens: 128 keys
+  if (kDense) tg.JC = 128 / tg.TQ;
   const cuuint64_t E = 2;  // bytes per bf16
   const cuuint64_t BG = cuuint64_t(p.B) * p.Hkv;
   CUtensorMap mQ, mK, mV, mKD, mVD;
@@ -568,7 +643,7 @@ cudaError_t launch_forward_d(const Problem& p, const void* q, const void* k, con
   args.scale_log2 = p.scale * kLog2e;
 
   {
-    cudaError_t e = cudaFuncSetAttribute(moda_fwd_kernel<D>,
+    cudaError_t e = cudaFuncSetAttribute(moda_fwd_kernel<D, kDense>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          Cfg::kSmemBytes);
     if (e != cudaSuccess) {
@@ -577,8 +652,8 @@ cudaError_t launch_forward_d(const Problem& p, const void* q, const void* k, con
     }
   }
   const unsigned grid = unsigned(BG) * unsigned(args.npairs);
-  moda_fwd_kernel<D><<<grid, kFwdThreads, Cfg::kSmemBytes, stream>>>(mQ, mK, mV, mKD, mVD,
-                                                                      args);
+  moda_fwd_kernel<D, kDense><<<grid, kFwdThreads, Cfg::kSmemBytes, stream>>>(
+      mQ, mK, mV, mKD, mVD, args);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) *why = "forward kernel launch failed";
   return e;
@@ -586,12 +661,23 @@ cudaError_t launch_forward_d(const Problem& p, const void* q, const void* k, con
 
 }  // namespace
 
+bool dense_depth_supported(const Problem& p) { return 128 % p.G == 0; }
+
+bool dense_depth_default(const Problem& p) {
+  return dense_depth_supported(p) && p.L >= kDenseDepthMinL;
+}
+
 cudaError_t launch_forward(const Problem& p, const void* q, const void* k, const void* v,
                            const void* kd, const void* vd, void* out, float* lse,
-                           EncodeTiledFn encode, cudaStream_t stream, const char** why) {
+                           int depth_path, EncodeTiledFn encode, cudaStream_t stream,
+                           const char** why) {
+  const bool dense = depth_path == kDepthPathDense ||
+                     (depth_path == kDepthPathAuto && dense_depth_default(p));
   if (p.d == 128)
-    return launch_forward_d<128>(p, q, k, v, kd, vd, out, lse, encode, stream, why);
-  return launch_forward_d<64>(p, q, k, v, kd, vd, out, lse, encode, stream, why);
+    return dense ? launch_forward_d<128, true>(p, q, k, v, kd, vd, out, lse, encode, stream, why)
+                 : launch_forward_d<128, false>(p, q, k, v, kd, vd, out, lse, encode, stream, why);
+  return dense ? launch_forward_d<64, true>(p, q, k, v, kd, vd, out, lse, encode, stream, why)
+               : launch_forward_d<64, false>(p, q, k, v, kd, vd, out, lse, encode, stream, why);
 }
 
 }  // namespace moda

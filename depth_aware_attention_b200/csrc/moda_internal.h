@@ -40,10 +40,21 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion,
                                   CUtensorMapFloatOOBfill);
 
+// Forward depth paths: the CUDA-core fold (each tile's depth rows folded into the softmax
+// state on CUDA cores before its sequence blocks) or dense depth blocks (the depth rows
+// run through the tensor-core pipeline as extra masked 128-key blocks; needs G | 128).
+constexpr int kDepthPathAuto = 0, kDepthPathFold = 1, kDepthPathDense = 2;
+// The automatic choice takes dense depth blocks from this many depth entries up (measured
+// on B200: as fast or faster than the fold from L = 24 to 128, and at L = 32, 64K tokens).
+constexpr int kDenseDepthMinL = 1;
+bool dense_depth_supported(const Problem& p);
+bool dense_depth_default(const Problem& p);
+
 // Forward launcher: returns a CUDA error code (cudaSuccess when enqueued).
 cudaError_t launch_forward(const Problem& p, const void* q, const void* k, const void* v,
                            const void* kd, const void* vd, void* out, float* lse,
-                           EncodeTiledFn encode, cudaStream_t stream, const char** why);
+                           int depth_path, EncodeTiledFn encode, cudaStream_t stream,
+                           const char** why);
 
 cudaError_t launch_backward(const Problem& p, const void* q, const void* k, const void* v,
                             const void* kd, const void* vd, const void* out,

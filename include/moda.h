@@ -69,6 +69,28 @@ moda_status_t moda_forward(const void *q, const void *k, const void *v, const vo
                            moda_stream_t stream);
 
 /*
+ * moda_forward with the depth path chosen by the caller; the result is the same
+ * operator either way (hyper.ai summary of arXiv 2603.15619, section "Hardware-efficient
+ * implementation": the depth logits enter the same on-chip softmax state as the
+ * sequence logits).  depth_path:
+ *   0  automatic: the choice moda_forward makes (dense depth blocks whenever L > 0 and
+ *      Hq/Hkv divides 128; the fold otherwise);
+ *   1  CUDA-core fold: each query tile's depth rows are folded into the softmax state on
+ *      CUDA cores before its sequence blocks;
+ *   2  dense depth blocks: the depth rows run through the tensor-core pipeline as extra
+ *      128-key blocks of (token, entry) rows, each query row masked to its own token's
+ *      entries.  Needs Hq/Hkv to divide 128 (MODA_ERR_UNSUPPORTED otherwise).
+ * The two paths round differently (the fold's logits are fp32 CUDA-core dot products,
+ * the dense path's come from the tensor cores), so results agree to rounding, not bits.
+ * Any other depth_path value: MODA_ERR_INVALID_ARGUMENT.  Everything else as moda_forward.
+ */
+moda_status_t moda_forward_depth_path(const void *q, const void *k, const void *v,
+                                      const void *kd, const void *vd, void *out, float *lse,
+                                      int B, int Hq, int Hkv, int T, int L, int d,
+                                      float scale, int causal, int depth_path,
+                                      moda_stream_t stream);
+
+/*
  * Bytes of device workspace moda_backward needs for these sizes (fp32 dQ accumulator
  * [B][Hq][T][d] plus the fp32 row terms D = <dO, out> [B][Hq][T]).
  */

@@ -67,6 +67,20 @@ def test_forward_rejects_bad_arguments_before_launch(kw, status):
     assert fwd(**kw) == status
 
 
+@pytest.mark.parametrize("kw,path,status", [
+    (dict(), 3, moda.MODA_ERR_INVALID_ARGUMENT),
+    (dict(), -1, moda.MODA_ERR_INVALID_ARGUMENT),
+    (dict(Hq=6, Hkv=2), 2, moda.MODA_ERR_UNSUPPORTED),  # group of 3 does not divide 128
+    (dict(q=None), 2, moda.MODA_ERR_INVALID_ARGUMENT),
+])
+def test_forward_depth_path_rejects_bad_arguments(kw, path, status):
+    args = dict(q=A, k=A * 2, v=A * 3, kd=A * 4, vd=A * 5, out=A * 64, lse=A * 128, B=1,
+                Hq=4, Hkv=2, T=16, L=2, d=64, scale=0.125, causal=1, depth_path=path,
+                stream=None)
+    args.update(kw)
+    assert moda.moda_forward_depth_path(**args) == status
+
+
 def test_forward_L0_allows_null_depth():
     # valid arguments: without a GPU the call gets as far as the device check
     st = fwd(L=0, kd=None, vd=None)

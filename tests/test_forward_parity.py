@@ -44,6 +44,50 @@ def test_forward_small_full(name, cfg, causal):
     compare_forward(out, lse, ref_out, ref_lse, name)
 
 
+@pytest.mark.parametrize("path", [1, 2], ids=["fold", "dense"])
+@pytest.mark.parametrize("name,cfg,causal", SMALL, ids=[s[0] for s in SMALL])
+def test_forward_small_full_each_depth_path(name, cfg, causal, path):
+    """Both depth paths (CUDA-core fold, dense tensor-core depth blocks) on every case;
+    the dense path refuses groups that do not divide 128."""
+    x = gpu_inputs(cfg, seed_base=100 + SMALL.index((name, cfg, causal)))
+    scale = 1.0 / math.sqrt(cfg["d"])
+    G = cfg["Hq"] // cfg["Hkv"]
+    if path == 2 and 128 % G != 0:
+        with pytest.raises(moda.ModaError) as e:
+            moda.forward(x["q"], x["k"], x["v"], x["kd"], x["vd"], scale, causal,
+                         depth_path=path)
+        assert e.value.status == moda.MODA_ERR_UNSUPPORTED
+        return
+    out, lse = moda.forward(x["q"], x["k"], x["v"], x["kd"], x["vd"], scale, causal,
+                            depth_path=path)
+    moda.check_device_errors()
+    ref_out, ref_lse = oracle_forward_window(x, 0, cfg["T"], scale, causal)
+    compare_forward(out, lse, ref_out, ref_lse, f"{name} path {path}")
+
+
+@pytest.mark.parametrize("path", [1, 2], ids=["fold", "dense"])
+def test_forward_deep_windows_each_depth_path(path):
+    """The deep-stack head layout (L = 128) at 4K tokens through each depth path, on
+    token windows at the start, middle and end; the dense path is also deterministic."""
+    cfg = workloads.CONFIGS["deep-4k"]
+    x = gpu_inputs(cfg, workloads.SEED_BASE["deep-4k"])
+    scale = workloads.default_scale(cfg["d"])
+    out, lse = moda.forward(x["q"], x["k"], x["v"], x["kd"], x["vd"], scale, True,
+                            depth_path=path)
+    out2, lse2 = moda.forward(x["q"], x["k"], x["v"], x["kd"], x["vd"], scale, True,
+                              depth_path=path)
+    moda.check_device_errors()
+    assert torch.equal(out, out2) and torch.equal(lse, lse2)
+    T, nt = cfg["T"], 48
+    for t0 in (0, T // 2 - 5, T - nt):
+        ref_out, ref_lse = oracle_forward_window(x, t0, nt, scale, True)
+        sl = slice(t0, t0 + nt)
+        compare_forward(out[:, :, sl], lse[:, :, sl], ref_out, ref_lse,
+                        f"deep-4k path {path} @{t0}")
+    del x, out, lse, out2, lse2
+    torch.cuda.empty_cache()
+
+
 def test_forward_is_deterministic_and_leaves_inputs_intact():
     cfg = dict(B=1, T=515, Hq=8, Hkv=2, d=128, L=6)
     x = gpu_inputs(cfg, seed_base=150)
