@@ -94,6 +94,38 @@ struct Bars {
   int abort;
 };
 
+// Order of a tile pair's steps.  With ND depth steps and NB0 sequence blocks in tile 0,
+// the first 2K steps (K = min(ND, NB0)) alternate depth step, sequence block; then come
+// the remaining depth steps, then the remaining sequence blocks.  Spreading the depth
+// steps (HBM-bound) among the sequence blocks (tensor-bound) keeps both busy.  Tile 1
+// shares the mapping of every common step (its at most one extra block comes last), and
+// every depth step comes before step ND + NB0.  ND = 0: step j is sequence block j.
+struct StepMap {
+  int ND, K;
+  __device__ __forceinline__ bool is_depth(int j) const {
+    return j < 2 * K ? (j & 1) == 0 : (j - 2 * K) < ND - K;
+  }
+  // depth step index or sequence block index of step j
+  __device__ __forceinline__ int index(int j) const {
+    if (j < 2 * K) return j >> 1;
+    const int jj = j - 2 * K;
+    return jj < ND - K ? K + jj : K + (jj - (ND - K));
+  }
+  // ring entries loaded before step j (4 per depth step, 2 per sequence block)
+  __device__ __forceinline__ int entry(int j) const {
+    int nd, ns;
+    if (j < 2 * K) {
+      nd = (j + 1) >> 1;
+      ns = j >> 1;
+    } else {
+      const int jj = j - 2 * K;
+      nd = K + min(jj, ND - K);
+      ns = K + max(0, jj - (ND - K));
+    }
+    return 4 * nd + 2 * ns;
+  }
+};
+
 __device__ __forceinline__ float dot8(const float (&a)[8], uint4 w) {
   float s = a[0] * bf16lo(w.x);
   s = fmaf(a[1], bf16hi(w.x), s);
@@ -141,10 +173,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const int ND = kDense ? nchunk : 0;  // tensor-core depth steps (ahead of the sequence)
   const int N0 = ND + NB0, N1 = ND + NB1;  // steps of tile 0 / tile 1
   constexpr int kDUses = 2 * Cfg::kRegions;   // depth stage uses per chunk: kd, vd regions
-  // Ring entries in load order.  Depth step j: kd of tile 0, kd of tile 1, vd of tile 0,
-  // vd of tile 1; sequence block j: K then V, shared by both tiles.
-  auto kidx = [&](int t, int j) { return j < ND ? 4 * j + t : 4 * ND + 2 * (j - ND); };
-  auto vidx = [&](int t, int j) { return j < ND ? 4 * j + 2 + t : 4 * ND + 2 * (j - ND) + 1; };
+  const StepMap sm{ND, min(ND, NB0)};
+  // Ring entries in load order.  Depth step: kd of tile 0, kd of tile 1, vd of tile 0,
+  // vd of tile 1; sequence block: K then V, shared by both tiles.
+  auto kidx = [&](int t, int j) { return sm.entry(j) + (sm.is_depth(j) ? t : 0); };
+  auto vidx = [&](int t, int j) { return sm.entry(j) + (sm.is_depth(j) ? 2 + t : 1); };
 
   if (threadIdx.x == 0) {
     mbar_init(bar(bars->q_full), 1);
@@ -204,23 +237,26 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         ++e;
         return s;
       };
-      if constexpr (kDense) {
-        // depth chunk j of a tile: entries [j*JC, j*JC+JC) of its TQ tokens, token-major
-        for (int j = 0; j < ND; ++j)
+      for (int j = 0; j < N1; ++j) {
+        const int ix = sm.index(j);
+        if (sm.is_depth(j)) {
+          // depth chunk ix of each tile: entries [ix*JC, ix*JC+JC) of its TQ tokens
           for (int u = 0; u < 4; ++u) {
             const int s = acquire(Cfg::kTileBytes);
             const CUtensorMap* map = (u < 2) ? &tmKD : &tmVD;
             for (int rg = 0; rg < Cfg::kRegions; ++rg)
-              tma_load_4d(sKV(s) + rg * kRegion, map, bar(bars->full[s]), rg * 64, j * a.JC,
-                          (u & 1) ? tq1 : tq0, bg);
+              tma_load_4d(sKV(s) + rg * kRegion, map, bar(bars->full[s]), rg * 64,
+                          ix * a.JC, (u & 1) ? tq1 : tq0, bg);
           }
-      }
-      for (int idx = 0; idx < 2 * NB1; ++idx) {
-        const int s = acquire(Cfg::kTileBytes);
-        const CUtensorMap* map = (idx & 1) ? &tmV : &tmK;
-        for (int rg = 0; rg < Cfg::kRegions; ++rg)
-          tma_load_3d(sKV(s) + rg * kRegion, map, bar(bars->full[s]), rg * 64,
-                      (idx >> 1) * kBN, bg);
+        } else {
+          for (int u = 0; u < 2; ++u) {
+            const int s = acquire(Cfg::kTileBytes);
+            const CUtensorMap* map = u ? &tmV : &tmK;
+            for (int rg = 0; rg < Cfg::kRegions; ++rg)
+              tma_load_3d(sKV(s) + rg * kRegion, map, bar(bars->full[s]), rg * 64, ix * kBN,
+                          bg);
+          }
+        }
       }
     } else if constexpr (!kDense) if ((lane == 1 || lane == 2) && NC > 0) {
       // Depth chunk ci of tile t: entries [ci*JC, ci*JC+JC) of the tile's TQ tokens as
@@ -288,7 +324,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                  make_sdesc_sw128(kbase + off, 16, 1024), idesc_s, ks > 0 ? 1u : 0u);
         }
         tc_commit(bar(bars->s_full[t]));
-        if (j < ND || t == 1) release(e);
+        if (sm.is_depth(j) || t == 1) release(e);
       };
       auto issue_pv = [&](int t, int j) {
         mbar_wait(bar(bars->p_full[t]), j & 1, abort_flag);
@@ -301,7 +337,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           mma_ts(tO, tmem + t * 128 + ks * 8,
                  make_sdesc_sw128(vbase + ks * 2048, kRegion, 1024), idesc_o,
                  (ks > 0 || j > 0 || NC > 0) ? 1u : 0u);
-        if (j < ND || t == 1) release(e);
+        if (sm.is_depth(j) || t == 1) release(e);
       };
       issue_s(0, 0);
       issue_s(1, 0);
@@ -418,7 +454,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       tmem_wait_st();
     }
 
-    // ---- depth steps (dense path), then sequence blocks
+    // ---- depth steps (dense path) and sequence blocks, in the order StepMap gives
     // A depth step's 128 keys are JC = G entries of each of the tile's TQ tokens,
     // token-major, so row r (token r / G) owns keys [r - hl, r - hl + G): all inside the
     // 32 keys of its warp's rows.  Only those 32 columns are read; P is zero elsewhere.
@@ -426,14 +462,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     for (int jb = 0; jb < NS; ++jb) {
       mbar_wait(bar(bars->s_full[tt]), jb & 1, abort_flag);
       tc_fence_after();
-      const bool dstep = kDense && jb < ND;
+      const bool dstep = kDense && sm.is_depth(jb);
+      const int ix = sm.index(jb);  // depth step or sequence block index
       uint32_t s[kBN];
       float mx = -INFINITY;  // row max on the raw scores (scale > 0); masked keys -> -inf
       if (dstep) {
         tmem_ld32(tS + 32 * (warp & 3), &s[0]);
         tmem_wait_ld();
         const int lo = (r & 31) - hl;
-        const int nval = min(a.JC, a.L - jb * a.JC);
+        const int nval = min(a.JC, a.L - ix * a.JC);
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
           if (c < lo || c >= lo + nval) s[c] = __float_as_uint(-INFINITY);
@@ -445,7 +482,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         tmem_ld32(tS + 64, &s[64]);
         tmem_ld32(tS + 96, &s[96]);
         tmem_wait_ld();
-        const int kbase = (jb - ND) * kBN;
+        const int kbase = ix * kBN;
         const bool need_mask = a.causal ? (kbase + kBN - 1 > t0) : (kbase + kBN > a.T);
         if (need_mask) {
 #pragma unroll
