@@ -10,8 +10,12 @@ point follows the definition of the operator on the hyper.ai summary of arXiv
 2603.15619, section "Mixture-of-Depths Attention (MoDA)": one softmax, jointly
 normalised, over the query's causal sequence keys and its own token's depth keys.
 
-Parity status: forward, backward, the backward with a given output and the row-weight
-view are pinned by the
+``depth_forward`` / ``depth_backward`` run the pages' depth-only operator (Flash Depth
+Attention: hyper.ai summary, section "Depth-stream mechanisms"): the same definition with
+no sequence keys, each row attending to its own token's depth keys only.
+
+Parity status: forward, backward, the backward with a given output, the row-weight view
+and the depth-only forward/backward are pinned by the
 ``-m "not gpu"`` tests in ``tests/test_oracle_pins.py`` (library special cases, closed
 forms, invariants, finite differences and hand-derived golden cases).
 """
@@ -49,6 +53,10 @@ def _load():
         lib.moda_oracle_row_weights.argtypes = [P] * 3 + [I] * 9 + [D, I, P, P]
         lib.moda_oracle_backward_given_out.argtypes = [P] * 12 + [I] * 8 + [D, I, I]
         lib.moda_oracle_backward_given_out.restype = I
+        lib.moda_oracle_depth_forward.argtypes = [P] * 5 + [I] * 8 + [D, I]
+        lib.moda_oracle_depth_forward.restype = I
+        lib.moda_oracle_depth_backward.argtypes = [P] * 10 + [I] * 8 + [D, I]
+        lib.moda_oracle_depth_backward.restype = I
         for f in (lib.moda_oracle_forward, lib.moda_oracle_backward,
                   lib.moda_oracle_row_weights):
             f.restype = I
@@ -185,3 +193,47 @@ def row_weights(q, k, kd, b, h, t, scale, causal=True):
     if rc != 0:
         raise ValueError("moda_oracle_row_weights rejected the arguments")
     return ws, wd[:L]
+
+
+def depth_forward(q, kd, vd, scale, t0=0, nthreads=None):
+    """Depth-only attention forward over the query tokens [t0, t0+nt).
+
+    q [B,Hq,nt,d]; kd,vd [B,Hkv,nt,L,d] with L >= 1.  Returns (out [B,Hq,nt,d],
+    lse [B,Hq,nt]) as float64 numpy arrays.  T is taken as t0 + nt (no sequence keys).
+    """
+    q, kd, vd = _f64(q), _f64(kd), _f64(vd)
+    B, Hq, nt, d = q.shape
+    Hkv, L = kd.shape[1], kd.shape[3]
+    out = np.empty((B, Hq, nt, d), np.float64)
+    lse = np.empty((B, Hq, nt), np.float64)
+    rc = _load().moda_oracle_depth_forward(_ptr(q), _ptr(kd), _ptr(vd), _ptr(out), _ptr(lse),
+                                           B, Hq, Hkv, t0 + nt, L, d, t0, nt, float(scale),
+                                           nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("moda_oracle_depth_forward rejected the sizes")
+    return out, lse
+
+
+def depth_backward(q, kd, vd, dout, scale, out=None, t0=0, nthreads=None):
+    """Depth-only attention backward over the query tokens [t0, t0+nt).
+
+    Returns dict(dq, dkd, dvd, out, lse) as float64 numpy arrays.  With ``out`` given
+    (window-sized, e.g. a forward's bf16 output widened), the row terms D = <dO, out> use
+    it, as backward_given_out does; otherwise they use the oracle's exact output.
+    """
+    q, kd, vd, dout = _f64(q), _f64(kd), _f64(vd), _f64(dout)
+    given = _f64(out)
+    B, Hq, nt, d = q.shape
+    Hkv, L = kd.shape[1], kd.shape[3]
+    dq = np.empty((B, Hq, nt, d), np.float64)
+    dkd = np.empty((B, Hkv, nt, L, d), np.float64)
+    dvd = np.empty((B, Hkv, nt, L, d), np.float64)
+    o = np.empty((B, Hq, nt, d), np.float64)
+    lse = np.empty((B, Hq, nt), np.float64)
+    rc = _load().moda_oracle_depth_backward(
+        _ptr(q), _ptr(kd), _ptr(vd), _ptr(dout), _ptr(given), _ptr(dq), _ptr(dkd), _ptr(dvd),
+        _ptr(o), _ptr(lse), B, Hq, Hkv, t0 + nt, L, d, t0, nt, float(scale),
+        nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("moda_oracle_depth_backward rejected the sizes")
+    return dict(dq=dq, dkd=dkd, dvd=dvd, out=o, lse=lse)

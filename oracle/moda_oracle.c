@@ -45,6 +45,13 @@
  * a test check sampled rows of a 64K-token problem without materialising its whole
  * depth cache in fp64.
  *
+ * Depth-only attention (Flash Depth Attention, the pages' other operator: hyper.ai
+ * summary, section "Depth-stream mechanisms" -- a layer's input is attention over the
+ * key/value pairs that earlier layers wrote for the SAME token; shijienb.com article,
+ * first half, names its kernel Flash Depth Attention): the same definition with no
+ * sequence keys, S(t) = {}.  The moda_oracle_depth_* entry points run it (causal = -1
+ * internally; k, v, dk, dv absent).
+ *
  * Parallelism: rows (forward) or (b, kv-head) units (backward) are handed to POSIX
  * threads through an atomic counter; each unit's arithmetic is the plain loop above.
  */
@@ -71,8 +78,11 @@ static double dot(const double *a, const double *b, int d) {
     return s;
 }
 
-/* Number of visible sequence keys for token t. */
-static int n_seq(int t, int T, int causal) { return causal ? t + 1 : T; }
+/* Number of visible sequence keys for token t (causal < 0: depth-only, none). */
+static int n_seq(int t, int T, int causal) {
+    if (causal < 0) return 0;
+    return causal ? t + 1 : T;
+}
 
 /* Offsets of window-sized arrays: row (b,h,w) of q/out, token (b,g,w) of kd/vd. */
 static int64_t qrow(const job_t *J, int b, int h, int w) {
@@ -88,12 +98,12 @@ static void forward_row(const job_t *J, int b, int h, int w, double *scratch,
                         double *out_row, double *lse_row) {
     const int d = J->d, T = J->T, L = J->L, G = J->Hq / J->Hkv, g = h / G;
     const int t = J->t0 + w;
-    const double *qr = J->q + qrow(J, b, h, w) * d;
-    const double *kb = J->k + ((int64_t)b * J->Hkv + g) * T * d;
-    const double *vb = J->v + ((int64_t)b * J->Hkv + g) * T * d;
-    const double *kdt = J->kd + dtok(J, b, g, w) * L * d;
-    const double *vdt = J->vd + dtok(J, b, g, w) * L * d;
     const int ns = n_seq(t, T, J->causal);
+    const double *qr = J->q + qrow(J, b, h, w) * d;
+    const double *kb = ns ? J->k + ((int64_t)b * J->Hkv + g) * T * d : NULL;
+    const double *vb = ns ? J->v + ((int64_t)b * J->Hkv + g) * T * d : NULL;
+    const double *kdt = L ? J->kd + dtok(J, b, g, w) * L * d : NULL;
+    const double *vdt = L ? J->vd + dtok(J, b, g, w) * L * d : NULL;
 
     /* pass 1: logits and their maximum */
     double m = -INFINITY;
@@ -144,16 +154,17 @@ static void *forward_worker(void *arg) {
 static void backward_unit(job_t *J, int b, int g, double *scratch, double *o_row) {
     const int d = J->d, T = J->T, L = J->L, G = J->Hq / J->Hkv;
     const int64_t kvoff = ((int64_t)b * J->Hkv + g) * T * d;
-    const double *kb = J->k + kvoff, *vb = J->v + kvoff;
-    double *dkb = J->dk + kvoff, *dvb = J->dv + kvoff;
+    const int has_seq = J->causal >= 0;
+    const double *kb = has_seq ? J->k + kvoff : NULL, *vb = has_seq ? J->v + kvoff : NULL;
+    double *dkb = has_seq ? J->dk + kvoff : NULL, *dvb = has_seq ? J->dv + kvoff : NULL;
     for (int h = g * G; h < (g + 1) * G; ++h) {
         for (int w = 0; w < J->nt; ++w) {
             const int64_t r = qrow(J, b, h, w);
             const double *qr = J->q + r * d, *dor = J->dout + r * d;
             double *dqr = J->dq + r * d;
             const int64_t doff = dtok(J, b, g, w) * L * d;
-            const double *kdt = J->kd + doff, *vdt = J->vd + doff;
-            double *dkdt = J->dkd + doff, *dvdt = J->dvd + doff;
+            const double *kdt = L ? J->kd + doff : NULL, *vdt = L ? J->vd + doff : NULL;
+            double *dkdt = L ? J->dkd + doff : NULL, *dvdt = L ? J->dvd + doff : NULL;
             const int ns = n_seq(J->t0 + w, T, J->causal);
             double lse;
             forward_row(J, b, h, w, scratch, o_row, &lse);
@@ -323,5 +334,45 @@ int moda_oracle_row_weights(const double *q, const double *k, const double *kd, 
     for (int j = 0; j < L; ++j) { w_depth[j] = exp(w_depth[j] - m); Z += w_depth[j]; }
     for (int s = 0; s < ns; ++s) w_seq[s] /= Z;
     for (int j = 0; j < L; ++j) w_depth[j] /= Z;
+    return 0;
+}
+
+/* Depth-only attention forward over the query tokens [t0, t0+nt): every row attends to
+ * its own token's L >= 1 depth keys only.  Returns 0 on success, 1 on bad sizes. */
+int moda_oracle_depth_forward(const double *q, const double *kd, const double *vd,
+                              double *out, double *lse, int B, int Hq, int Hkv, int T, int L,
+                              int d, int t0, int nt, double scale, int nthreads) {
+    if (bad_dims(B, Hq, Hkv, T, L, d, t0, nt) || L < 1) return 1;
+    job_t J = {0};
+    J.q = q; J.kd = kd; J.vd = vd; J.out = out; J.lse = lse;
+    J.B = B; J.Hq = Hq; J.Hkv = Hkv; J.T = T; J.L = L; J.d = d; J.causal = -1;
+    J.t0 = t0; J.nt = nt; J.scale = scale;
+    J.nunits = (int64_t)B * Hq * nt;
+    run(&J, forward_worker, nthreads);
+    return 0;
+}
+
+/* Depth-only attention backward over the window's rows: dq, dkd, dvd (all exact for the
+ * window).  out_given: NULL for the exact row terms D = <dO, out>, else D is taken from
+ * the given (window-sized) out, as in moda_oracle_backward_given_out.  If out/lse are
+ * non-NULL the oracle's own forward results are written there too. */
+int moda_oracle_depth_backward(const double *q, const double *kd, const double *vd,
+                               const double *dout, const double *out_given, double *dq,
+                               double *dkd, double *dvd, double *out, double *lse, int B,
+                               int Hq, int Hkv, int T, int L, int d, int t0, int nt,
+                               double scale, int nthreads) {
+    if (bad_dims(B, Hq, Hkv, T, L, d, t0, nt) || L < 1) return 1;
+    const size_t nq = (size_t)B * Hq * nt * d;
+    const size_t nd = (size_t)B * Hkv * nt * (size_t)L * d;
+    memset(dq, 0, nq * sizeof(double));
+    memset(dkd, 0, nd * sizeof(double));
+    memset(dvd, 0, nd * sizeof(double));
+    job_t J = {0};
+    J.q = q; J.kd = kd; J.vd = vd; J.dout = dout; J.out_given = out_given;
+    J.dq = dq; J.dkd = dkd; J.dvd = dvd; J.out = out; J.lse = lse;
+    J.B = B; J.Hq = Hq; J.Hkv = Hkv; J.T = T; J.L = L; J.d = d; J.causal = -1;
+    J.t0 = t0; J.nt = nt; J.scale = scale;
+    J.nunits = (int64_t)B * Hkv;
+    run(&J, backward_worker, nthreads);
     return 0;
 }

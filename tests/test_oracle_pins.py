@@ -332,3 +332,98 @@ def test_backward_given_out_shifts_only_the_row_terms():
     total = got["dk"].sum(2) + got["dkd"].sum(axis=(2, 3))
     np.testing.assert_allclose(total, expect, rtol=1e-9, atol=1e-13)
     assert np.abs(ref["dk"].sum(2) + ref["dkd"].sum(axis=(2, 3))).max() < 1e-12
+
+
+# ---------------------------------------------------------------- depth-only attention
+def sdpa_depth_reference(q, kd, vd, scale):
+    """Depth-only attention via torch SDPA: row t sees exactly its own token's L depth
+    keys (a block-diagonal mask over the flattened [T*L] depth keys).  fp64."""
+    B, Hq, T, d = q.shape
+    Hkv, L = kd.shape[1], kd.shape[3]
+    G = Hq // Hkv
+    kf = kd.reshape(B, Hkv, T * L, d).repeat_interleave(G, dim=1)
+    vf = vd.reshape(B, Hkv, T * L, d).repeat_interleave(G, dim=1)
+    mask = torch.zeros(T, T * L, dtype=torch.bool)
+    for t in range(T):
+        mask[t, t * L:(t + 1) * L] = True
+    out = F.scaled_dot_product_attention(q, kf, vf, attn_mask=mask, scale=scale)
+    scores = torch.einsum("bhtc,bhsc->bhts", q, kf) * scale
+    lse = torch.logsumexp(scores.masked_fill(~mask, float("-inf")), dim=-1)
+    return out, lse
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+def test_depth_forward_equals_masked_sdpa(shape):
+    x = rand_problem(**shape, seed=41)
+    scale = 0.37
+    out, lse = oracle.depth_forward(x["q"], x["kd"], x["vd"], scale)
+    ref_out, ref_lse = sdpa_depth_reference(x["q"], x["kd"], x["vd"], scale)
+    assert np.abs(out - ref_out.numpy()).max() < 1e-12
+    assert np.abs(lse - ref_lse.numpy()).max() < 1e-12
+
+
+def test_depth_backward_equals_sdpa_autograd():
+    x = rand_problem(B=1, T=6, Hq=4, Hkv=2, d=8, L=3, seed=43)
+    scale = 0.45
+    g = oracle.depth_backward(x["q"], x["kd"], x["vd"], x["dout"], scale)
+    leaves = {n: x[n].clone().requires_grad_(True) for n in ("q", "kd", "vd")}
+    ref_out, _ = sdpa_depth_reference(leaves["q"], leaves["kd"], leaves["vd"], scale)
+    (ref_out * x["dout"]).sum().backward()
+    for n in ("q", "kd", "vd"):
+        assert np.abs(g["d" + n] - leaves[n].grad.numpy()).max() < 1e-12, n
+
+
+def test_depth_single_entry_closed_form():
+    """L = 1: the one depth key takes all the weight, so out is its value, lse its logit,
+    and only dvd is non-zero (the sum of the group's dO)."""
+    x = rand_problem(B=2, T=4, Hq=6, Hkv=2, d=8, L=1, seed=45)
+    scale = 0.5
+    g = oracle.depth_backward(x["q"], x["kd"], x["vd"], x["dout"], scale)
+    G = 3
+    vd = x["vd"][:, :, :, 0].numpy().repeat(G, axis=1)
+    kd = x["kd"][:, :, :, 0].numpy().repeat(G, axis=1)
+    assert np.abs(g["out"] - vd).max() < 1e-14
+    assert np.abs(g["lse"] - scale * (x["q"].numpy() * kd).sum(-1)).max() < 1e-13
+    assert np.abs(g["dq"]).max() < 1e-14 and np.abs(g["dkd"]).max() < 1e-14
+    dsum = x["dout"].numpy().reshape(2, 2, G, 4, 8).sum(2)
+    assert np.abs(g["dvd"][:, :, :, 0] - dsum).max() < 1e-13
+
+
+def test_depth_only_is_moda_at_one_token():
+    """A one-token MoDA problem (its sequence key is its own k) equals depth-only attention
+    over the depth keys with k prepended: the two oracle modes agree on the definition."""
+    x = rand_problem(B=1, T=1, Hq=4, Hkv=2, d=8, L=3, seed=47)
+    scale = 0.3
+    out, lse = oracle.forward(x["q"], x["k"], x["v"], x["kd"], x["vd"], scale)
+    kd = torch.cat([x["k"][:, :, :, None], x["kd"]], dim=3)
+    vd = torch.cat([x["v"][:, :, :, None], x["vd"]], dim=3)
+    out2, lse2 = oracle.depth_forward(x["q"], kd, vd, scale)
+    assert np.abs(out - out2).max() < 1e-14 and np.abs(lse - lse2).max() < 1e-14
+
+
+def test_depth_backward_matches_finite_differences():
+    x = rand_problem(B=1, T=3, Hq=2, Hkv=1, d=4, L=4, seed=49)
+    scale = 0.7
+    g = oracle.depth_backward(x["q"], x["kd"], x["vd"], x["dout"], scale)
+    dO = x["dout"].numpy()
+    eps = 1e-6
+    rng = np.random.default_rng(5)
+    for n in ("q", "kd", "vd"):
+        for _ in range(3):
+            direction = torch.from_numpy(rng.standard_normal(tuple(x[n].shape)))
+            plus = dict(x); minus = dict(x)
+            plus[n] = x[n] + eps * direction
+            minus[n] = x[n] - eps * direction
+            fp, _ = oracle.depth_forward(plus["q"], plus["kd"], plus["vd"], scale)
+            fm, _ = oracle.depth_forward(minus["q"], minus["kd"], minus["vd"], scale)
+            numeric = float(((fp - fm) * dO).sum() / (2 * eps))
+            analytic = float((g["d" + n] * direction.numpy()).sum())
+            assert abs(numeric - analytic) < 1e-7 * max(1.0, abs(analytic)), (n, numeric, analytic)
+
+
+def test_depth_backward_given_own_out_equals_exact():
+    x = rand_problem(B=1, T=5, Hq=4, Hkv=1, d=8, L=6, seed=51)
+    g = oracle.depth_backward(x["q"], x["kd"], x["vd"], x["dout"], 0.4)
+    h = oracle.depth_backward(x["q"], x["kd"], x["vd"], x["dout"], 0.4, out=g["out"])
+    for n in ("dq", "dkd", "dvd"):
+        assert np.abs(g[n] - h[n]).max() < 1e-14, n
