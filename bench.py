@@ -57,6 +57,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle sample")
+    ap.add_argument("--fda", action="store_true",
+                    help="time depth-only attention (forward, backward) on --workload")
     ap.add_argument("--sweep", action="store_true",
                     help="forward efficiency sweep over T x L (not the headline step)")
     return ap.parse_args()
@@ -500,10 +502,10 @@ def run_sweep(args):
     dev = torch.device("cuda", 0)
     stream = torch.cuda.current_stream(dev)
     rows = []
-    for T in (4096, 8192, 16384, 32768, 65536):
+    for G, T in [(g, t) for g in (4, 8) for t in (4096, 8192, 16384, 32768, 65536)]:
         ms0 = None
         for L in (0, 8, 32, 128):
-            cfg = dict(B=1, T=T, Hq=16, Hkv=4, d=128, L=L)
+            cfg = dict(B=1, T=T, Hq=4 * G, Hkv=4, d=128, L=L)
             x = workloads.make_inputs(cfg, 900 + T // 4096, dev)
             out = torch.empty_like(x["q"])
             lse = torch.empty(x["q"].shape[:3], device=dev, dtype=torch.float32)
@@ -524,7 +526,7 @@ def run_sweep(args):
             if L == 0:
                 ms0 = ms
             tf = workloads.forward_flops(**cfg) / (ms * 1e-3) / 1e12
-            row = {"T": T, "L": L, "ms": round(ms, 4), "tflops": round(tf, 1),
+            row = {"G": G, "T": T, "L": L, "ms": round(ms, 4), "tflops": round(tf, 1),
                    "time_ratio_L0_over_L": round(ms0 / ms, 4),
                    "depth_gbs_from_difference": (round(workloads.depth_bytes(**cfg) /
                                                        ((ms - ms0) * 1e-3) / 1e9, 1)
@@ -533,17 +535,69 @@ def run_sweep(args):
             rows.append(row)
             del x, out, lse
             torch.cuda.empty_cache()
-    print("| T | L | ms | TFLOP/s | time(L=0)/time(L) |")
-    print("|---|---|---|---|---|")
+    print("| G | T | L | ms | TFLOP/s | time(L=0)/time(L) |")
+    print("|---|---|---|---|---|---|")
     for r in rows:
-        print(f"| {r['T']} | {r['L']} | {r['ms']:.3f} | {r['tflops']:.0f} | "
+        print(f"| {r['G']} | {r['T']} | {r['L']} | {r['ms']:.3f} | {r['tflops']:.0f} | "
               f"{r['time_ratio_L0_over_L']:.3f} |")
+
+
+def run_fda(args):
+    """Depth-only attention (Flash Depth Attention) forward and backward on the workload's
+    depth cache: average CUDA-event times and the algorithmic HBM rate of each (forward:
+    q, kd, vd read, out and lse written; backward: q, kd, vd, out, dout read, dkd, dvd,
+    dq written, fp32 dq accumulator written and read)."""
+    import depth_aware_attention_b200 as moda
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+    cfg = workloads.CONFIGS[args.workload]
+    if cfg["L"] < 1:
+        raise SystemExit("depth-only attention needs a workload with L >= 1")
+    x = workloads.make_inputs(cfg, workloads.SEED_BASE[args.workload], dev, with_dout=True)
+    B, Hq, Hkv, T, L, d = (cfg[n] for n in ("B", "Hq", "Hkv", "T", "L", "d"))
+    out = torch.empty_like(x["q"])
+    lse = torch.empty((B, Hq, T), device=dev, dtype=torch.float32)
+    ws = torch.empty(moda.moda_backward_workspace_size(B, Hq, Hkv, T, L, d), device=dev,
+                     dtype=torch.uint8)
+    grads = dict(dq=torch.empty_like(x["q"]), dkd=torch.empty_like(x["kd"]),
+                 dvd=torch.empty_like(x["vd"]))
+    fwd = lambda: moda.depth_attention_forward(x["q"], x["kd"], x["vd"], out=out, lse=lse)
+    bwd = lambda: moda.depth_attention_backward(x["q"], x["kd"], x["vd"], out, lse, x["dout"],
+                                                workspace=ws, grads=grads)
+    res = {}
+    for name, f in (("forward", fwd), ("backward", bwd)):
+        for _ in range(max(3, args.warmup)):
+            f()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            f()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        res[name] = e0.elapsed_time(e1) / args.steps
+    moda.check_device_errors()
+    rows = B * Hq * T
+    dep = workloads.depth_bytes(**cfg)
+    fbytes = dep + rows * d * 2 * 2 + rows * 4
+    bbytes = 2 * dep + rows * d * 2 * 4 + rows * d * 4 * 2 + rows * 8
+    pk = peaks()
+    line = {"op": "depth-only attention", "workload": args.workload, "config": cfg,
+            "forward_ms": round(res["forward"], 4),
+            "forward_gbs": round(fbytes / (res["forward"] * 1e-3) / 1e9, 1),
+            "backward_ms": round(res["backward"], 4),
+            "backward_gbs": round(bbytes / (res["backward"] * 1e-3) / 1e9, 1),
+            "hbm_peak_gbs": pk["hbm"], "steps": args.steps}
+    print(json.dumps(line), flush=True)
 
 
 def main():
     args = parse()
     if args.sweep:
         run_sweep(args)
+        return
+    if args.fda:
+        run_fda(args)
         return
     world, rank, local = dist_setup(args.gpus)
     cfg = workloads.CONFIGS[args.workload]

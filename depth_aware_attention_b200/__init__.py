@@ -29,7 +29,8 @@ MODA_ERR_INTERNAL = 5
 BACKWARD_LAUNCHES = 3
 
 # Every symbol include/moda.h declares (checked by the ABI tests).
-EXPORTED = ("moda_forward", "moda_forward_depth_path", "moda_backward", "moda_backward_workspace_size",
+EXPORTED = ("moda_forward", "moda_forward_depth_path", "moda_depth_attention_forward",
+            "moda_depth_attention_backward", "moda_backward", "moda_backward_workspace_size",
             "moda_backward_stages", "moda_backward_noalloc", "moda_check_device_errors", "moda_status_string",
             "moda_last_error_message")
 
@@ -51,6 +52,10 @@ def _load():
     lib.moda_forward.restype = I
     lib.moda_forward_depth_path.argtypes = [P] * 7 + [I] * 6 + [F, I, I, P]
     lib.moda_forward_depth_path.restype = I
+    lib.moda_depth_attention_forward.argtypes = [P] * 5 + [I] * 6 + [F, P]
+    lib.moda_depth_attention_forward.restype = I
+    lib.moda_depth_attention_backward.argtypes = [P] * 10 + [S] + [I] * 6 + [F, P]
+    lib.moda_depth_attention_backward.restype = I
     lib.moda_backward_workspace_size.argtypes = [I] * 6
     lib.moda_backward_workspace_size.restype = S
     lib.moda_backward.argtypes = [P] * 14 + [S] + [I] * 6 + [F, I, P]
@@ -94,6 +99,20 @@ def moda_forward_depth_path(q, k, v, kd, vd, out, lse, B, Hq, Hkv, T, L, d, scal
     """Direct call of moda_forward_depth_path with raw pointers (ints) and a stream handle."""
     return lib.moda_forward_depth_path(q, k, v, kd, vd, out, lse, B, Hq, Hkv, T, L, d,
                                        float(scale), int(causal), int(depth_path), stream)
+
+
+def moda_depth_attention_forward(q, kd, vd, out, lse, B, Hq, Hkv, T, L, d, scale, stream):
+    """Direct call of moda_depth_attention_forward with raw pointers (ints)."""
+    return lib.moda_depth_attention_forward(q, kd, vd, out, lse, B, Hq, Hkv, T, L, d,
+                                            float(scale), stream)
+
+
+def moda_depth_attention_backward(q, kd, vd, out, lse, dout, dq, dkd, dvd, workspace,
+                                  workspace_bytes, B, Hq, Hkv, T, L, d, scale, stream):
+    """Direct call of moda_depth_attention_backward with raw pointers (ints)."""
+    return lib.moda_depth_attention_backward(q, kd, vd, out, lse, dout, dq, dkd, dvd,
+                                             workspace, workspace_bytes, B, Hq, Hkv, T, L, d,
+                                             float(scale), stream)
 
 
 def moda_backward(q, k, v, kd, vd, out, lse, dout, dq, dk, dv, dkd, dvd, workspace,
@@ -226,3 +245,52 @@ def check_device_errors(device=None):
     import torch
     st, flags = moda_check_device_errors(_stream_handle(device or torch.cuda.current_device()))
     _check(st, f"device error word 0x{flags:x}")
+
+
+def depth_attention_forward(q, kd, vd, scale=None, out=None, lse=None):
+    """Depth-only attention (Flash Depth Attention) forward on the current CUDA stream:
+    each row attends to its own token's L >= 1 depth keys.  Returns (out bf16, lse fp32).
+
+    q [B,Hq,T,d], kd/vd [B,Hkv,T,L,d]: contiguous bf16 CUDA tensors.
+    """
+    import torch
+    B, Hq, T, d = q.shape
+    Hkv, L = kd.shape[1], kd.shape[3]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, T), device=q.device, dtype=torch.float32)
+    st = lib.moda_depth_attention_forward(_ptr(q), _ptr(kd), _ptr(vd), _ptr(out), _ptr(lse),
+                                          B, Hq, Hkv, T, L, d, float(scale),
+                                          _stream_handle(q.device))
+    _check(st, "moda_depth_attention_forward")
+    return out, lse
+
+
+def depth_attention_backward(q, kd, vd, out, lse, dout, scale=None, workspace=None,
+                             grads=None):
+    """Depth-only attention backward on the current CUDA stream.  Returns dict(dq, dkd,
+    dvd); ``workspace``/``grads`` as for backward()."""
+    import torch
+    B, Hq, T, d = q.shape
+    Hkv, L = kd.shape[1], kd.shape[3]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    ws = moda_backward_workspace_size(B, Hq, Hkv, T, L, d)
+    if workspace is None:
+        workspace = torch.empty(ws, device=q.device, dtype=torch.uint8)
+    g = dict(grads or {})
+    if g.get("dq") is None:
+        g["dq"] = torch.empty_like(q)
+    if g.get("dkd") is None:
+        g["dkd"] = torch.empty_like(kd)
+    if g.get("dvd") is None:
+        g["dvd"] = torch.empty_like(vd)
+    st = lib.moda_depth_attention_backward(
+        _ptr(q), _ptr(kd), _ptr(vd), _ptr(out), _ptr(lse), _ptr(dout), _ptr(g["dq"]),
+        _ptr(g["dkd"]), _ptr(g["dvd"]), _ptr(workspace), workspace.numel(), B, Hq, Hkv, T,
+        L, d, float(scale), _stream_handle(q.device))
+    _check(st, "moda_depth_attention_backward")
+    return g

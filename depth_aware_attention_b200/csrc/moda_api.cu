@@ -106,10 +106,16 @@ const char* moda_last_error_message(void) { return g_msg; }
 static moda_status_t forward_entry(const void* q, const void* k, const void* v,
                                    const void* kd, const void* vd, void* out, float* lse,
                                    int B, int Hq, int Hkv, int T, int L, int d, float scale,
-                                   int causal, int depth_path, moda_stream_t stream) {
+                                   int causal, int depth_path, int depth_only,
+                                   moda_stream_t stream) {
   g_msg[0] = 0;
   moda_status_t s = check_sizes(B, Hq, Hkv, T, L, d);
   if (s != MODA_OK) return s;
+  if (depth_only) {
+    if (L < 1) return fail(MODA_ERR_INVALID_ARGUMENT, "depth-only attention needs L >= 1");
+    // no sequence keys; the kernel's K/V tensor maps are described over q and never read
+    k = v = q;
+  }
   if (depth_path < moda::kDepthPathAuto || depth_path > moda::kDepthPathDense)
     return fail(MODA_ERR_INVALID_ARGUMENT, "depth_path must be 0, 1 or 2");
   if (!q || !k || !v || !out || !lse)
@@ -131,6 +137,7 @@ static moda_status_t forward_entry(const void* q, const void* k, const void* v,
   if (overlaps(out, nq, lse, nl))
     return fail(MODA_ERR_INVALID_ARGUMENT, "out and lse must not overlap");
   moda::Problem p{B, Hq, Hkv, T, L, d, Hq / Hkv, causal ? 1 : 0, scale};
+  p.depth_only = depth_only ? 1 : 0;
   if (depth_path == moda::kDepthPathDense && !moda::dense_depth_supported(p))
     return fail(MODA_ERR_UNSUPPORTED, "dense depth blocks need Hq/Hkv to divide 128");
   s = check_device();
@@ -152,7 +159,15 @@ moda_status_t moda_forward(const void* q, const void* k, const void* v, const vo
                            int T, int L, int d, float scale, int causal,
                            moda_stream_t stream) {
   return forward_entry(q, k, v, kd, vd, out, lse, B, Hq, Hkv, T, L, d, scale, causal,
-                       moda::kDepthPathAuto, stream);
+                       moda::kDepthPathAuto, 0, stream);
+}
+
+moda_status_t moda_depth_attention_forward(const void* q, const void* kd, const void* vd,
+                                           void* out, float* lse, int B, int Hq, int Hkv,
+                                           int T, int L, int d, float scale,
+                                           moda_stream_t stream) {
+  return forward_entry(q, nullptr, nullptr, kd, vd, out, lse, B, Hq, Hkv, T, L, d, scale, 1,
+                       moda::kDepthPathAuto, 1, stream);
 }
 
 moda_status_t moda_forward_depth_path(const void* q, const void* k, const void* v,
@@ -161,7 +176,7 @@ moda_status_t moda_forward_depth_path(const void* q, const void* k, const void* 
                                       float scale, int causal, int depth_path,
                                       moda_stream_t stream) {
   return forward_entry(q, k, v, kd, vd, out, lse, B, Hq, Hkv, T, L, d, scale, causal,
-                       depth_path, stream);
+                       depth_path, 0, stream);
 }
 
 size_t moda_backward_workspace_size(int B, int Hq, int Hkv, int T, int L, int d) {
@@ -179,11 +194,17 @@ moda_status_t backward_entry(const void* q, const void* k, const void* v, const 
                              const void* dout, void* dq, void* dk, void* dv, void* dkd,
                              void* dvd, void* workspace, size_t workspace_bytes, int B,
                              int Hq, int Hkv, int T, int L, int d, float scale, int causal,
-                             unsigned stages, moda_stream_t stream) {
+                             unsigned stages, int depth_only, moda_stream_t stream) {
   g_msg[0] = 0;
   moda_status_t s = check_sizes(B, Hq, Hkv, T, L, d);
   if (s != MODA_OK) return s;
-  if (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv || !workspace)
+  if (depth_only) {
+    if (L < 1) return fail(MODA_ERR_INVALID_ARGUMENT, "depth-only attention needs L >= 1");
+    k = v = nullptr;  // no sequence keys: k, v, dk, dv are not used
+    dk = dv = nullptr;
+    stages = moda::kStageDepth | moda::kStageConvert;
+  }
+  if (!q || !out || !lse || !dout || !dq || !workspace || (!depth_only && (!k || !v || !dk || !dv)))
     return fail(MODA_ERR_INVALID_ARGUMENT,
                 "q, k, v, out, lse, dout, dq, dk, dv and workspace must be non-NULL");
   if (L > 0 && (!kd || !vd || !dkd || !dvd))
@@ -199,11 +220,12 @@ moda_status_t backward_entry(const void* q, const void* k, const void* v, const 
   if (Hq / Hkv > 16)
     return fail(MODA_ERR_UNSUPPORTED, "the backward supports at most 16 query heads per KV head");
   moda::Problem p{B, Hq, Hkv, T, L, d, Hq / Hkv, causal ? 1 : 0, scale};
+  p.depth_only = depth_only ? 1 : 0;
   const size_t need = moda::backward_workspace_bytes(p);
   if (workspace_bytes < need)
     return fail(MODA_ERR_INVALID_ARGUMENT, "workspace is smaller than moda_backward_workspace_size()");
   const size_t nq = size_t(B) * Hq * T * d * 2, nk = size_t(B) * Hkv * T * d * 2;
-  const size_t nd = nk * size_t(L), nl = size_t(B) * Hq * T * 4;
+  const size_t nd = nk * size_t(L), nl = size_t(B) * Hq * T * 4;  // (k, v unused: NULL)
   const void* ins[8] = {q, k, v, kd, vd, out, lse, dout};
   const size_t insz[8] = {nq, nk, nk, nd, nd, nq, nl, nq};
   void* outs[6] = {dq, dk, dv, dkd, dvd, workspace};
@@ -243,7 +265,7 @@ moda_status_t moda_backward(const void* q, const void* k, const void* v, const v
                             moda_stream_t stream) {
   return backward_entry(q, k, v, kd, vd, out, lse, dout, dq, dk, dv, dkd, dvd, workspace,
                         workspace_bytes, B, Hq, Hkv, T, L, d, scale, causal, moda::kStagesAll,
-                        stream);
+                        0, stream);
 }
 
 moda_status_t moda_backward_stages(const void* q, const void* k, const void* v,
@@ -258,7 +280,19 @@ moda_status_t moda_backward_stages(const void* q, const void* k, const void* v,
     return fail(MODA_ERR_INVALID_ARGUMENT, "stages must be a non-empty subset of {1, 2, 4}");
   }
   return backward_entry(q, k, v, kd, vd, out, lse, dout, dq, dk, dv, dkd, dvd, workspace,
-                        workspace_bytes, B, Hq, Hkv, T, L, d, scale, causal, stages, stream);
+                        workspace_bytes, B, Hq, Hkv, T, L, d, scale, causal, stages, 0,
+                        stream);
+}
+
+moda_status_t moda_depth_attention_backward(const void* q, const void* kd, const void* vd,
+                                            const void* out, const float* lse,
+                                            const void* dout, void* dq, void* dkd, void* dvd,
+                                            void* workspace, size_t workspace_bytes, int B,
+                                            int Hq, int Hkv, int T, int L, int d, float scale,
+                                            moda_stream_t stream) {
+  return backward_entry(q, nullptr, nullptr, kd, vd, out, lse, dout, dq, nullptr, nullptr,
+                        dkd, dvd, workspace, workspace_bytes, B, Hq, Hkv, T, L, d, scale, 1,
+                        moda::kStagesAll, 1, stream);
 }
 
 moda_status_t moda_check_device_errors(moda_stream_t stream, uint32_t* flags) {

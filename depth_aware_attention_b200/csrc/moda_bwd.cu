@@ -1101,89 +1101,89 @@ cudaError_t launch_backward_d(const Problem& p, const void* q, const void* k, co
       e = launch_depth<D, 16>(da, stream, why);
     if (e != cudaSuccess) return e;
   }
-  if (!(stages & (kStageSeq | kStageConvert))) return cudaSuccess;
-
-  // 2. sequence part
-  const cuuint64_t E = 2;
-  const cuuint64_t BG = cuuint64_t(p.B) * p.Hkv;
-  CUtensorMap mQ, mDO, mK, mV;
-  {
-    const cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(p.G), cuuint64_t(p.T), BG};
-    const cuuint64_t str[3] = {cuuint64_t(p.T) * D * E, cuuint64_t(D) * E,
-                               cuuint64_t(p.G) * p.T * D * E};
-    const cuuint32_t box[4] = {64, cuuint32_t(p.G), cuuint32_t(tg.TQ), 1};
-    if (!make_map_b(encode, &mQ, q, 4, dims, str, box) ||
-        !make_map_b(encode, &mDO, dout, 4, dims, str, box)) {
-      *why = "cuTensorMapEncodeTiled failed for q/dout";
-      return cudaErrorInvalidValue;
+  // 2. sequence part (none for depth-only attention)
+  if (stages & kStageSeq) {
+    const cuuint64_t E = 2;
+    const cuuint64_t BG = cuuint64_t(p.B) * p.Hkv;
+    CUtensorMap mQ, mDO, mK, mV;
+    {
+      const cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(p.G), cuuint64_t(p.T), BG};
+      const cuuint64_t str[3] = {cuuint64_t(p.T) * D * E, cuuint64_t(D) * E,
+                                 cuuint64_t(p.G) * p.T * D * E};
+      const cuuint32_t box[4] = {64, cuuint32_t(p.G), cuuint32_t(tg.TQ), 1};
+      if (!make_map_b(encode, &mQ, q, 4, dims, str, box) ||
+          !make_map_b(encode, &mDO, dout, 4, dims, str, box)) {
+        *why = "cuTensorMapEncodeTiled failed for q/dout";
+        return cudaErrorInvalidValue;
+      }
     }
-  }
-  {
-    const cuuint64_t dims[3] = {cuuint64_t(D), cuuint64_t(p.T), BG};
-    const cuuint64_t str[2] = {cuuint64_t(D) * E, cuuint64_t(p.T) * D * E};
-    const cuuint32_t box[3] = {64, 128, 1};
-    if (!make_map_b(encode, &mK, k, 3, dims, str, box) ||
-        !make_map_b(encode, &mV, v, 3, dims, str, box)) {
-      *why = "cuTensorMapEncodeTiled failed for k/v";
-      return cudaErrorInvalidValue;
+    {
+      const cuuint64_t dims[3] = {cuuint64_t(D), cuuint64_t(p.T), BG};
+      const cuuint64_t str[2] = {cuuint64_t(D) * E, cuuint64_t(p.T) * D * E};
+      const cuuint32_t box[3] = {64, 128, 1};
+      if (!make_map_b(encode, &mK, k, 3, dims, str, box) ||
+          !make_map_b(encode, &mV, v, 3, dims, str, box)) {
+        *why = "cuTensorMapEncodeTiled failed for k/v";
+        return cudaErrorInvalidValue;
+      }
     }
-  }
-  CUtensorMap mDQ;
-  {
-    // fp32 dq accumulator viewed like q: [bg][t][head-in-group][c]; a box is 32 columns
-    // (128 bytes) of one tile's rows (token, head), 128B-swizzled.
-    const cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(p.G), cuuint64_t(p.T), BG};
-    const cuuint64_t str[3] = {cuuint64_t(p.T) * D * 4, cuuint64_t(D) * 4,
-                               cuuint64_t(p.G) * p.T * D * 4};
-    const cuuint32_t box[4] = {32, cuuint32_t(p.G), cuuint32_t(tg.TQ), 1};
-    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-    if (encode(&mDQ, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dqacc, dims, str, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
-      *why = "cuTensorMapEncodeTiled failed for the dq accumulator";
-      return cudaErrorInvalidValue;
+    CUtensorMap mDQ;
+    {
+      // fp32 dq accumulator viewed like q: [bg][t][head-in-group][c]; a box is 32 columns
+      // (128 bytes) of one tile's rows (token, head), 128B-swizzled.
+      const cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(p.G), cuuint64_t(p.T), BG};
+      const cuuint64_t str[3] = {cuuint64_t(p.T) * D * 4, cuuint64_t(D) * 4,
+                                 cuuint64_t(p.G) * p.T * D * 4};
+      const cuuint32_t box[4] = {32, cuuint32_t(p.G), cuuint32_t(tg.TQ), 1};
+      cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+      if (encode(&mDQ, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dqacc, dims, str, box, estr,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
+        *why = "cuTensorMapEncodeTiled failed for the dq accumulator";
+        return cudaErrorInvalidValue;
+      }
     }
-  }
-  SeqArgs sa;
-  sa.dk = static_cast<__nv_bfloat16*>(dk);
-  sa.dv = static_cast<__nv_bfloat16*>(dv);
-  sa.dqacc = dqacc;
-  sa.lse = lse;
-  sa.drow = drow;
-  sa.Hkv = p.Hkv;
-  sa.T = p.T;
-  sa.G = p.G;
-  sa.TQ = tg.TQ;
-  sa.nqt = tg.nqt;
-  sa.BG = int(BG);
-  sa.causal = p.causal;
-  sa.scale = p.scale;
-  sa.scale_log2 = p.scale * kLog2eBwd;
-  e = cudaFuncSetAttribute(moda_bwd_seq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           SeqCfg<D>::kSmemBytes);
-  if (e != cudaSuccess) {
-    *why = "cudaFuncSetAttribute(sequence backward) failed";
-    return e;
-  }
-  const int nkb = (p.T + 127) / 128;
-  if ((stages & kStageSeq) && D == 128) {
-    e = cudaFuncSetAttribute(moda_bwd_seq_h_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             SeqCfg<128>::kSmemBytes);
+    SeqArgs sa;
+    sa.dk = static_cast<__nv_bfloat16*>(dk);
+    sa.dv = static_cast<__nv_bfloat16*>(dv);
+    sa.dqacc = dqacc;
+    sa.lse = lse;
+    sa.drow = drow;
+    sa.Hkv = p.Hkv;
+    sa.T = p.T;
+    sa.G = p.G;
+    sa.TQ = tg.TQ;
+    sa.nqt = tg.nqt;
+    sa.BG = int(BG);
+    sa.causal = p.causal;
+    sa.scale = p.scale;
+    sa.scale_log2 = p.scale * kLog2eBwd;
+    e = cudaFuncSetAttribute(moda_bwd_seq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SeqCfg<D>::kSmemBytes);
     if (e != cudaSuccess) {
-      *why = "cudaFuncSetAttribute(sequence backward, halves) failed";
+      *why = "cudaFuncSetAttribute(sequence backward) failed";
       return e;
     }
-    moda_bwd_seq_h_kernel<<<unsigned(BG) * nkb, kSeqHThreads, SeqCfg<128>::kSmemBytes,
-                            stream>>>(mQ, mDO, mK, mV, sa);
-  } else if (stages & kStageSeq) {
-    moda_bwd_seq_kernel<D><<<unsigned(BG) * nkb, kSeqThreads, SeqCfg<D>::kSmemBytes, stream>>>(
-      mQ, mDO, mK, mV, mDQ, sa);
-  }
-  e = cudaGetLastError();
-  if (e != cudaSuccess) {
-    *why = "sequence backward launch failed";
-    return e;
+    const int nkb = (p.T + 127) / 128;
+    if ((stages & kStageSeq) && D == 128) {
+      e = cudaFuncSetAttribute(moda_bwd_seq_h_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               SeqCfg<128>::kSmemBytes);
+      if (e != cudaSuccess) {
+        *why = "cudaFuncSetAttribute(sequence backward, halves) failed";
+        return e;
+      }
+      moda_bwd_seq_h_kernel<<<unsigned(BG) * nkb, kSeqHThreads, SeqCfg<128>::kSmemBytes,
+                              stream>>>(mQ, mDO, mK, mV, sa);
+    } else if (stages & kStageSeq) {
+      moda_bwd_seq_kernel<D><<<unsigned(BG) * nkb, kSeqThreads, SeqCfg<D>::kSmemBytes, stream>>>(
+        mQ, mDO, mK, mV, mDQ, sa);
+    }
+    e = cudaGetLastError();
+    if (e != cudaSuccess) {
+      *why = "sequence backward launch failed";
+      return e;
+    }
   }
 
   // 3. dq (bf16)

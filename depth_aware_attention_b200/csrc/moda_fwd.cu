@@ -78,6 +78,7 @@ struct FwdArgs {
   __nv_bfloat16* out;
   float* lse;
   int B, Hq, Hkv, T, L, G, TQ, JC, nqt, npairs, causal;
+  int depth_only;  // no sequence blocks: each row attends to its own token's depth only
   float scale_log2;
 };
 
@@ -164,9 +165,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const int bg = blockIdx.x % nbg;
   const int pair = a.npairs - 1 - blockIdx.x / nbg;  // heaviest (latest) pairs first
   const int tq0 = 2 * pair * a.TQ, tq1 = tq0 + a.TQ;  // first token of tile 0 / tile 1
-  const int NB0 = ((a.causal ? min(a.T, tq0 + a.TQ) : a.T) + kBN - 1) / kBN;
+  const int NB0 =
+      a.depth_only ? 0 : ((a.causal ? min(a.T, tq0 + a.TQ) : a.T) + kBN - 1) / kBN;
   // NB0 <= NB1; a tile 1 past the end of the sequence is computed but never stored
-  const int NB1 = tq1 >= a.T ? NB0 : ((a.causal ? min(a.T, tq1 + a.TQ) : a.T) + kBN - 1) / kBN;
+  const int NB1 = (tq1 >= a.T || a.depth_only)
+                      ? NB0
+                      : ((a.causal ? min(a.T, tq1 + a.TQ) : a.T) + kBN - 1) / kBN;
   const bool has_depth = a.L > 0;
   const int nchunk = has_depth ? (a.L + a.JC - 1) / a.JC : 0;
   const int NC = kDense ? 0 : nchunk;  // CUDA-core fold chunks
@@ -339,8 +343,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                  (ks > 0 || j > 0 || NC > 0) ? 1u : 0u);
         if (sm.is_depth(j) || t == 1) release(e);
       };
-      issue_s(0, 0);
-      issue_s(1, 0);
+      // (no steps at all: depth-only attention on the fold path, whose O is the fold's)
+      if (N1 > 0) {
+        issue_s(0, 0);
+        issue_s(1, 0);
+      }
       for (int j = 0; j < N1; ++j) {
         if (j < N0) {
           issue_pv(0, j);
@@ -564,7 +571,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
 
     // ---- epilogue
-    mbar_wait(bar(bars->o_final[tt]), 0, abort_flag);
+    if (NS > 0) mbar_wait(bar(bars->o_final[tt]), 0, abort_flag);
     tc_fence_after();
     const float inv_l = 1.f / l;
     const int h = (bg % a.Hkv) * a.G + hl;
@@ -677,6 +684,7 @@ cudaError_t launch_forward_d(const Problem& p, const void* q, const void* k, con
   args.nqt = tg.nqt;
   args.npairs = (tg.nqt + 1) / 2;
   args.causal = p.causal;
+  args.depth_only = p.depth_only;
   args.scale_log2 = p.scale * kLog2e;
 
   {

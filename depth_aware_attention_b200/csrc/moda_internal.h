@@ -13,6 +13,7 @@ struct Problem {
   int B, Hq, Hkv, T, L, d, G;
   int causal;
   float scale;
+  int depth_only = 0;  // 1: no sequence keys (depth-only attention); k, v unused
 };
 
 // Tile geometry shared by the kernels: a query tile holds 128 (token, head) rows, TQ

@@ -91,6 +91,35 @@ moda_status_t moda_forward_depth_path(const void *q, const void *k, const void *
                                       moda_stream_t stream);
 
 /*
+ * Depth-only attention forward: the pages' other operator (hyper.ai summary of arXiv
+ * 2603.15619, section "Depth-stream mechanisms": a layer's input is attention over the
+ * key/value pairs that earlier layers wrote for the same token position; the
+ * shijienb.com article, first half, calls its kernel Flash Depth Attention).  It is the
+ * MoDA definition with no sequence keys:
+ *   y_j = scale * <q[b,h,t], kd[b,g,t,j]>  (j < L),  out = sum_j softmax(y)_j vd[b,g,t,j],
+ *   lse = ln sum_j exp(y_j).
+ * Arguments as moda_forward without k, v and causal; L >= 1 (MODA_ERR_INVALID_ARGUMENT
+ * otherwise).  Same kernel as moda_forward with its sequence blocks removed.
+ */
+moda_status_t moda_depth_attention_forward(const void *q, const void *kd, const void *vd,
+                                           void *out, float *lse, int B, int Hq, int Hkv,
+                                           int T, int L, int d, float scale,
+                                           moda_stream_t stream);
+
+/*
+ * Depth-only attention backward: dq (bf16), dkd, dvd (bf16) of moda_depth_attention_forward
+ * given dout, from its out and lse.  Workspace as for moda_backward (size from
+ * moda_backward_workspace_size with the same sizes).  L >= 1.  Two launches: the depth
+ * part (row terms, dkd, dvd, fp32 dq) and the dq conversion; dq is deterministic here.
+ */
+moda_status_t moda_depth_attention_backward(const void *q, const void *kd, const void *vd,
+                                            const void *out, const float *lse,
+                                            const void *dout, void *dq, void *dkd, void *dvd,
+                                            void *workspace, size_t workspace_bytes, int B,
+                                            int Hq, int Hkv, int T, int L, int d, float scale,
+                                            moda_stream_t stream);
+
+/*
  * Bytes of device workspace moda_backward needs for these sizes (fp32 dQ accumulator
  * [B][Hq][T][d] plus the fp32 row terms D = <dO, out> [B][Hq][T]).
  */

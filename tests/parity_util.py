@@ -10,6 +10,11 @@ from the exact value by 1e-2 plus half a bf16 ULP of x.  No bf16 number lies wit
 some reals above 4 (bf16's spacing there is 1/32), so an exact kernel would otherwise fail
 on large gradient entries.  For |x| < 2 the extra term is at most 2^-8.  Gradients are also
 held to a relative RMS error of 1e-2 (bf16 operands carry 2^-9 relative rounding).
+
+Depth-only attention's outputs average only the L values of one token's depth keys, so
+they are O(1) and their bf16 rounding alone averages about |x| * 2^-10 (1e-3 at |x| ~ 1);
+for it the mean-abs bound too is applied beyond the output rounding
+(``mean_beyond_rounding``): the mean of max(0, err - half ULP).
 """
 from __future__ import annotations
 
@@ -60,7 +65,7 @@ def oracle_forward_window(x, t0, nt, scale, causal):
     return oracle.forward(w["q"], w["k"], w["v"], w["kd"], w["vd"], scale, causal, t0=t0)
 
 
-def compare_forward(out, lse, ref_out, ref_lse, what=""):
+def compare_forward(out, lse, ref_out, ref_lse, what="", mean_beyond_rounding=False):
     o = out.detach().to("cpu", torch.float64).numpy()
     ls = lse.detach().to("cpu", torch.float64).numpy()
     err = np.abs(o - ref_out)
@@ -68,18 +73,20 @@ def compare_forward(out, lse, ref_out, ref_lse, what=""):
     assert np.isfinite(o).all(), f"{what}: non-finite output"
     ex = excess(err, ref_out)
     assert ex.max() <= OUT_MAX, f"{what}: out max-abs {err.max():.3e} (beyond rounding {ex.max():.3e})"
-    assert err.mean() <= OUT_MEAN, f"{what}: out mean-abs {err.mean():.3e}"
+    mean = np.maximum(ex, 0.0).mean() if mean_beyond_rounding else err.mean()
+    assert mean <= OUT_MEAN, f"{what}: out mean-abs {mean:.3e}"
     assert lerr.max() <= LSE_MAX, f"{what}: lse max-abs {lerr.max():.3e}"
     return float(err.max()), float(err.mean()), float(lerr.max())
 
 
-def compare_grad(g, ref, what, max_tol=OUT_MAX, mean_tol=OUT_MEAN):
+def compare_grad(g, ref, what, max_tol=OUT_MAX, mean_tol=OUT_MEAN, mean_beyond_rounding=False):
     a = g.detach().to("cpu", torch.float64).numpy()
     err = np.abs(a - ref)
     assert np.isfinite(a).all(), f"{what}: non-finite"
     ex = excess(err, ref)
     assert ex.max() <= max_tol, f"{what}: max-abs {err.max():.3e} (beyond rounding {ex.max():.3e})"
-    assert err.mean() <= mean_tol, f"{what}: mean-abs {err.mean():.3e}"
+    mean = np.maximum(ex, 0.0).mean() if mean_beyond_rounding else err.mean()
+    assert mean <= mean_tol, f"{what}: mean-abs {mean:.3e}"
     rms = float(np.sqrt((ref ** 2).mean()))
     if rms > 0:
         rel = float(np.sqrt((err ** 2).mean())) / rms

@@ -81,6 +81,23 @@ def test_forward_depth_path_rejects_bad_arguments(kw, path, status):
     assert moda.moda_forward_depth_path(**args) == status
 
 
+def test_depth_attention_rejects_bad_arguments():
+    f = dict(q=A, kd=A * 4, vd=A * 5, out=A * 64, lse=A * 128, B=1, Hq=4, Hkv=2, T=16, L=2,
+             d=64, scale=0.125, stream=None)
+    assert moda.moda_depth_attention_forward(**dict(f, L=0)) == moda.MODA_ERR_INVALID_ARGUMENT
+    assert moda.moda_depth_attention_forward(**dict(f, kd=None)) == moda.MODA_ERR_INVALID_ARGUMENT
+    assert moda.moda_depth_attention_forward(**dict(f, d=96)) == moda.MODA_ERR_UNSUPPORTED
+    b = dict(q=A, kd=A * 4, vd=A * 5, out=A * 6, lse=A * 7, dout=A * 8, dq=A * 9, dkd=A * 12,
+             dvd=A * 13, workspace=A * 64, workspace_bytes=1 << 20, B=1, Hq=4, Hkv=2, T=16,
+             L=2, d=64, scale=0.125, stream=None)
+    assert moda.moda_depth_attention_backward(**dict(b, L=0)) == moda.MODA_ERR_INVALID_ARGUMENT
+    assert moda.moda_depth_attention_backward(**dict(b, dq=None)) == moda.MODA_ERR_INVALID_ARGUMENT
+    assert moda.moda_depth_attention_backward(**dict(b, workspace_bytes=16)) == \
+        moda.MODA_ERR_INVALID_ARGUMENT
+    assert moda.moda_depth_attention_backward(**dict(b, dkd=A * 4)) == \
+        moda.MODA_ERR_INVALID_ARGUMENT  # dkd aliases kd
+
+
 def test_forward_L0_allows_null_depth():
     # valid arguments: without a GPU the call gets as far as the device check
     st = fwd(L=0, kd=None, vd=None)
