@@ -54,16 +54,21 @@ struct BwdDepthArgs {
 
 // One token slot = D/8 consecutive threads (one 16-byte column chunk each); a CTA works
 // on kDepthThreads/(D/8) consecutive tokens of the flattened [B*Hkv][T] token list at a
-// time.  The G query rows of the token keep q and dO in shared memory (bf16); the dq
-// partial sums of up to GM heads stay in registers.
+// time.  The G query rows of the token keep q and dO unpacked to fp32 in registers when
+// GM <= 4, else in shared memory (bf16); the dq partial sums of up to GM heads stay in
+// registers.
 template <int D, int GM>
-__global__ void __launch_bounds__(kDepthThreads) moda_bwd_depth_kernel(const BwdDepthArgs a) {
+// (GM <= 4: at most 168 registers, three CTAs per SM; measured faster than 188 registers
+// and two CTAs)
+__global__ void __launch_bounds__(kDepthThreads, GM <= 4 ? 3 : 1)
+    moda_bwd_depth_kernel(const BwdDepthArgs a) {
   constexpr int NT = D / 8;
   constexpr int TPB = kDepthThreads / NT;
   extern __shared__ __align__(16) uint8_t dsm[];
   const int tid = threadIdx.x;
   const int slot = tid / NT, cs = tid % NT;
   const int G = a.G;
+  constexpr bool kReg = GM <= 4;  // q, dO of the token's heads held in registers
   const uint32_t q_s = smem_u32(dsm) + uint32_t(slot * 2 * G * D * 2);
   const uint32_t do_s = q_s + uint32_t(G * D * 2);
   const long long L = a.L;
@@ -77,10 +82,15 @@ __global__ void __launch_bounds__(kDepthThreads) moda_bwd_depth_kernel(const Bwd
     const int t = int(tkc - bg * a.T);
 
     float lse2[GM], drw[GM];
+    float qreg[kReg ? GM : 1][8], dreg[kReg ? GM : 1][8];
 #pragma unroll
     for (int h = 0; h < GM; ++h) {
       lse2[h] = 0.f;
       drw[h] = 0.f;
+      if constexpr (kReg) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) qreg[h][e] = dreg[h][e] = 0.f;
+      }
       if (h < G) {
         const long long row = (bg * G + h) * a.T + t;
         float part = 0.f;
@@ -88,11 +98,17 @@ __global__ void __launch_bounds__(kDepthThreads) moda_bwd_depth_kernel(const Bwd
           const uint4 qw = ldg_nc_v4(a.q + row * D + cs * 8);
           const uint4 dw = ldg_nc_v4(a.dout + row * D + cs * 8);
           const uint4 ow = ldg_nc_v4(a.out + row * D + cs * 8);
-          sts128(q_s + uint32_t((h * D + cs * 8) * 2), qw);
-          sts128(do_s + uint32_t((h * D + cs * 8) * 2), dw);
           float df[8], of[8];
           unpack8(dw, df);
           unpack8(ow, of);
+          if constexpr (kReg) {
+            unpack8(qw, qreg[h]);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) dreg[h][e] = df[e];
+          } else {
+            sts128(q_s + uint32_t((h * D + cs * 8) * 2), qw);
+            sts128(do_s + uint32_t((h * D + cs * 8) * 2), dw);
+          }
 #pragma unroll
           for (int e = 0; e < 8; ++e) part = fmaf(df[e], of[e], part);
           lse2[h] = a.lse[row] * kLog2eBwd;
@@ -137,8 +153,16 @@ __global__ void __launch_bounds__(kDepthThreads) moda_bwd_depth_kernel(const Bwd
         p[h] = 0.f;
         if (h < G) {
           float qf[8], df[8];
-          unpack8(lds128(q_s + uint32_t((h * D + cs * 8) * 2)), qf);
-          unpack8(lds128(do_s + uint32_t((h * D + cs * 8) * 2)), df);
+          if constexpr (kReg) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              qf[e] = qreg[h][e];
+              df[e] = dreg[h][e];
+            }
+          } else {
+            unpack8(lds128(q_s + uint32_t((h * D + cs * 8) * 2)), qf);
+            unpack8(lds128(do_s + uint32_t((h * D + cs * 8) * 2)), df);
+          }
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             y[h] = fmaf(qf[e], kf[e], y[h]);
@@ -165,8 +189,16 @@ __global__ void __launch_bounds__(kDepthThreads) moda_bwd_depth_kernel(const Bwd
           const float P = ex2(y[h] * a.scale_log2 - lse2[h]);
           const float dS = P * (p[h] - drw[h]);
           float qf[8], df[8];
-          unpack8(lds128(q_s + uint32_t((h * D + cs * 8) * 2)), qf);
-          unpack8(lds128(do_s + uint32_t((h * D + cs * 8) * 2)), df);
+          if constexpr (kReg) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              qf[e] = qreg[h][e];
+              df[e] = dreg[h][e];
+            }
+          } else {
+            unpack8(lds128(q_s + uint32_t((h * D + cs * 8) * 2)), qf);
+            unpack8(lds128(do_s + uint32_t((h * D + cs * 8) * 2)), df);
+          }
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             dv[e] = fmaf(P, df[e], dv[e]);
