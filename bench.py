@@ -57,6 +57,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle sample")
+    ap.add_argument("--decode", action="store_true",
+                    help="time single-token decode against a cache of the workload's length")
+    ap.add_argument("--decode-batch", type=int, default=8)
     ap.add_argument("--fda", action="store_true",
                     help="time depth-only attention (forward, backward) on --workload")
     ap.add_argument("--sweep", action="store_true",
@@ -591,6 +594,46 @@ def run_fda(args):
     print(json.dumps(line), flush=True)
 
 
+def run_decode(args):
+    """Single-token decode against a K/V cache of the workload's length T (per sequence),
+    batch --decode-batch sequences: average CUDA-event time and the algorithmic HBM rate
+    (K/V cache and depth entries read once, q read, out and lse written)."""
+    import depth_aware_attention_b200 as moda
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+    cfg = dict(workloads.CONFIGS[args.workload])
+    B, Hq, Hkv, S, L, d = (args.decode_batch, cfg["Hq"], cfg["Hkv"], cfg["T"], cfg["L"],
+                           cfg["d"])
+    g = torch.Generator(device=dev)
+    g.manual_seed(workloads.SEED_BASE[args.workload] * 1000 + 7)
+    mk = lambda *sh: torch.randn(*sh, generator=g, device=dev, dtype=torch.bfloat16)
+    q, k, v = mk(B, Hq, d), mk(B, Hkv, S, d), mk(B, Hkv, S, d)
+    kd = mk(B, Hkv, L, d) if L else None
+    vd = mk(B, Hkv, L, d) if L else None
+    out = torch.empty_like(q)
+    lse = torch.empty((B, Hq), device=dev, dtype=torch.float32)
+    ws = torch.empty(max(256, moda.moda_decode_workspace_size(B, Hq, Hkv, S, L, d)),
+                     device=dev, dtype=torch.uint8)
+    f = lambda: moda.decode(q, k, v, kd, vd, out=out, lse=lse, workspace=ws)
+    for _ in range(max(3, args.warmup)):
+        f()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        f()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    moda.check_device_errors()
+    ms = e0.elapsed_time(e1) / args.steps
+    nbytes = 2 * B * Hkv * S * d * 2 + 2 * B * Hkv * L * d * 2 + 2 * B * Hq * d * 2 + B * Hq * 4
+    pk = peaks()
+    print(json.dumps({"op": "decode", "workload": args.workload, "batch": B, "cache_len": S,
+                      "Hq": Hq, "Hkv": Hkv, "d": d, "L": L, "ms": round(ms, 4),
+                      "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1), "hbm_peak_gbs": pk["hbm"],
+                      "steps": args.steps}), flush=True)
+
+
 def main():
     args = parse()
     if args.sweep:
@@ -598,6 +641,9 @@ def main():
         return
     if args.fda:
         run_fda(args)
+        return
+    if args.decode:
+        run_decode(args)
         return
     world, rank, local = dist_setup(args.gpus)
     cfg = workloads.CONFIGS[args.workload]

@@ -30,7 +30,8 @@ BACKWARD_LAUNCHES = 3
 
 # Every symbol include/moda.h declares (checked by the ABI tests).
 EXPORTED = ("moda_forward", "moda_forward_depth_path", "moda_depth_attention_forward",
-            "moda_depth_attention_backward", "moda_backward", "moda_backward_workspace_size",
+            "moda_depth_attention_backward", "moda_decode", "moda_decode_workspace_size",
+            "moda_backward", "moda_backward_workspace_size",
             "moda_backward_stages", "moda_backward_noalloc", "moda_check_device_errors", "moda_status_string",
             "moda_last_error_message")
 
@@ -56,6 +57,10 @@ def _load():
     lib.moda_depth_attention_forward.restype = I
     lib.moda_depth_attention_backward.argtypes = [P] * 10 + [S] + [I] * 6 + [F, P]
     lib.moda_depth_attention_backward.restype = I
+    lib.moda_decode_workspace_size.argtypes = [I] * 6
+    lib.moda_decode_workspace_size.restype = S
+    lib.moda_decode.argtypes = [P] * 8 + [S] + [I] * 6 + [F, P]
+    lib.moda_decode.restype = I
     lib.moda_backward_workspace_size.argtypes = [I] * 6
     lib.moda_backward_workspace_size.restype = S
     lib.moda_backward.argtypes = [P] * 14 + [S] + [I] * 6 + [F, I, P]
@@ -113,6 +118,17 @@ def moda_depth_attention_backward(q, kd, vd, out, lse, dout, dq, dkd, dvd, works
     return lib.moda_depth_attention_backward(q, kd, vd, out, lse, dout, dq, dkd, dvd,
                                              workspace, workspace_bytes, B, Hq, Hkv, T, L, d,
                                              float(scale), stream)
+
+
+def moda_decode_workspace_size(B, Hq, Hkv, S, L, d):
+    return lib.moda_decode_workspace_size(B, Hq, Hkv, S, L, d)
+
+
+def moda_decode(q, k, v, kd, vd, out, lse, workspace, workspace_bytes, B, Hq, Hkv, S, L, d,
+                scale, stream):
+    """Direct call of moda_decode with raw pointers (ints)."""
+    return lib.moda_decode(q, k, v, kd, vd, out, lse, workspace, workspace_bytes, B, Hq, Hkv,
+                           S, L, d, float(scale), stream)
 
 
 def moda_backward(q, k, v, kd, vd, out, lse, dout, dq, dk, dv, dkd, dvd, workspace,
@@ -294,3 +310,29 @@ def depth_attention_backward(q, kd, vd, out, lse, dout, scale=None, workspace=No
         L, d, float(scale), _stream_handle(q.device))
     _check(st, "moda_depth_attention_backward")
     return g
+
+
+def decode(q, k, v, kd=None, vd=None, scale=None, out=None, lse=None, workspace=None):
+    """Single-token decode on the current CUDA stream: the newest token of each sequence
+    (query q [B,Hq,d]) against its K/V cache k/v [B,Hkv,S,d] (the last entry its own) and
+    its own depth entries kd/vd [B,Hkv,L,d] (or None for L = 0).  Returns (out [B,Hq,d]
+    bf16, lse [B,Hq] fp32)."""
+    import torch
+    B, Hq, d = q.shape
+    Hkv, S = k.shape[1], k.shape[2]
+    L = 0 if kd is None else kd.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq), device=q.device, dtype=torch.float32)
+    ws = lib.moda_decode_workspace_size(B, Hq, Hkv, S, L, d)
+    if workspace is None:
+        workspace = torch.empty(max(ws, 256), device=q.device, dtype=torch.uint8)
+    st = lib.moda_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(kd) if L else None,
+                         _ptr(vd) if L else None, _ptr(out), _ptr(lse), _ptr(workspace),
+                         workspace.numel(), B, Hq, Hkv, S, L, d, float(scale),
+                         _stream_handle(q.device))
+    _check(st, "moda_decode")
+    return out, lse

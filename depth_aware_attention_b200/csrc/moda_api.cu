@@ -179,6 +179,65 @@ moda_status_t moda_forward_depth_path(const void* q, const void* k, const void* 
                        depth_path, 0, stream);
 }
 
+size_t moda_decode_workspace_size(int B, int Hq, int Hkv, int S, int L, int d) {
+  if (check_sizes(B, Hq, Hkv, S, L, d) != MODA_OK || Hq / Hkv > 16) return 0;
+  moda::Problem p{B, Hq, Hkv, S, L, d, Hq / Hkv, 1, 1.f};
+  return moda::decode_workspace_bytes(p);
+}
+
+moda_status_t moda_decode(const void* q, const void* k, const void* v, const void* kd,
+                          const void* vd, void* out, float* lse, void* workspace,
+                          size_t workspace_bytes, int B, int Hq, int Hkv, int S, int L, int d,
+                          float scale, moda_stream_t stream) {
+  g_msg[0] = 0;
+  moda_status_t s = check_sizes(B, Hq, Hkv, S, L, d);
+  if (s != MODA_OK) return s;
+  if (Hq / Hkv > 16)
+    return fail(MODA_ERR_UNSUPPORTED, "decode supports at most 16 query heads per KV head");
+  if (!q || !k || !v || !out || !lse || !workspace)
+    return fail(MODA_ERR_INVALID_ARGUMENT, "q, k, v, out, lse and workspace must be non-NULL");
+  if (L > 0 && (!kd || !vd))
+    return fail(MODA_ERR_INVALID_ARGUMENT, "kd and vd must be non-NULL when L > 0");
+  const void* all[8] = {q, k, v, kd, vd, out, lse, workspace};
+  for (int i = 0; i < 8; ++i)
+    if (all[i] && !aligned16(all[i]))
+      return fail(MODA_ERR_INVALID_ARGUMENT, "every pointer must be 16-byte aligned");
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u)
+    return fail(MODA_ERR_INVALID_ARGUMENT, "workspace must be 256-byte aligned");
+  if (!(scale == scale) || scale == INFINITY || scale == -INFINITY)
+    return fail(MODA_ERR_INVALID_ARGUMENT, "scale must be finite");
+  moda::Problem p{B, Hq, Hkv, S, L, d, Hq / Hkv, 1, scale};
+  const size_t need = moda::decode_workspace_bytes(p);
+  if (workspace_bytes < need)
+    return fail(MODA_ERR_INVALID_ARGUMENT, "workspace is smaller than moda_decode_workspace_size()");
+  const size_t nq = size_t(B) * Hq * d * 2, nk = size_t(B) * Hkv * S * d * 2;
+  const size_t nd = size_t(B) * Hkv * L * d * 2, nl = size_t(B) * Hq * 4;
+  const void* ins[5] = {q, k, v, kd, vd};
+  const size_t insz[5] = {nq, nk, nk, nd, nd};
+  void* outs[3] = {out, lse, workspace};
+  const size_t outsz[3] = {nq, nl, need};
+  for (int o = 0; o < 3; ++o) {
+    for (int i = 0; i < 5; ++i)
+      if (overlaps(outs[o], outsz[o], ins[i], insz[i]))
+        return fail(MODA_ERR_INVALID_ARGUMENT, "out/lse/workspace must not overlap an input");
+    for (int o2 = o + 1; o2 < 3; ++o2)
+      if (overlaps(outs[o], outsz[o], outs[o2], outsz[o2]))
+        return fail(MODA_ERR_INVALID_ARGUMENT, "out, lse and workspace must not overlap");
+  }
+  s = check_device();
+  if (s != MODA_OK) return s;
+  moda::EncodeTiledFn enc = get_encoder();
+  if (!enc) return fail(MODA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
+  const char* why = "";
+  cudaError_t e = moda::launch_decode(p, q, k, v, kd, vd, out, lse, workspace, enc,
+                                      static_cast<cudaStream_t>(stream), &why);
+  if (e != cudaSuccess) {
+    snprintf(g_msg, sizeof(g_msg), "%s: %s", why, cudaGetErrorString(e));
+    return MODA_ERR_CUDA;
+  }
+  return MODA_OK;
+}
+
 size_t moda_backward_workspace_size(int B, int Hq, int Hkv, int T, int L, int d) {
   if (check_sizes(B, Hq, Hkv, T, L, d) != MODA_OK) return 0;
   moda::Problem p{B, Hq, Hkv, T, L, d, Hq / Hkv, 1, 1.f};

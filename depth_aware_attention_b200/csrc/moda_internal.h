@@ -64,6 +64,18 @@ cudaError_t launch_backward(const Problem& p, const void* q, const void* k, cons
                             unsigned stages, EncodeTiledFn encode, cudaStream_t stream,
                             const char** why);
 
+// Single-token decode: the sequence is split into ranges of 128-key blocks, one CTA per
+// (batch, KV head, range); `T` of the Problem is the cache length S.
+struct DecodeSplit {
+  int nsplit, blocks_per_split;
+};
+DecodeSplit decode_split(const Problem& p);
+size_t decode_workspace_bytes(const Problem& p);
+cudaError_t launch_decode(const Problem& p, const void* q, const void* k, const void* v,
+                          const void* kd, const void* vd, void* out, float* lse,
+                          void* workspace, EncodeTiledFn encode, cudaStream_t stream,
+                          const char** why);
+
 // Backward stages (bit mask): 1 row terms + depth part + dq accumulator initialisation,
 // 2 sequence part (adds to the dq accumulator), 4 dq conversion to bf16.
 constexpr unsigned kStageDepth = 1u, kStageSeq = 2u, kStageConvert = 4u, kStagesAll = 7u;

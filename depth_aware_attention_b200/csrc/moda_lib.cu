@@ -4,3 +4,4 @@
 #include "moda_fwd.cu"
 #include "moda_bwd.cu"
 #include "moda_noalloc.cu"
+#include "moda_decode.cu"

@@ -361,6 +361,13 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
                : "memory");
 }
 
+// 16-bit shared-memory load (zero-extended).
+__device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
+  uint16_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+  return v;
+}
+
 // 16-byte global load through the read-only (non-coherent) path.
 __device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
   uint4 v;

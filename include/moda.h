@@ -120,6 +120,26 @@ moda_status_t moda_depth_attention_backward(const void *q, const void *kd, const
                                             moda_stream_t stream);
 
 /*
+ * Single-token decode: the forward's row for the newest token of each sequence.  The
+ * K/V cache holds S sequence keys/values, the last of them the newest token's own; its
+ * query row sees all S of them (the causal row of position S-1) and its own L depth
+ * keys, in one joint softmax (hyper.ai summary of arXiv 2603.15619, section
+ * "Mixture-of-Depths Attention (MoDA)").  The pages do not describe decoding; this is
+ * that definition restricted to one query token per sequence.
+ *   q, out: [B, Hq, d]    k, v: [B, Hkv, S, d]    kd, vd: [B, Hkv, L, d] (NULL iff L == 0)
+ *   lse: [B, Hq] fp32     workspace: >= moda_decode_workspace_size(...) bytes, 256-byte
+ *   aligned, owned by the caller, contents irrelevant between calls.
+ * Hq/Hkv <= 16 (MODA_ERR_UNSUPPORTED otherwise).  The sequence is split over CTAs
+ * (a function of the sizes only) and the partial softmax states are combined by a second
+ * launch.  Other argument rules as moda_forward.
+ */
+size_t moda_decode_workspace_size(int B, int Hq, int Hkv, int S, int L, int d);
+moda_status_t moda_decode(const void *q, const void *k, const void *v, const void *kd,
+                          const void *vd, void *out, float *lse, void *workspace,
+                          size_t workspace_bytes, int B, int Hq, int Hkv, int S, int L, int d,
+                          float scale, moda_stream_t stream);
+
+/*
  * Bytes of device workspace moda_backward needs for these sizes (fp32 dQ accumulator
  * [B][Hq][T][d] plus the fp32 row terms D = <dO, out> [B][Hq][T]).
  */

@@ -98,6 +98,22 @@ def test_depth_attention_rejects_bad_arguments():
         moda.MODA_ERR_INVALID_ARGUMENT  # dkd aliases kd
 
 
+def test_decode_rejects_bad_arguments():
+    base = dict(q=A, k=A * 2, v=A * 3, kd=A * 4, vd=A * 5, out=A * 64, lse=A * 128,
+                workspace=A * 256, workspace_bytes=1 << 24, B=1, Hq=4, Hkv=2, S=16, L=2, d=64,
+                scale=0.125, stream=None)
+    st = lambda **kw: moda.moda_decode(**dict(base, **kw))
+    assert st(S=0) == moda.MODA_ERR_INVALID_ARGUMENT
+    assert st(kd=None) == moda.MODA_ERR_INVALID_ARGUMENT
+    assert st(workspace_bytes=16) == moda.MODA_ERR_INVALID_ARGUMENT
+    assert st(workspace=A * 256 + 16) == moda.MODA_ERR_INVALID_ARGUMENT
+    assert st(out=A * 2) == moda.MODA_ERR_INVALID_ARGUMENT  # out aliases k
+    assert st(Hq=64, Hkv=2) == moda.MODA_ERR_UNSUPPORTED
+    assert st(d=96) == moda.MODA_ERR_UNSUPPORTED
+    assert moda.moda_decode_workspace_size(1, 16, 4, 65536, 32, 128) > 0
+    assert moda.moda_decode_workspace_size(1, 64, 2, 100, 1, 128) == 0
+
+
 def test_forward_L0_allows_null_depth():
     # valid arguments: without a GPU the call gets as far as the device check
     st = fwd(L=0, kd=None, vd=None)
