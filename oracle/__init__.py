@@ -237,3 +237,20 @@ def depth_backward(q, kd, vd, dout, scale, out=None, t0=0, nthreads=None):
     if rc != 0:
         raise ValueError("moda_oracle_depth_backward rejected the sizes")
     return dict(dq=dq, dkd=dkd, dvd=dvd, out=o, lse=lse)
+
+
+def depth_kv_projection(x, w, Hkv, d):
+    """The layer's depth-stream key/value pair that the fused write stores into slot l:
+    K = x W_k^T and V = x W_v^T for every token, per KV head (hyper.ai summary,
+    section "Hardware-efficient implementation": each layer appends its K/V to the depth
+    stream that later layers read; the depth cache layout is [B, Hkv, T, L, d]).
+
+    x [B,T,hidden]; w [2*Hkv*d, hidden] (rows 0..Hkv*d-1 project K, the rest V, the
+    nn.Linear weight convention).  Returns (k_slot, v_slot), each [B,Hkv,T,d] float64: the
+    values slot l of kd / vd must hold.  One fp64 matrix product, then a reshape.
+    """
+    x, w = _f64(x), _f64(w)
+    B, T, _ = x.shape
+    y = x.reshape(B * T, -1) @ w.T                       # [B*T, 2*Hkv*d]
+    y = y.reshape(B, T, 2, Hkv, d).transpose(2, 0, 3, 1, 4)  # [2, B, Hkv, T, d]
+    return np.ascontiguousarray(y[0]), np.ascontiguousarray(y[1])

@@ -427,3 +427,33 @@ def test_depth_backward_given_own_out_equals_exact():
     h = oracle.depth_backward(x["q"], x["kd"], x["vd"], x["dout"], 0.4, out=g["out"])
     for n in ("dq", "dkd", "dvd"):
         assert np.abs(g[n] - h[n]).max() < 1e-14, n
+
+
+# ---------------------------------------------------------------- depth-stream write
+def test_depth_kv_projection_selects_columns_with_one_hot_weights():
+    """A weight row that is one-hot at column c copies x[..., c]: checks the K/V split
+    and the (head, column) placement of every output element."""
+    B, T, hidden, Hkv, d = 2, 3, 16, 2, 4
+    x = torch.randn(B, T, hidden, dtype=torch.float64)
+    rng = np.random.default_rng(7)
+    src = rng.integers(0, hidden, size=2 * Hkv * d)
+    w = np.zeros((2 * Hkv * d, hidden))
+    w[np.arange(2 * Hkv * d), src] = 1.0
+    k, v = oracle.depth_kv_projection(x, w, Hkv, d)
+    xn = x.numpy()
+    for part, arr in ((0, k), (1, v)):
+        for g in range(Hkv):
+            for c in range(d):
+                col = src[part * Hkv * d + g * d + c]
+                assert np.array_equal(arr[:, g, :, c], xn[:, :, col])
+
+
+def test_depth_kv_projection_is_linear_in_weights():
+    B, T, hidden, Hkv, d = 1, 5, 8, 1, 4
+    x = torch.randn(B, T, hidden, dtype=torch.float64)
+    w1 = np.random.default_rng(1).standard_normal((2 * Hkv * d, hidden))
+    w2 = np.random.default_rng(2).standard_normal((2 * Hkv * d, hidden))
+    a1, b1 = oracle.depth_kv_projection(x, w1, Hkv, d)
+    a2, b2 = oracle.depth_kv_projection(x, w2, Hkv, d)
+    a3, b3 = oracle.depth_kv_projection(x, 2.0 * w1 - w2, Hkv, d)
+    assert np.abs(a3 - (2 * a1 - a2)).max() < 1e-12 and np.abs(b3 - (2 * b1 - b2)).max() < 1e-12
