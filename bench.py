@@ -57,6 +57,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle sample")
+    ap.add_argument("--kvwrite", action="store_true",
+                    help="time the fused depth-stream write for the workload's tokens")
     ap.add_argument("--decode", action="store_true",
                     help="time single-token decode against a cache of the workload's length")
     ap.add_argument("--decode-batch", type=int, default=8)
@@ -634,6 +636,54 @@ def run_decode(args):
                       "steps": args.steps}), flush=True)
 
 
+def run_kvwrite(args):
+    """Fused depth-stream write for the workload's tokens at the 1.5B-layer projection
+    shape (hidden 2048 -> K|V of Hkv x d): CUDA-event time and TFLOP/s of the fused
+    kernel, beside torch's matmul followed by the copy into the depth-cache slot (the
+    unfused two-step it replaces; cuBLAS, for context)."""
+    import depth_aware_attention_b200 as moda
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+    cfg = workloads.CONFIGS[args.workload]
+    B, T, Hkv, d, L = cfg["B"], cfg["T"], cfg["Hkv"], cfg["d"], max(cfg["L"], 1)
+    hidden = 2048
+    g = torch.Generator(device=dev)
+    g.manual_seed(workloads.SEED_BASE[args.workload] * 1000 + 8)
+    x = torch.randn(B, T, hidden, generator=g, device=dev, dtype=torch.bfloat16)
+    w = (torch.randn(2 * Hkv * d, hidden, generator=g, device=dev) / 45.25).to(torch.bfloat16)
+    kd = torch.zeros(B, Hkv, T, L, d, device=dev, dtype=torch.bfloat16)
+    vd = torch.zeros_like(kd)
+    slot = L - 1
+
+    def unfused():
+        y = torch.matmul(x, w.t()).view(B, T, 2, Hkv, d)
+        kd[:, :, :, slot].copy_(y[:, :, 0].transpose(1, 2))
+        vd[:, :, :, slot].copy_(y[:, :, 1].transpose(1, 2))
+
+    res = {}
+    for name, f in (("fused", lambda: moda.depth_kv_write(x, w, kd, vd, slot)),
+                    ("torch_matmul_then_copy", unfused)):
+        for _ in range(max(3, args.warmup)):
+            f()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            f()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        res[name] = e0.elapsed_time(e1) / args.steps
+    moda.check_device_errors()
+    flops = 2.0 * B * T * hidden * 2 * Hkv * d
+    pk = peaks()
+    print(json.dumps({"op": "depth-stream write", "workload": args.workload, "tokens": B * T,
+                      "hidden": hidden, "Hkv": Hkv, "d": d, "L": L,
+                      "fused_ms": round(res["fused"], 4),
+                      "fused_tflops": round(flops / (res["fused"] * 1e-3) / 1e12, 1),
+                      "unfused_ms": round(res["torch_matmul_then_copy"], 4),
+                      "bf16_peak_tflops": pk["bf16"], "steps": args.steps}), flush=True)
+
+
 def main():
     args = parse()
     if args.sweep:
@@ -644,6 +694,9 @@ def main():
         return
     if args.decode:
         run_decode(args)
+        return
+    if args.kvwrite:
+        run_kvwrite(args)
         return
     world, rank, local = dist_setup(args.gpus)
     cfg = workloads.CONFIGS[args.workload]

@@ -31,6 +31,7 @@ BACKWARD_LAUNCHES = 3
 # Every symbol include/moda.h declares (checked by the ABI tests).
 EXPORTED = ("moda_forward", "moda_forward_depth_path", "moda_depth_attention_forward",
             "moda_depth_attention_backward", "moda_decode", "moda_decode_workspace_size",
+            "moda_depth_kv_write",
             "moda_backward", "moda_backward_workspace_size",
             "moda_backward_stages", "moda_backward_noalloc", "moda_check_device_errors", "moda_status_string",
             "moda_last_error_message")
@@ -61,6 +62,8 @@ def _load():
     lib.moda_decode_workspace_size.restype = S
     lib.moda_decode.argtypes = [P] * 8 + [S] + [I] * 6 + [F, P]
     lib.moda_decode.restype = I
+    lib.moda_depth_kv_write.argtypes = [P] * 4 + [I] * 7 + [P]
+    lib.moda_depth_kv_write.restype = I
     lib.moda_backward_workspace_size.argtypes = [I] * 6
     lib.moda_backward_workspace_size.restype = S
     lib.moda_backward.argtypes = [P] * 14 + [S] + [I] * 6 + [F, I, P]
@@ -129,6 +132,11 @@ def moda_decode(q, k, v, kd, vd, out, lse, workspace, workspace_bytes, B, Hq, Hk
     """Direct call of moda_decode with raw pointers (ints)."""
     return lib.moda_decode(q, k, v, kd, vd, out, lse, workspace, workspace_bytes, B, Hq, Hkv,
                            S, L, d, float(scale), stream)
+
+
+def moda_depth_kv_write(x, w, kd, vd, B, T, hidden, Hkv, d, L, slot, stream):
+    """Direct call of moda_depth_kv_write with raw pointers (ints)."""
+    return lib.moda_depth_kv_write(x, w, kd, vd, B, T, hidden, Hkv, d, L, slot, stream)
 
 
 def moda_backward(q, k, v, kd, vd, out, lse, dout, dq, dk, dv, dkd, dvd, workspace,
@@ -336,3 +344,14 @@ def decode(q, k, v, kd=None, vd=None, scale=None, out=None, lse=None, workspace=
                          _stream_handle(q.device))
     _check(st, "moda_decode")
     return out, lse
+
+
+def depth_kv_write(x, w, kd, vd, slot):
+    """Fused depth-stream write on the current CUDA stream: slot ``slot`` of kd / vd
+    [B,Hkv,T,L,d] receives K|V = x w^T for x [B,T,hidden] and w [2*Hkv*d, hidden] (rows
+    0..Hkv*d-1 project K, the rest V).  Other slots are untouched."""
+    B, T, hidden = x.shape
+    _, Hkv, _, L, d = kd.shape
+    st = lib.moda_depth_kv_write(_ptr(x), _ptr(w), _ptr(kd), _ptr(vd), B, T, hidden, Hkv, d,
+                                 L, int(slot), _stream_handle(x.device))
+    _check(st, "moda_depth_kv_write")

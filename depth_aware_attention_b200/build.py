@@ -15,7 +15,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmoda_b200.so")
-SOURCES = ["moda_lib.cu", "moda_api.cu", "moda_fwd.cu", "moda_bwd.cu", "moda_noalloc.cu", "moda_decode.cu",
+SOURCES = ["moda_lib.cu", "moda_api.cu", "moda_fwd.cu", "moda_bwd.cu", "moda_noalloc.cu", "moda_decode.cu", "moda_kvwrite.cu",
            "sm100.cuh", "moda_internal.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

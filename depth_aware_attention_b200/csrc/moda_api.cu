@@ -238,6 +238,42 @@ moda_status_t moda_decode(const void* q, const void* k, const void* v, const voi
   return MODA_OK;
 }
 
+moda_status_t moda_depth_kv_write(const void* x, const void* w, void* kd, void* vd, int B,
+                                  int T, int hidden, int Hkv, int d, int L, int slot,
+                                  moda_stream_t stream) {
+  g_msg[0] = 0;
+  if (B < 1 || T < 1 || hidden < 1 || Hkv < 1 || L < 1)
+    return fail(MODA_ERR_INVALID_ARGUMENT, "B, T, hidden, Hkv and L must be positive");
+  if (slot < 0 || slot >= L) return fail(MODA_ERR_INVALID_ARGUMENT, "slot must lie in [0, L)");
+  if (d != 64 && d != 128) return fail(MODA_ERR_UNSUPPORTED, "d must be 64 or 128");
+  if ((Hkv * d) % 128 != 0)
+    return fail(MODA_ERR_UNSUPPORTED, "Hkv * d must be a multiple of 128");
+  if (hidden % 8 != 0)
+    return fail(MODA_ERR_UNSUPPORTED, "hidden must be a multiple of 8 (16-byte rows)");
+  if (!x || !w || !kd || !vd)
+    return fail(MODA_ERR_INVALID_ARGUMENT, "x, w, kd and vd must be non-NULL");
+  if (!aligned16(x) || !aligned16(w) || !aligned16(kd) || !aligned16(vd))
+    return fail(MODA_ERR_INVALID_ARGUMENT, "every pointer must be 16-byte aligned");
+  const size_t nx = size_t(B) * T * hidden * 2, nw = size_t(2) * Hkv * d * hidden * 2;
+  const size_t nd = size_t(B) * Hkv * T * L * d * 2;
+  if (overlaps(kd, nd, x, nx) || overlaps(kd, nd, w, nw) || overlaps(vd, nd, x, nx) ||
+      overlaps(vd, nd, w, nw) || overlaps(kd, nd, vd, nd))
+    return fail(MODA_ERR_INVALID_ARGUMENT, "kd/vd must not overlap x, w or each other");
+  moda_status_t s = check_device();
+  if (s != MODA_OK) return s;
+  moda::EncodeTiledFn enc = get_encoder();
+  if (!enc) return fail(MODA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
+  moda::KvWriteProblem p{B, T, hidden, Hkv, d, L, slot};
+  const char* why = "";
+  cudaError_t e = moda::launch_kvwrite(p, x, w, kd, vd, enc, static_cast<cudaStream_t>(stream),
+                                       &why);
+  if (e != cudaSuccess) {
+    snprintf(g_msg, sizeof(g_msg), "%s: %s", why, cudaGetErrorString(e));
+    return MODA_ERR_CUDA;
+  }
+  return MODA_OK;
+}
+
 size_t moda_backward_workspace_size(int B, int Hq, int Hkv, int T, int L, int d) {
   if (check_sizes(B, Hq, Hkv, T, L, d) != MODA_OK) return 0;
   moda::Problem p{B, Hq, Hkv, T, L, d, Hq / Hkv, 1, 1.f};

@@ -76,6 +76,15 @@ cudaError_t launch_decode(const Problem& p, const void* q, const void* k, const 
                           void* workspace, EncodeTiledFn encode, cudaStream_t stream,
                           const char** why);
 
+// Fused depth-stream write: K|V = X W^T for B*T tokens, stored into slot `slot` of the
+// [B, Hkv, T, L, d] depth caches.
+struct KvWriteProblem {
+  int B, T, hidden, Hkv, d, L, slot;
+};
+cudaError_t launch_kvwrite(const KvWriteProblem& p, const void* x, const void* w, void* kd,
+                           void* vd, EncodeTiledFn encode, cudaStream_t stream,
+                           const char** why);
+
 // Backward stages (bit mask): 1 row terms + depth part + dq accumulator initialisation,
 // 2 sequence part (adds to the dq accumulator), 4 dq conversion to bf16.
 constexpr unsigned kStageDepth = 1u, kStageSeq = 2u, kStageConvert = 4u, kStagesAll = 7u;

@@ -1,0 +1,210 @@
+// moda_kvwrite.cu -- fused depth-stream write for B200 (sm_100a).
+//
+// Every sublayer appends its key/value pair to the depth stream that later layers read
+// (hyper.ai summary of arXiv 2603.15619, section "Hardware-efficient implementation":
+// the depth cache is kept flattened per (batch, KV head) so that token t's entries are
+// the contiguous rows [t*L, (t+1)*L), layout [B, Hkv, T, L, d]).  This kernel is the
+// projection that produces layer l's pair, K|V = X W^T, with the depth cache as its
+// epilogue: each token's K and V rows go straight into slot l of kd / vd, with no
+// separate copy of a [B*T, 2*Hkv*d] product.
+//
+// One CTA computes a 128-token x 128-column tile of X W^T on the tensor cores:
+//   warp 4     TMA producer: 64-wide K-slices of the X tile and the W tile (both K-major,
+//              128B-swizzled) through a ring of shared-memory stages;
+//   warp 5     tcgen05 issuer: four 128x128x16 MMAs per stage into a TMEM accumulator,
+//              the stage released by a commit once they are done;
+//   warps 0-3  epilogue: TMEM lane r = the tile's token r; 128 columns = one head (d =
+//              128) or two (d = 64) of K or of V, converted to bf16 and stored as
+//              contiguous 16-byte words into the token's slot-l row(s).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "moda_internal.h"
+#include "sm100.cuh"
+
+namespace moda {
+
+namespace {
+
+constexpr int kKwRows = 128;    // tokens per tile
+constexpr int kKwCols = 128;    // output columns per tile
+constexpr int kKwBK = 64;       // K (hidden) elements per stage: 128 bytes per row
+constexpr int kKwStages = 6;
+constexpr int kKwThreads = 192; // warps 0-3 epilogue, 4 producer, 5 issuer
+constexpr int kKwTile = 16384;  // 128 rows x 128 bytes
+
+struct KwArgs {
+  __nv_bfloat16 *kd, *vd;
+  int M, T, hidden, Hkv, d, L, slot, nk;
+};
+
+struct KwBars {
+  uint64_t full[kKwStages], empty[kKwStages];
+  uint64_t done;
+  uint32_t tmem_base;
+  int abort;
+};
+
+constexpr int kKwOffBar = 2 * kKwStages * kKwTile;
+constexpr int kKwSmemBytes = 1024 + kKwOffBar + 256;
+
+__global__ void __launch_bounds__(kKwThreads, 1)
+    moda_kvwrite_kernel(const __grid_constant__ CUtensorMap tmX,
+                        const __grid_constant__ CUtensorMap tmW, const KwArgs a) {
+  extern __shared__ uint8_t kw_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(kw_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t s0 = smem_u32(smem);
+  KwBars* bars = reinterpret_cast<KwBars*>(smem + kKwOffBar);
+  volatile int* abort_flag = &bars->abort;
+  auto bar = [&](uint64_t& b) { return smem_u32(&b); };
+  auto sA = [&](int s) { return s0 + uint32_t(2 * s) * kKwTile; };
+  auto sB = [&](int s) { return s0 + uint32_t(2 * s + 1) * kKwTile; };
+
+  const int warp = threadIdx.x >> 5;
+  const int m0 = blockIdx.x * kKwRows;
+  const int n0 = blockIdx.y * kKwCols;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kKwStages; ++s) {
+      mbar_init(bar(bars->full[s]), 1);
+      mbar_init(bar(bars->empty[s]), 1);
+    }
+    mbar_init(bar(bars->done), 1);
+    bars->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_u32(&bars->tmem_base), kKwCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ TMA producer
+    if (elect_one()) {
+      tma_prefetch_desc(&tmX);
+      tma_prefetch_desc(&tmW);
+      for (int kb = 0; kb < a.nk; ++kb) {
+        const int s = kb % kKwStages;
+        if (kb >= kKwStages)
+          mbar_wait(bar(bars->empty[s]), ((kb / kKwStages) - 1) & 1, abort_flag);
+        mbar_expect_tx(bar(bars->full[s]), 2 * kKwTile);
+        tma_load_2d(sA(s), &tmX, bar(bars->full[s]), kb * kKwBK, m0);
+        tma_load_2d(sB(s), &tmW, bar(bars->full[s]), kb * kKwBK, n0);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ tcgen05 issuer
+    if (elect_one()) {
+      constexpr uint32_t idesc = make_idesc_bf16(kKwRows, kKwCols, 0, 0);
+      for (int kb = 0; kb < a.nk; ++kb) {
+        const int s = kb % kKwStages;
+        mbar_wait(bar(bars->full[s]), (kb / kKwStages) & 1, abort_flag);
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < kKwBK / 16; ++ks)
+          mma_ss(tmem, make_sdesc_sw128(sA(s) + ks * 32, 16, 1024),
+                 make_sdesc_sw128(sB(s) + ks * 32, 16, 1024), idesc,
+                 (kb > 0 || ks > 0) ? 1u : 0u);
+        tc_commit(bar(bars->empty[s]));
+      }
+      tc_commit(bar(bars->done));
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue warps 0-3
+    const int r = threadIdx.x;  // TMEM lane = token m0 + r
+    const uint32_t lane_base = uint32_t(warp * 32) << 16;
+    mbar_wait(bar(bars->done), 0, abort_flag);
+    tc_fence_after();
+    const int m = m0 + r;
+    const bool valid = m < a.M;
+    const int b = valid ? m / a.T : 0, t = valid ? m - (m / a.T) * a.T : 0;
+    const int hd = a.Hkv * a.d;
+    const int part = n0 / hd;  // 0: K columns, 1: V columns (tiles never straddle)
+    __nv_bfloat16* base = part ? a.vd : a.kd;
+#pragma unroll
+    for (int cc = 0; cc < kKwCols / 32; ++cc) {
+      uint32_t o[32];
+      tmem_ld32(tmem + lane_base + cc * 32, o);
+      tmem_wait_ld();
+      if (valid) {
+        const int n = (n0 - part * hd) + cc * 32;  // column within K (or V)
+        const int g = n / a.d, c = n - g * a.d;
+        uint4* dst = reinterpret_cast<uint4*>(
+            base + ((((size_t(b) * a.Hkv + g) * a.T + t) * a.L + a.slot) * a.d + c));
+#pragma unroll
+        for (int v4 = 0; v4 < 4; ++v4) {
+          float f[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(o[v4 * 8 + e]);
+          dst[v4] = pack8(f, 1.f);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kKwCols);
+  }
+}
+
+bool make_map_2d(EncodeTiledFn encode, CUtensorMap* map, const void* base, cuuint64_t inner,
+                 cuuint64_t rows) {
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t str[1] = {inner * 2};
+  const cuuint32_t box[2] = {kKwBK, 128};
+  cuuint32_t estr[2] = {1, 1};
+  return encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, str,
+                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_kvwrite(const KvWriteProblem& p, const void* x, const void* w, void* kd,
+                           void* vd, EncodeTiledFn encode, cudaStream_t stream,
+                           const char** why) {
+  const int M = p.B * p.T, N = 2 * p.Hkv * p.d;
+  CUtensorMap mX, mW;
+  if (!make_map_2d(encode, &mX, x, cuuint64_t(p.hidden), cuuint64_t(M)) ||
+      !make_map_2d(encode, &mW, w, cuuint64_t(p.hidden), cuuint64_t(N))) {
+    *why = "cuTensorMapEncodeTiled failed for x/w";
+    return cudaErrorInvalidValue;
+  }
+  KwArgs a;
+  a.kd = static_cast<__nv_bfloat16*>(kd);
+  a.vd = static_cast<__nv_bfloat16*>(vd);
+  a.M = M;
+  a.T = p.T;
+  a.hidden = p.hidden;
+  a.Hkv = p.Hkv;
+  a.d = p.d;
+  a.L = p.L;
+  a.slot = p.slot;
+  a.nk = (p.hidden + kKwBK - 1) / kKwBK;
+  cudaError_t e = cudaFuncSetAttribute(moda_kvwrite_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kKwSmemBytes);
+  if (e != cudaSuccess) {
+    *why = "cudaFuncSetAttribute(depth-stream write) failed";
+    return e;
+  }
+  const dim3 grid(unsigned((M + kKwRows - 1) / kKwRows), unsigned(N / kKwCols));
+  moda_kvwrite_kernel<<<grid, kKwThreads, kKwSmemBytes, stream>>>(mX, mW, a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) *why = "depth-stream write launch failed";
+  return e;
+}
+
+}  // namespace moda

@@ -5,3 +5,4 @@
 #include "moda_bwd.cu"
 #include "moda_noalloc.cu"
 #include "moda_decode.cu"
+#include "moda_kvwrite.cu"

@@ -140,6 +140,23 @@ moda_status_t moda_decode(const void *q, const void *k, const void *v, const voi
                           float scale, moda_stream_t stream);
 
 /*
+ * Fused depth-stream write: the projection that produces a sublayer's depth key/value
+ * pair, with the depth cache as its output (hyper.ai summary of arXiv 2603.15619,
+ * section "Hardware-efficient implementation": every layer appends its K/V to the
+ * depth stream, kept as [B, Hkv, T, L, d] so that token t's entries are contiguous).
+ *   x:  [B, T, hidden] bf16 (the sublayer's input hidden states)
+ *   w:  [2*Hkv*d, hidden] bf16 (rows 0..Hkv*d-1 project K, the rest V; nn.Linear layout)
+ *   kd, vd: [B, Hkv, T, L, d] bf16; slot l of each receives
+ *           kd[b,g,t,l,:] = (x[b,t,:] . w[g*d + c, :])_c,  vd likewise with rows Hkv*d + ...
+ *           computed with fp32 accumulation and rounded to bf16; other slots are untouched.
+ * Requirements: 0 <= slot < L; d in {64, 128}; Hkv*d a multiple of 128; hidden a multiple
+ * of 8 (MODA_ERR_UNSUPPORTED otherwise).  One tcgen05 GEMM launch; no workspace.
+ */
+moda_status_t moda_depth_kv_write(const void *x, const void *w, void *kd, void *vd, int B,
+                                  int T, int hidden, int Hkv, int d, int L, int slot,
+                                  moda_stream_t stream);
+
+/*
  * Bytes of device workspace moda_backward needs for these sizes (fp32 dQ accumulator
  * [B][Hq][T][d] plus the fp32 row terms D = <dO, out> [B][Hq][T]).
  */

@@ -114,6 +114,21 @@ def test_decode_rejects_bad_arguments():
     assert moda.moda_decode_workspace_size(1, 64, 2, 100, 1, 128) == 0
 
 
+def test_depth_kv_write_rejects_bad_arguments():
+    base = dict(x=A, w=A * 2, kd=A * 64, vd=A * 128, B=1, T=16, hidden=64, Hkv=2, d=64, L=3,
+                slot=1, stream=None)
+    st = lambda **kw: moda.moda_depth_kv_write(**dict(base, **kw))
+    assert st(slot=3) == moda.MODA_ERR_INVALID_ARGUMENT
+    assert st(slot=-1) == moda.MODA_ERR_INVALID_ARGUMENT
+    assert st(L=0) == moda.MODA_ERR_INVALID_ARGUMENT
+    assert st(x=None) == moda.MODA_ERR_INVALID_ARGUMENT
+    assert st(kd=A * 64 + 8) == moda.MODA_ERR_INVALID_ARGUMENT
+    assert st(vd=A * 64 + 16) == moda.MODA_ERR_INVALID_ARGUMENT  # vd overlaps kd
+    assert st(d=96) == moda.MODA_ERR_UNSUPPORTED
+    assert st(Hkv=1) == moda.MODA_ERR_UNSUPPORTED      # Hkv*d = 64
+    assert st(hidden=60) == moda.MODA_ERR_UNSUPPORTED  # rows not 16-byte multiples
+
+
 def test_forward_L0_allows_null_depth():
     # valid arguments: without a GPU the call gets as far as the device check
     st = fwd(L=0, kd=None, vd=None)
