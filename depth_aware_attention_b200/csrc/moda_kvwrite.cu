@@ -8,14 +8,15 @@
 // epilogue: each token's K and V rows go straight into slot l of kd / vd, with no
 // separate copy of a [B*T, 2*Hkv*d] product.
 //
-// One CTA computes a 128-token x 128-column tile of X W^T on the tensor cores:
-//   warp 4     TMA producer: 64-wide K-slices of the X tile and the W tile (both K-major,
-//              128B-swizzled) through a ring of shared-memory stages;
-//   warp 5     tcgen05 issuer: four 128x128x16 MMAs per stage into a TMEM accumulator,
-//              the stage released by a commit once they are done;
-//   warps 0-3  epilogue: TMEM lane r = the tile's token r; 128 columns = one head (d =
-//              128) or two (d = 64) of K or of V, converted to bf16 and stored as
-//              contiguous 16-byte words into the token's slot-l row(s).
+// One CTA computes a 128-token x 256-column tile of X W^T on the tensor cores:
+//   warp 4     TMA producer: 64-wide K-slices of the X tile (128 rows) and the W tile
+//              (256 rows; both K-major, 128B-swizzled) through a ring of shared-memory
+//              stages;
+//   warp 5     tcgen05 issuer: four 128x256x16 MMAs per stage into a 256-column TMEM
+//              accumulator, the stage released by a commit once they are done;
+//   warps 0-3  epilogue: TMEM lane r = the tile's token r; each 32-column chunk lies in
+//              one head of K or of V, converted to bf16 and stored as contiguous 16-byte
+//              words into the token's slot-l row.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -28,11 +29,11 @@ namespace moda {
 namespace {
 
 constexpr int kKwRows = 128;    // tokens per tile
-constexpr int kKwCols = 128;    // output columns per tile
+constexpr int kKwCols = 256;    // output columns per tile
 constexpr int kKwBK = 64;       // K (hidden) elements per stage: 128 bytes per row
-constexpr int kKwStages = 6;
+constexpr int kKwStages = 4;
 constexpr int kKwThreads = 192; // warps 0-3 epilogue, 4 producer, 5 issuer
-constexpr int kKwTile = 16384;  // 128 rows x 128 bytes
+constexpr int kKwTile = 16384;  // 128 rows x 128 bytes: the x slice; the W slice is two
 
 struct KwArgs {
   __nv_bfloat16 *kd, *vd;
@@ -46,7 +47,8 @@ struct KwBars {
   int abort;
 };
 
-constexpr int kKwOffBar = 2 * kKwStages * kKwTile;
+constexpr int kKwStage = 3 * kKwTile;  // x slice (128 rows) + W slice (256 rows)
+constexpr int kKwOffBar = kKwStages * kKwStage;
 constexpr int kKwSmemBytes = 1024 + kKwOffBar + 256;
 
 __global__ void __launch_bounds__(kKwThreads, 1)
@@ -59,8 +61,8 @@ __global__ void __launch_bounds__(kKwThreads, 1)
   KwBars* bars = reinterpret_cast<KwBars*>(smem + kKwOffBar);
   volatile int* abort_flag = &bars->abort;
   auto bar = [&](uint64_t& b) { return smem_u32(&b); };
-  auto sA = [&](int s) { return s0 + uint32_t(2 * s) * kKwTile; };
-  auto sB = [&](int s) { return s0 + uint32_t(2 * s + 1) * kKwTile; };
+  auto sA = [&](int s) { return s0 + uint32_t(s) * kKwStage; };
+  auto sB = [&](int s) { return s0 + uint32_t(s) * kKwStage + kKwTile; };
 
   const int warp = threadIdx.x >> 5;
   const int m0 = blockIdx.x * kKwRows;
@@ -93,9 +95,10 @@ __global__ void __launch_bounds__(kKwThreads, 1)
         const int s = kb % kKwStages;
         if (kb >= kKwStages)
           mbar_wait(bar(bars->empty[s]), ((kb / kKwStages) - 1) & 1, abort_flag);
-        mbar_expect_tx(bar(bars->full[s]), 2 * kKwTile);
+        mbar_expect_tx(bar(bars->full[s]), kKwStage);
         tma_load_2d(sA(s), &tmX, bar(bars->full[s]), kb * kKwBK, m0);
         tma_load_2d(sB(s), &tmW, bar(bars->full[s]), kb * kKwBK, n0);
+        tma_load_2d(sB(s) + kKwTile, &tmW, bar(bars->full[s]), kb * kKwBK, n0 + 128);
       }
     }
     __syncwarp();
@@ -127,15 +130,16 @@ __global__ void __launch_bounds__(kKwThreads, 1)
     const bool valid = m < a.M;
     const int b = valid ? m / a.T : 0, t = valid ? m - (m / a.T) * a.T : 0;
     const int hd = a.Hkv * a.d;
-    const int part = n0 / hd;  // 0: K columns, 1: V columns (tiles never straddle)
-    __nv_bfloat16* base = part ? a.vd : a.kd;
 #pragma unroll
     for (int cc = 0; cc < kKwCols / 32; ++cc) {
       uint32_t o[32];
       tmem_ld32(tmem + lane_base + cc * 32, o);
       tmem_wait_ld();
       if (valid) {
-        const int n = (n0 - part * hd) + cc * 32;  // column within K (or V)
+        const int na = n0 + cc * 32;
+        const int part = na / hd;  // 0: K columns, 1: V columns
+        __nv_bfloat16* base = part ? a.vd : a.kd;
+        const int n = na - part * hd;  // column within K (or V)
         const int g = n / a.d, c = n - g * a.d;
         uint4* dst = reinterpret_cast<uint4*>(
             base + ((((size_t(b) * a.Hkv + g) * a.T + t) * a.L + a.slot) * a.d + c));
