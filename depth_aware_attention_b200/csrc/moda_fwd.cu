@@ -493,14 +493,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const bool need_mask = a.causal ? (kbase + kBN - 1 > t0) : (kbase + kBN > a.T);
         if (need_mask) {
 #pragma unroll
-          for (int c = 0; c < kBN; ++c) {
+          for (int c = 0; c < kBN; ++c)
             if (kbase + c > key_lim) s[c] = __float_as_uint(-INFINITY);
-            mx = fmaxf(mx, __uint_as_float(s[c]));
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < kBN; ++c) mx = fmaxf(mx, __uint_as_float(s[c]));
         }
+        // two chains of three-input maxima
+        float mx1 = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < kBN; c += 4) {
+          mx = fmax3(mx, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+          mx1 = fmax3(mx1, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
+        }
+        mx = fmaxf(mx, mx1);
       }
       const float m_cand = fmaxf(m, mx * a.scale_log2);
       const bool grow = m_cand > m + kRescaleThreshold;
@@ -530,22 +533,27 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             tmem_st16(tS + 16 * q, zero);
         }
       } else {
+        // p = 2^(s*scale*log2e - m): one packed FFMA feeds each pair of exp2, one packed
+        // add accumulates each pair
+        const float2 sl2 = make_float2(a.scale_log2, a.scale_log2);
+        const float2 nm2 = make_float2(-m_use, -m_use);
+        float2 ps2 = make_float2(0.f, 0.f);
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           uint32_t pk[32];
 #pragma unroll
           for (int c = 0; c < 64; c += 2) {
-            // p = 2^(s*scale*log2e - m): one FFMA feeds each exp2
-            const float p0 =
-                ex2(fmaf(__uint_as_float(s[half * 64 + c]), a.scale_log2, -m_use));
-            const float p1 =
-                ex2(fmaf(__uint_as_float(s[half * 64 + c + 1]), a.scale_log2, -m_use));
-            ps0 += p0;
-            ps1 += p1;
-            pk[c / 2] = pack_bf16x2(p0, p1);
+            const float2 x = ffma2(make_float2(__uint_as_float(s[half * 64 + c]),
+                                               __uint_as_float(s[half * 64 + c + 1])),
+                                   sl2, nm2);
+            const float2 p = make_float2(ex2(x.x), ex2(x.y));
+            ps2 = fadd2(ps2, p);
+            pk[c / 2] = pack_bf16x2(p.x, p.y);
           }
           tmem_st32(tS + half * 32, pk);
         }
+        ps0 = ps2.x;
+        ps1 = ps2.y;
       }
       const float ps = ps0 + ps1;
       l = l * alpha + ps;

@@ -457,6 +457,13 @@ __device__ __forceinline__ void axpy8_bf16(uint16_t p, uint4 v, float (&acc)[8])
       : "h"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w));
 }
 
+// Maximum of three floats in one instruction (sm_100a).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // Packed fp32 pair arithmetic (sm_100a: one instruction for both lanes of the pair).
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
   uint64_t d;
