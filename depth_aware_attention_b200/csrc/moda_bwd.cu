@@ -163,11 +163,15 @@ __global__ void __launch_bounds__(kDepthThreads, GM <= 4 ? 3 : 1)
             unpack8(lds128(q_s + uint32_t((h * D + cs * 8) * 2)), qf);
             unpack8(lds128(do_s + uint32_t((h * D + cs * 8) * 2)), df);
           }
+          // packed pairs: one f32x2 FMA per two products
+          float2 y2 = make_float2(0.f, 0.f), p2 = make_float2(0.f, 0.f);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            y[h] = fmaf(qf[e], kf[e], y[h]);
-            p[h] = fmaf(df[e], vf[e], p[h]);
+          for (int e = 0; e < 8; e += 2) {
+            y2 = ffma2(make_float2(qf[e], qf[e + 1]), make_float2(kf[e], kf[e + 1]), y2);
+            p2 = ffma2(make_float2(df[e], df[e + 1]), make_float2(vf[e], vf[e + 1]), p2);
           }
+          y[h] = y2.x + y2.y;
+          p[h] = p2.x + p2.y;
         }
       }
 #pragma unroll
@@ -199,11 +203,18 @@ __global__ void __launch_bounds__(kDepthThreads, GM <= 4 ? 3 : 1)
             unpack8(lds128(q_s + uint32_t((h * D + cs * 8) * 2)), qf);
             unpack8(lds128(do_s + uint32_t((h * D + cs * 8) * 2)), df);
           }
+          const float2 P2 = make_float2(P, P), dS2 = make_float2(dS, dS);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            dv[e] = fmaf(P, df[e], dv[e]);
-            dk[e] = fmaf(dS, qf[e], dk[e]);
-            dq[h][e] = fmaf(dS, kf[e], dq[h][e]);
+          for (int e = 0; e < 8; e += 2) {
+            const float2 v2 = ffma2(P2, make_float2(df[e], df[e + 1]),
+                                    make_float2(dv[e], dv[e + 1]));
+            const float2 k2 = ffma2(dS2, make_float2(qf[e], qf[e + 1]),
+                                    make_float2(dk[e], dk[e + 1]));
+            const float2 q2 = ffma2(dS2, make_float2(kf[e], kf[e + 1]),
+                                    make_float2(dq[h][e], dq[h][e + 1]));
+            dv[e] = v2.x; dv[e + 1] = v2.y;
+            dk[e] = k2.x; dk[e + 1] = k2.y;
+            dq[h][e] = q2.x; dq[h][e + 1] = q2.y;
           }
         }
       }
