@@ -499,10 +499,11 @@ def run_reference(args, world, rank):
 
 
 def run_sweep(args):
-    """Forward time over T in {4K..64K} x L in {0, 8, 32, 128} at the 1.5B-layer head shape
-    (B=1, Hq=16, Hkv=4, d=128): TFLOP/s and the ratio time(L=0)/time(L) per point, the
-    shape of the pages' efficiency-scaling experiment (the depth overhead shrinks as T
-    grows).  Prints one JSON line per point, then a markdown table."""
+    """Forward time over T in {4K..64K} x L in {0, 8, 32, 128} x group size G in {4, 8}
+    (B=1, Hkv=4, Hq=4G, d=128; G=4 is the 1.5B-layer head shape): TFLOP/s and the ratio
+    time(L=0)/time(L) per point, the shape of the pages' efficiency-scaling experiment
+    (the depth overhead shrinks as T grows).  Prints one JSON line per point, then a
+    markdown table."""
     import depth_aware_attention_b200 as moda
     dev = torch.device("cuda", 0)
     stream = torch.cuda.current_stream(dev)
