@@ -34,8 +34,6 @@ __device__ __forceinline__ uint64_t globaltimer() {
   return t;
 }
 
-__device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31; }
-
 __device__ __forceinline__ bool elect_one() {
   uint32_t pred = 0;
   asm volatile(
@@ -170,14 +168,6 @@ __device__ __forceinline__ void tma_reduce_add_4d(const CUtensorMap* map, uint32
       "r"(x), "r"(y), "r"(z), "r"(w), "r"(src)
       : "memory");
 }
-// global[gdst, gdst+bytes) += shared[ssrc, ssrc+bytes) (fp32 add in L2); both addresses
-// 16-byte aligned, bytes a multiple of 16.  Tracked by this thread's bulk async-group.
-__device__ __forceinline__ void bulk_reduce_add_f32(float* gdst, uint32_t ssrc, uint32_t bytes) {
-  asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(
-                   gdst),
-               "r"(ssrc), "r"(bytes)
-               : "memory");
-}
 __device__ __forceinline__ void bulk_commit_group() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
@@ -294,17 +284,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
       : "r"(taddr));
 }
 
-// 32 lanes x 32 bit, 16 consecutive columns per thread.
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* r) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
-        "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]),
-        "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-}
-
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -391,13 +370,6 @@ __device__ __forceinline__ void red_add_f32(float* p, float a) {
   asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(a) : "memory");
 }
 
-// Atomic add of four consecutive floats (16-byte aligned) in global memory.
-__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1,%2,%3,%4};" ::"l"(p), "f"(a), "f"(b),
-               "f"(c), "f"(d)
-               : "memory");
-}
-
 // Unpacks 8 bf16 (one 16-byte word group) to fp32.
 __device__ __forceinline__ void unpack8(uint4 w, float (&f)[8]) {
   f[0] = bf16lo(w.x); f[1] = bf16hi(w.x); f[2] = bf16lo(w.y); f[3] = bf16hi(w.y);
@@ -411,17 +383,6 @@ __device__ __forceinline__ uint4 pack8(const float (&f)[8], float s) {
   w.z = pack_bf16x2(f[4] * s, f[5] * s);
   w.w = pack_bf16x2(f[6] * s, f[7] * s);
   return w;
-}
-
-// Copies the 16-byte aligned gmem region [src, src+bytes) into shared memory; the
-// mbarrier's transaction count receives `bytes` on completion.
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
-                                          uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, "
-      "[%3];" ::"r"(dst),
-      "l"(src), "r"(bytes), "r"(bar)
-      : "memory");
 }
 
 // acc + <a, b> over 8 bf16 pairs (a, b: 8 packed bf16 each) with the mixed-precision
