@@ -40,6 +40,9 @@ constexpr float kLog2eBwd = 1.4426950408889634f;
 
 // ============================================================ 1. depth + row terms
 constexpr int kDepthThreads = 128;
+constexpr int kDepthU = 4;     // depth entries per load batch
+constexpr int kDepthRing = 4;  // per-thread cp.async ring stages (batches in flight: 3)
+constexpr int kDepthRingBytes = kDepthRing * kDepthU * 2 * kDepthThreads * 16;
 
 struct BwdDepthArgs {
   const __nv_bfloat16 *q, *out, *dout, *kd, *vd;
@@ -71,6 +74,15 @@ __global__ void __launch_bounds__(kDepthThreads, GM <= 4 ? 3 : 1)
   constexpr bool kReg = GM <= 4;  // q, dO of the token's heads held in registers
   const uint32_t q_s = smem_u32(dsm) + uint32_t(slot * 2 * G * D * 2);
   const uint32_t do_s = q_s + uint32_t(G * D * 2);
+  // Per-thread ring of depth-entry chunks filled by cp.async, kDNS batches of kU entries
+  // (kd and vd) deep, after the q/dO slots (none when they live in registers): each thread
+  // copies and reads back only its own 16-byte chunks, so no barrier is involved.
+  constexpr int kU = kDepthU;
+  constexpr int kDNS = kDepthRing;
+  const uint32_t ring = smem_u32(dsm) + (kReg ? 0u : uint32_t(TPB * 2 * G * D * 2));
+  auto rslot = [&](int stg, int u, int kv) {
+    return ring + uint32_t((((stg * kU + u) * 2 + kv) * kDepthThreads + tid) * 16);
+  };
   const long long L = a.L;
 
   for (long long base = (long long)blockIdx.x * TPB; base < a.ntok;
@@ -128,15 +140,34 @@ __global__ void __launch_bounds__(kDepthThreads, GM <= 4 ? 3 : 1)
       for (int e = 0; e < 8; ++e) dq[h][e] = 0.f;
 
     const long long tok_off = (bg * a.T + t) * L * D + cs * 8;
-    constexpr int kU = 4;  // depth entries whose loads are in flight together
+    const long long nbat = (L + kU - 1) / kU;
+    // batch b's copies (an empty group past the last batch keeps the group count uniform)
+    auto issue = [&](long long b) {
+      const int stg = int(b % kDNS);
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const long long j = b * kU + u;
+        if (valid && j < L) {
+          cp_async16(rslot(stg, u, 0), a.kd + tok_off + j * D);
+          cp_async16(rslot(stg, u, 1), a.vd + tok_off + j * D);
+        }
+      }
+      cp_async_commit();
+    };
+#pragma unroll
+    for (int b = 0; b < kDNS - 1; ++b) issue(b);
     for (long long j0 = 0; j0 < L; j0 += kU) {
+      const long long b = j0 / kU;
+      issue(b + kDNS - 1);
+      cp_async_wait<kDNS - 1>();  // batch b has landed
+      const int stg = int(b % kDNS);
       uint4 kwu[kU], vwu[kU];
 #pragma unroll
       for (int u = 0; u < kU; ++u) {
         kwu[u] = vwu[u] = make_uint4(0, 0, 0, 0);
         if (valid && j0 + u < L) {
-          kwu[u] = ldg_nc_v4(a.kd + tok_off + (j0 + u) * D);
-          vwu[u] = ldg_nc_v4(a.vd + tok_off + (j0 + u) * D);
+          kwu[u] = lds128(rslot(stg, u, 0));
+          vwu[u] = lds128(rslot(stg, u, 1));
         }
       }
 #pragma unroll
@@ -224,6 +255,8 @@ __global__ void __launch_bounds__(kDepthThreads, GM <= 4 ? 3 : 1)
       }
       }
     }
+    cp_async_wait<0>();  // (only empty groups remain) before the ring is reused
+    (void)nbat;
     if (valid) {
 #pragma unroll
       for (int h = 0; h < GM; ++h) {
@@ -1080,7 +1113,8 @@ int sm_count() {
 template <int D, int GM>
 cudaError_t launch_depth(const BwdDepthArgs& a, cudaStream_t stream, const char** why) {
   const int tpb = kDepthThreads / (D / 8);
-  const size_t smem = size_t(tpb) * 2 * a.G * D * 2;
+  // q/dO slots (not needed when they live in registers) + the per-thread cp.async ring
+  const size_t smem = (GM <= 4 ? 0 : size_t(tpb) * 2 * a.G * D * 2) + kDepthRingBytes;
   cudaError_t e = cudaFuncSetAttribute(moda_bwd_depth_kernel<D, GM>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) {
