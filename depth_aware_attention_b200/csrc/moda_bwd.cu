@@ -40,8 +40,8 @@ constexpr float kLog2eBwd = 1.4426950408889634f;
 
 // ============================================================ 1. depth + row terms
 constexpr int kDepthThreads = 128;
-constexpr int kDepthU = 4;     // depth entries per load batch
-constexpr int kDepthRing = 4;  // per-thread cp.async ring stages (batches in flight: 3)
+constexpr int kDepthU = 2;     // depth entries per load batch
+constexpr int kDepthRing = 8;  // per-thread cp.async ring stages (batches in flight: 7)
 constexpr int kDepthRingBytes = kDepthRing * kDepthU * 2 * kDepthThreads * 16;
 
 struct BwdDepthArgs {
