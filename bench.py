@@ -337,18 +337,11 @@ def run_moda(args, world, rank, local):
     # Extras the metric names: the L=0 causal ratio and the depth stream's HBM rate.
     extras = {}
     if args.workload.startswith("long-64k") and L > 0:
-        def t_fwd(kdx, vdx, n=3):
-            for _ in range(2):
-                moda.forward(q, k, v, kdx, vdx, scale, True, out=out, lse=lse)
-            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a0.record(stream)
-            for _ in range(n):
-                moda.forward(q, k, v, kdx, vdx, scale, True, out=out, lse=lse)
-            a1.record(stream)
-            torch.cuda.synchronize(dev)
-            return a0.elapsed_time(a1) / n
-        ms_l = t_fwd(kd, vd)
-        ms_0 = t_fwd(None, None)
+        fwd_ms = interleaved_ms(
+            {"L": lambda: moda.forward(q, k, v, kd, vd, scale, True, out=out, lse=lse),
+             "L0": lambda: moda.forward(q, k, v, None, None, scale, True, out=out, lse=lse)},
+            stream, dev, rounds=7)
+        ms_l, ms_0 = fwd_ms["L"], fwd_ms["L0"]
         cfg0 = dict(cfg, L=0)
         tf_l = fwd_flops / (ms_l * 1e-3) / 1e12
         tf_0 = workloads.forward_flops(**cfg0) / (ms_0 * 1e-3) / 1e12
@@ -498,6 +491,29 @@ def run_reference(args, world, rank):
     return dict(value=value, ms=flops / (value * 1e12) * 1e3, cpu=dict(last, value=value))
 
 
+def interleaved_ms(fns, stream, dev, rounds, warmup=2):
+    """Median CUDA-event time (ms) of one call of each function in ``fns``, the calls
+    interleaved round by round with the starting function rotated each round.  On a
+    power-capped GPU the clock drifts over a run, so timing one variant after another
+    biases their ratio toward whichever ran first; interleaving cancels that."""
+    keys = list(fns)
+    for _ in range(warmup):
+        for key in keys:
+            fns[key]()
+    torch.cuda.synchronize(dev)
+    ev = {key: [] for key in keys}
+    for r in range(rounds):
+        for i in range(len(keys)):
+            key = keys[(r + i) % len(keys)]
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fns[key]()
+            e1.record(stream)
+            ev[key].append((e0, e1))
+    torch.cuda.synchronize(dev)
+    return {key: statistics.median(a.elapsed_time(b) for a, b in ev[key]) for key in keys}
+
+
 def run_sweep(args):
     """Forward time over T in {4K..64K} x L in {0, 8, 32, 128} x group size G in {4, 8}
     (B=1, Hkv=4, Hq=4G, d=128; G=4 is the 1.5B-layer head shape): TFLOP/s and the ratio
@@ -508,39 +524,31 @@ def run_sweep(args):
     dev = torch.device("cuda", 0)
     stream = torch.cuda.current_stream(dev)
     rows = []
+    Ls = (0, 8, 32, 128)
     for G, T in [(g, t) for g in (4, 8) for t in (4096, 8192, 16384, 32768, 65536)]:
-        ms0 = None
-        for L in (0, 8, 32, 128):
+        # q, k, v are shared by every L (same seeds); each L gets its own depth cache.
+        xs = {L: workloads.make_inputs(dict(B=1, T=T, Hq=4 * G, Hkv=4, d=128, L=L),
+                                       900 + T // 4096, dev) for L in Ls}
+        x0 = xs[0]
+        out = torch.empty_like(x0["q"])
+        lse = torch.empty(x0["q"].shape[:3], device=dev, dtype=torch.float32)
+        fns = {L: (lambda L=L: moda.forward(x0["q"], x0["k"], x0["v"], xs[L]["kd"],
+                                             xs[L]["vd"], None, True, out=out, lse=lse))
+               for L in Ls}
+        ms = interleaved_ms(fns, stream, dev, rounds=5 if T >= 32768 else 15)
+        moda.check_device_errors()
+        for L in Ls:
             cfg = dict(B=1, T=T, Hq=4 * G, Hkv=4, d=128, L=L)
-            x = workloads.make_inputs(cfg, 900 + T // 4096, dev)
-            out = torch.empty_like(x["q"])
-            lse = torch.empty(x["q"].shape[:3], device=dev, dtype=torch.float32)
-            f = lambda: moda.forward(x["q"], x["k"], x["v"], x["kd"], x["vd"], None, True,
-                                     out=out, lse=lse)
-            for _ in range(3):
-                f()
-            torch.cuda.synchronize(dev)
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            n = 3 if T >= 32768 else 10
-            e0.record(stream)
-            for _ in range(n):
-                f()
-            e1.record(stream)
-            torch.cuda.synchronize(dev)
-            ms = e0.elapsed_time(e1) / n
-            moda.check_device_errors()
-            if L == 0:
-                ms0 = ms
-            tf = workloads.forward_flops(**cfg) / (ms * 1e-3) / 1e12
-            row = {"G": G, "T": T, "L": L, "ms": round(ms, 4), "tflops": round(tf, 1),
-                   "time_ratio_L0_over_L": round(ms0 / ms, 4),
+            tf = workloads.forward_flops(**cfg) / (ms[L] * 1e-3) / 1e12
+            row = {"G": G, "T": T, "L": L, "ms": round(ms[L], 4), "tflops": round(tf, 1),
+                   "time_ratio_L0_over_L": round(ms[0] / ms[L], 4),
                    "depth_gbs_from_difference": (round(workloads.depth_bytes(**cfg) /
-                                                       ((ms - ms0) * 1e-3) / 1e9, 1)
-                                                 if L and ms > ms0 * 1.02 else None)}
+                                                       ((ms[L] - ms[0]) * 1e-3) / 1e9, 1)
+                                                 if L and ms[L] > ms[0] * 1.02 else None)}
             print(json.dumps(row), flush=True)
             rows.append(row)
-            del x, out, lse
-            torch.cuda.empty_cache()
+        del xs, x0, fns, out, lse
+        torch.cuda.empty_cache()
     print("| G | T | L | ms | TFLOP/s | time(L=0)/time(L) |")
     print("|---|---|---|---|---|---|")
     for r in rows:
