@@ -1,0 +1,48 @@
+"""bench.py's host side on CPU: the reference arm's JSON line and the L2 statement.
+
+The reference arm times the fp64 oracle on the host cores in the same metric as the GPU
+arm, so it runs here; the GPU arm's line is checked by the GPU runs themselves.
+"""
+import json
+import os
+import subprocess
+import sys
+
+import bench
+import workloads
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_reference_arm_prints_one_contract_line():
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps",
+           "1", "--warmup", "3", "--cpu-seconds", "1", "--workload", "layer-4k"]
+    r = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference"
+    assert line["metric"] == bench.METRIC and line["unit"] == "TFLOP/s"
+    assert line["n_gpus"] == 1 and line["steps"] == 1 and line["warmup"] == 3
+    assert line["higher_is_better"] is True and line["vs_baseline"] is None
+    assert line["config"]["workload"] == "layer-4k"
+    assert line["config"]["T"] == 4096 and line["config"]["L"] == 24
+    assert line["value"] > 0
+    # ms_per_step is the whole step's algorithmic FLOPs at the measured rate
+    flops = workloads.forward_flops(**workloads.CONFIGS["layer-4k"]) * (1 + bench.BWD_FLOP_FACTOR)
+    assert abs(line["ms_per_step"] - flops / (line["value"] * 1e12) * 1e3) <= \
+        1e-3 * line["ms_per_step"] + 1e-3
+    cpu = line["cpu_baseline"]
+    assert cpu["kind"] == "oracle" and cpu["value"] == line["value"] and cpu["cores"] >= 1
+    assert cpu["unit"] == "TFLOP/s" and cpu["sample"]
+    e2e = line["e2e"]
+    assert e2e["value"] == line["value"] and e2e["unit"] == "TFLOP/s"
+    assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+
+
+def test_l2_statement_follows_the_workload_size():
+    assert bench.l2_note(workloads.CONFIGS["long-64k"]) == "inputs larger than L2 (no flush)"
+    assert bench.l2_note(workloads.CONFIGS["fwd-bwd-16k"]) == "inputs larger than L2 (no flush)"
+    note = bench.l2_note(workloads.CONFIGS["tiny"])
+    assert "fit in L2" in note and "not a headline figure" in note
