@@ -185,11 +185,46 @@ def _stream_handle(device):
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
 
 
+def _ndim(name, t, n):
+    if t is None or t.dim() != n:
+        raise ValueError(f"{name} must be a {n}-D tensor")
+
+
 def _dims(q, k, kd):
+    _ndim("q", q, 4)
+    _ndim("k", k, 4)
+    if kd is not None:
+        _ndim("kd", kd, 5)
     B, Hq, T, d = q.shape
     Hkv = k.shape[1]
     L = 0 if kd is None else kd.shape[3]
     return B, Hq, Hkv, T, L, d
+
+
+def _validate(device, specs, workspace=None):
+    """Check each tensor's shape, dtype, contiguity and device before its pointer goes to
+    the library, which sees only pointers and sizes: a tensor smaller than the sizes say,
+    a strided view or another dtype would make a kernel read or write outside it.
+    ``specs`` maps a name to (tensor, expected shape, expected dtype)."""
+    for name, (t, shape, dtype) in specs.items():
+        if t is None:
+            raise ValueError(f"{name} is required")
+        if tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{name} has shape {tuple(t.shape)}; expected {tuple(shape)}")
+        if t.dtype != dtype:
+            raise TypeError(f"{name} has dtype {t.dtype}; expected {dtype}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        if t.device != device:
+            raise ValueError(f"{name} is on {t.device}; expected {device}")
+    if workspace is not None and (not workspace.is_contiguous() or workspace.device != device):
+        raise ValueError(f"workspace must be a contiguous tensor on {device}")
+    if device.type != "cuda":
+        raise ValueError(f"the library runs on CUDA tensors, not on {device}")
+
+
+def _nbytes(t):
+    return t.numel() * t.element_size()
 
 
 def forward(q, k, v, kd=None, vd=None, scale=None, causal=True, out=None, lse=None,
@@ -209,6 +244,12 @@ def forward(q, k, v, kd=None, vd=None, scale=None, causal=True, out=None, lse=No
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, Hq, T), device=q.device, dtype=torch.float32)
+    bf, kv = torch.bfloat16, (B, Hkv, T, d)
+    spec = dict(q=(q, (B, Hq, T, d), bf), k=(k, kv, bf), v=(v, kv, bf),
+                out=(out, (B, Hq, T, d), bf), lse=(lse, (B, Hq, T), torch.float32))
+    if L:
+        spec.update(kd=(kd, (B, Hkv, T, L, d), bf), vd=(vd, (B, Hkv, T, L, d), bf))
+    _validate(q.device, spec)
     args = (_ptr(q), _ptr(k), _ptr(v), _ptr(kd) if L else None, _ptr(vd) if L else None,
             _ptr(out), _ptr(lse), B, Hq, Hkv, T, L, d, float(scale), int(bool(causal)))
     if depth_path == 0:
@@ -250,11 +291,18 @@ def backward(q, k, v, kd, vd, out, lse, dout, scale=None, causal=True, workspace
         g["dvd"] = torch.empty_like(vd)
     if not L:
         g["dkd"] = g["dvd"] = None
+    bf, qs, kv, ds = torch.bfloat16, (B, Hq, T, d), (B, Hkv, T, d), (B, Hkv, T, L, d)
+    spec = dict(q=(q, qs, bf), k=(k, kv, bf), v=(v, kv, bf), out=(out, qs, bf),
+                lse=(lse, (B, Hq, T), torch.float32), dout=(dout, qs, bf),
+                dq=(g["dq"], qs, bf), dk=(g["dk"], kv, bf), dv=(g["dv"], kv, bf))
+    if L:
+        spec.update(kd=(kd, ds, bf), vd=(vd, ds, bf), dkd=(g["dkd"], ds, bf),
+                    dvd=(g["dvd"], ds, bf))
+    _validate(q.device, spec, workspace)
     args = (_ptr(q), _ptr(k), _ptr(v), _ptr(kd) if L else None, _ptr(vd) if L else None,
             _ptr(out), _ptr(lse), _ptr(dout), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]),
-            _ptr(g["dkd"]), _ptr(g["dvd"]), _ptr(workspace),
-            workspace.numel() * workspace.element_size(), B, Hq, Hkv, T, L, d, float(scale),
-            int(bool(causal)))
+            _ptr(g["dkd"]), _ptr(g["dvd"]), _ptr(workspace), _nbytes(workspace),
+            B, Hq, Hkv, T, L, d, float(scale), int(bool(causal)))
     if stages == 7:
         st = lib.moda_backward(*args, _stream_handle(q.device))
         _check(st, "moda_backward")
@@ -278,6 +326,8 @@ def depth_attention_forward(q, kd, vd, scale=None, out=None, lse=None):
     q [B,Hq,T,d], kd/vd [B,Hkv,T,L,d]: contiguous bf16 CUDA tensors.
     """
     import torch
+    _ndim("q", q, 4)
+    _ndim("kd", kd, 5)
     B, Hq, T, d = q.shape
     Hkv, L = kd.shape[1], kd.shape[3]
     if scale is None:
@@ -286,6 +336,10 @@ def depth_attention_forward(q, kd, vd, scale=None, out=None, lse=None):
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, Hq, T), device=q.device, dtype=torch.float32)
+    bf, ds = torch.bfloat16, (B, Hkv, T, L, d)
+    _validate(q.device, dict(q=(q, (B, Hq, T, d), bf), kd=(kd, ds, bf), vd=(vd, ds, bf),
+                             out=(out, (B, Hq, T, d), bf),
+                             lse=(lse, (B, Hq, T), torch.float32)))
     st = lib.moda_depth_attention_forward(_ptr(q), _ptr(kd), _ptr(vd), _ptr(out), _ptr(lse),
                                           B, Hq, Hkv, T, L, d, float(scale),
                                           _stream_handle(q.device))
@@ -298,6 +352,8 @@ def depth_attention_backward(q, kd, vd, out, lse, dout, scale=None, workspace=No
     """Depth-only attention backward on the current CUDA stream.  Returns dict(dq, dkd,
     dvd); ``workspace``/``grads`` as for backward()."""
     import torch
+    _ndim("q", q, 4)
+    _ndim("kd", kd, 5)
     B, Hq, T, d = q.shape
     Hkv, L = kd.shape[1], kd.shape[3]
     if scale is None:
@@ -312,9 +368,14 @@ def depth_attention_backward(q, kd, vd, out, lse, dout, scale=None, workspace=No
         g["dkd"] = torch.empty_like(kd)
     if g.get("dvd") is None:
         g["dvd"] = torch.empty_like(vd)
+    bf, qs, ds = torch.bfloat16, (B, Hq, T, d), (B, Hkv, T, L, d)
+    _validate(q.device, dict(q=(q, qs, bf), kd=(kd, ds, bf), vd=(vd, ds, bf),
+                             out=(out, qs, bf), lse=(lse, (B, Hq, T), torch.float32),
+                             dout=(dout, qs, bf), dq=(g["dq"], qs, bf),
+                             dkd=(g["dkd"], ds, bf), dvd=(g["dvd"], ds, bf)), workspace)
     st = lib.moda_depth_attention_backward(
         _ptr(q), _ptr(kd), _ptr(vd), _ptr(out), _ptr(lse), _ptr(dout), _ptr(g["dq"]),
-        _ptr(g["dkd"]), _ptr(g["dvd"]), _ptr(workspace), workspace.numel(), B, Hq, Hkv, T,
+        _ptr(g["dkd"]), _ptr(g["dvd"]), _ptr(workspace), _nbytes(workspace), B, Hq, Hkv, T,
         L, d, float(scale), _stream_handle(q.device))
     _check(st, "moda_depth_attention_backward")
     return g
@@ -326,6 +387,10 @@ def decode(q, k, v, kd=None, vd=None, scale=None, out=None, lse=None, workspace=
     its own depth entries kd/vd [B,Hkv,L,d] (or None for L = 0).  Returns (out [B,Hq,d]
     bf16, lse [B,Hq] fp32)."""
     import torch
+    _ndim("q", q, 3)
+    _ndim("k", k, 4)
+    if kd is not None:
+        _ndim("kd", kd, 4)
     B, Hq, d = q.shape
     Hkv, S = k.shape[1], k.shape[2]
     L = 0 if kd is None else kd.shape[2]
@@ -338,9 +403,15 @@ def decode(q, k, v, kd=None, vd=None, scale=None, out=None, lse=None, workspace=
     ws = lib.moda_decode_workspace_size(B, Hq, Hkv, S, L, d)
     if workspace is None:
         workspace = torch.empty(max(ws, 256), device=q.device, dtype=torch.uint8)
+    bf, kv = torch.bfloat16, (B, Hkv, S, d)
+    spec = dict(q=(q, (B, Hq, d), bf), k=(k, kv, bf), v=(v, kv, bf), out=(out, (B, Hq, d), bf),
+                lse=(lse, (B, Hq), torch.float32))
+    if L:
+        spec.update(kd=(kd, (B, Hkv, L, d), bf), vd=(vd, (B, Hkv, L, d), bf))
+    _validate(q.device, spec, workspace)
     st = lib.moda_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(kd) if L else None,
                          _ptr(vd) if L else None, _ptr(out), _ptr(lse), _ptr(workspace),
-                         workspace.numel(), B, Hq, Hkv, S, L, d, float(scale),
+                         _nbytes(workspace), B, Hq, Hkv, S, L, d, float(scale),
                          _stream_handle(q.device))
     _check(st, "moda_decode")
     return out, lse
@@ -350,8 +421,14 @@ def depth_kv_write(x, w, kd, vd, slot):
     """Fused depth-stream write on the current CUDA stream: slot ``slot`` of kd / vd
     [B,Hkv,T,L,d] receives K|V = x w^T for x [B,T,hidden] and w [2*Hkv*d, hidden] (rows
     0..Hkv*d-1 project K, the rest V).  Other slots are untouched."""
+    import torch
+    _ndim("x", x, 3)
+    _ndim("kd", kd, 5)
     B, T, hidden = x.shape
     _, Hkv, _, L, d = kd.shape
+    bf, ds = torch.bfloat16, (B, Hkv, T, L, d)
+    _validate(x.device, dict(x=(x, (B, T, hidden), bf), w=(w, (2 * Hkv * d, hidden), bf),
+                             kd=(kd, ds, bf), vd=(vd, ds, bf)))
     st = lib.moda_depth_kv_write(_ptr(x), _ptr(w), _ptr(kd), _ptr(vd), B, T, hidden, Hkv, d,
                                  L, int(slot), _stream_handle(x.device))
     _check(st, "moda_depth_kv_write")
