@@ -18,6 +18,8 @@ Parity status: forward, backward, the backward with a given output, the row-weig
 and the depth-only forward/backward are pinned by the
 ``-m "not gpu"`` tests in ``tests/test_oracle_pins.py`` (library special cases, closed
 forms, invariants, finite differences and hand-derived golden cases).
+``tests/test_oracle_mutants.py`` plants single mistakes in copies of this package and
+checks that those pins catch every one.
 """
 from __future__ import annotations
 
@@ -46,22 +48,26 @@ def build(force: bool = False) -> str:
 def _load():
     global _lib
     if _lib is None:
-        lib = ctypes.CDLL(build())
-        P, I, D = ctypes.c_void_p, ctypes.c_int, ctypes.c_double
-        lib.moda_oracle_forward.argtypes = [P] * 7 + [I] * 8 + [D, I, I]
-        lib.moda_oracle_backward.argtypes = [P] * 13 + [I] * 8 + [D, I, I]
-        lib.moda_oracle_row_weights.argtypes = [P] * 3 + [I] * 9 + [D, I, P, P]
-        lib.moda_oracle_backward_given_out.argtypes = [P] * 12 + [I] * 8 + [D, I, I]
-        lib.moda_oracle_backward_given_out.restype = I
-        lib.moda_oracle_depth_forward.argtypes = [P] * 5 + [I] * 8 + [D, I]
-        lib.moda_oracle_depth_forward.restype = I
-        lib.moda_oracle_depth_backward.argtypes = [P] * 10 + [I] * 8 + [D, I]
-        lib.moda_oracle_depth_backward.restype = I
-        for f in (lib.moda_oracle_forward, lib.moda_oracle_backward,
-                  lib.moda_oracle_row_weights):
-            f.restype = I
-        _lib = lib
+        _lib = _configure(ctypes.CDLL(build()))
     return _lib
+
+
+def _configure(lib):
+    """Declare the argument and return types of the oracle's entry points on ``lib``."""
+    P, I, D = ctypes.c_void_p, ctypes.c_int, ctypes.c_double
+    lib.moda_oracle_forward.argtypes = [P] * 7 + [I] * 8 + [D, I, I]
+    lib.moda_oracle_backward.argtypes = [P] * 13 + [I] * 8 + [D, I, I]
+    lib.moda_oracle_row_weights.argtypes = [P] * 3 + [I] * 9 + [D, I, P, P]
+    lib.moda_oracle_backward_given_out.argtypes = [P] * 12 + [I] * 8 + [D, I, I]
+    lib.moda_oracle_backward_given_out.restype = I
+    lib.moda_oracle_depth_forward.argtypes = [P] * 5 + [I] * 8 + [D, I]
+    lib.moda_oracle_depth_forward.restype = I
+    lib.moda_oracle_depth_backward.argtypes = [P] * 10 + [I] * 8 + [D, I]
+    lib.moda_oracle_depth_backward.restype = I
+    for f in (lib.moda_oracle_forward, lib.moda_oracle_backward,
+              lib.moda_oracle_row_weights):
+        f.restype = I
+    return lib
 
 
 def _f64(x):
