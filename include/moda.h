@@ -22,7 +22,12 @@
  *   kd, vd, dkd, dvd : bf16 [B][Hkv][T][L][d]     (may be NULL when L == 0)
  *   lse              : fp32 [B][Hq][T]
  * Sizes: B, T >= 1; Hq, Hkv >= 1 with Hq % Hkv == 0 and Hq / Hkv <= 64; L >= 0;
- * d in {64, 128}.  scale is applied to every logit (typically 1/sqrt(d)).
+ * d in {64, 128}.  scale is applied to every logit (typically 1/sqrt(d)) and must be
+ * finite.  Violations give MODA_ERR_INVALID_ARGUMENT, except d outside {64, 128}, a
+ * group above the entry point's limit, and problems beyond the kernels' index ranges
+ * (B*Hq*T > 2^31 rows, B*Hkv > 65535, T > 2^30 or L > 65535), which give
+ * MODA_ERR_UNSUPPORTED.  Output buffers must not overlap any input or each other
+ * (MODA_ERR_INVALID_ARGUMENT).
  * causal != 0: sequence key s is visible to token t iff s <= t; causal == 0: every
  * sequence key is visible.  Depth keys are always the query's own token's only.
  *
@@ -109,7 +114,8 @@ moda_status_t moda_depth_attention_forward(const void *q, const void *kd, const 
 /*
  * Depth-only attention backward: dq (bf16), dkd, dvd (bf16) of moda_depth_attention_forward
  * given dout, from its out and lse.  Workspace as for moda_backward (size from
- * moda_backward_workspace_size with the same sizes).  L >= 1.  Two launches: the depth
+ * moda_backward_workspace_size with the same sizes).  L >= 1; Hq/Hkv <= 16 as for
+ * moda_backward (MODA_ERR_UNSUPPORTED beyond).  Two launches: the depth
  * part (row terms, dkd, dvd, fp32 dq) and the dq conversion; dq is deterministic here.
  */
 moda_status_t moda_depth_attention_backward(const void *q, const void *kd, const void *vd,
@@ -149,8 +155,11 @@ moda_status_t moda_decode(const void *q, const void *k, const void *v, const voi
  *   kd, vd: [B, Hkv, T, L, d] bf16; slot l of each receives
  *           kd[b,g,t,l,:] = (x[b,t,:] . w[g*d + c, :])_c,  vd likewise with rows Hkv*d + ...
  *           computed with fp32 accumulation and rounded to bf16; other slots are untouched.
- * Requirements: 0 <= slot < L; d in {64, 128}; Hkv*d a multiple of 128; hidden a multiple
- * of 8 (MODA_ERR_UNSUPPORTED otherwise).  One tcgen05 GEMM launch; no workspace.
+ * Requirements: B, T, hidden, Hkv, L >= 1 and 0 <= slot < L; x, w, kd, vd non-NULL and
+ * 16-byte aligned; kd and vd overlapping neither x, w nor each other
+ * (MODA_ERR_INVALID_ARGUMENT otherwise).  d in {64, 128}, Hkv*d a multiple of 128 and
+ * hidden a multiple of 8 (MODA_ERR_UNSUPPORTED otherwise).  One tcgen05 GEMM launch; no
+ * workspace.
  */
 moda_status_t moda_depth_kv_write(const void *x, const void *w, void *kd, void *vd, int B,
                                   int T, int hidden, int Hkv, int d, int L, int slot,
