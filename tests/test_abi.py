@@ -62,6 +62,12 @@ def fwd(**kw):
     (dict(out=A * 2), moda.MODA_ERR_INVALID_ARGUMENT),  # out aliases k
     (dict(scale=float("nan")), moda.MODA_ERR_INVALID_ARGUMENT),
     (dict(scale=float("inf")), moda.MODA_ERR_INVALID_ARGUMENT),
+    # beyond the kernels' index ranges
+    (dict(B=40000), moda.MODA_ERR_UNSUPPORTED),                 # B*Hkv > 65535
+    (dict(T=(1 << 30) + 16), moda.MODA_ERR_UNSUPPORTED),        # T > 2^30
+    (dict(L=70000), moda.MODA_ERR_UNSUPPORTED),                 # L > 65535
+    (dict(B=600, Hq=64, Hkv=64, T=1 << 16), moda.MODA_ERR_UNSUPPORTED),  # rows > 2^31
+    (dict(lse=A * 64 + 64), moda.MODA_ERR_INVALID_ARGUMENT),    # lse overlaps out
 ])
 def test_forward_rejects_bad_arguments_before_launch(kw, status):
     assert fwd(**kw) == status
@@ -124,6 +130,8 @@ def test_depth_kv_write_rejects_bad_arguments():
     assert st(x=None) == moda.MODA_ERR_INVALID_ARGUMENT
     assert st(kd=A * 64 + 8) == moda.MODA_ERR_INVALID_ARGUMENT
     assert st(vd=A * 64 + 16) == moda.MODA_ERR_INVALID_ARGUMENT  # vd overlaps kd
+    assert st(kd=A) == moda.MODA_ERR_INVALID_ARGUMENT            # kd overlaps x
+    assert st(vd=A * 2) == moda.MODA_ERR_INVALID_ARGUMENT        # vd overlaps w
     assert st(d=96) == moda.MODA_ERR_UNSUPPORTED
     assert st(Hkv=1) == moda.MODA_ERR_UNSUPPORTED      # Hkv*d = 64
     assert st(hidden=60) == moda.MODA_ERR_UNSUPPORTED  # rows not 16-byte multiples
