@@ -721,7 +721,13 @@ def main():
     if args.kvwrite:
         run_kvwrite(args)
         return
-    world, rank, local = dist_setup(args.gpus)
+    if args.impl == "reference":
+        # The reference arm is the oracle on rank 0's host cores: no device work and no
+        # collective, so no process group; the other ranks exit at once.
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank, local = int(os.environ.get("RANK", "0")), 0
+    else:
+        world, rank, local = dist_setup(args.gpus)
     cfg = workloads.CONFIGS[args.workload]
     config = {"workload": args.workload, **{k: cfg[k] for k in ("B", "T", "Hq", "Hkv", "d", "L")},
               "causal": True, "scale": "1/sqrt(d)",
@@ -740,8 +746,6 @@ def main():
                         e2e={"value": round(r["value"], 6), "unit": UNIT,
                              "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0})
             print(json.dumps(line), flush=True)
-        if world > 1:
-            torch.distributed.destroy_process_group()
         return
 
     r = run_moda(args, world, rank, local)

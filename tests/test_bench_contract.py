@@ -46,3 +46,22 @@ def test_l2_statement_follows_the_workload_size():
     assert bench.l2_note(workloads.CONFIGS["fwd-bwd-16k"]) == "inputs larger than L2 (no flush)"
     note = bench.l2_note(workloads.CONFIGS["tiny"])
     assert "fit in L2" in note and "not a headline figure" in note
+
+
+def test_reference_arm_under_two_ranks_prints_on_rank_zero_only():
+    """As under torchrun --nproc-per-node 2: rank 1 exits 0 without work or output,
+    rank 0 prints the line for the whole job (n_gpus = 2)."""
+    base = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus",
+            "2", "--steps", "1", "--warmup", "3", "--cpu-seconds", "1", "--workload", "tiny"]
+    outs = {}
+    for rank in (1, 0):
+        env = dict(os.environ, RANK=str(rank), LOCAL_RANK=str(rank), WORLD_SIZE="2",
+                   MASTER_ADDR="127.0.0.1", MASTER_PORT="29533")
+        r = subprocess.run(base, cwd=ROOT, env=env, capture_output=True, text=True,
+                           timeout=300)
+        assert r.returncode == 0, r.stderr[-2000:]
+        outs[rank] = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert outs[1] == []
+    assert len(outs[0]) == 1
+    line = json.loads(outs[0][0])
+    assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
