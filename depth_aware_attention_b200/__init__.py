@@ -175,6 +175,11 @@ def moda_status_string(status):
     return lib.moda_status_string(status).decode()
 
 
+def moda_last_error_message():
+    """The message the calling thread's last failed call left (empty after a success)."""
+    return lib.moda_last_error_message().decode()
+
+
 # ---------------------------------------------------------------- torch conveniences
 def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
