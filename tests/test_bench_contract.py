@@ -65,3 +65,19 @@ def test_reference_arm_under_two_ranks_prints_on_rank_zero_only():
     assert len(outs[0]) == 1
     line = json.loads(outs[0][0])
     assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
+
+
+def test_clock_summary_reads_nvidia_smi_samples():
+    """The clocks object of the bench line: median SM clock under load, the maximum, and
+    every throttle reason seen active in any sample."""
+    c = bench.ClockSampler(0)
+    c.lines = [
+        "0, 1612, 1965, 950.10, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, 1590, 1965, 990.00, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, 1700, 1965, 700.00, 0x0000000000000000, Not Active, Active, Not Active, Not Active",
+        "[N/A], [N/A]",
+    ]
+    s = c.summary()
+    assert s == {"sm_mhz": 1612.0, "sm_max_mhz": 1965.0, "samples": 3,
+                 "reasons": ["hw_thermal_slowdown", "sw_power_cap"]}
+    assert bench.ClockSampler(0).summary()["reasons"] == ["unsampled"]
