@@ -250,6 +250,9 @@ moda_status_t moda_depth_kv_write(const void* x, const void* w, void* kd, void* 
     return fail(MODA_ERR_UNSUPPORTED, "Hkv * d must be a multiple of 128");
   if (hidden % 8 != 0)
     return fail(MODA_ERR_UNSUPPORTED, "hidden must be a multiple of 8 (16-byte rows)");
+  // the kernel indexes the B*T tokens with 32-bit integers
+  if (1LL * B * T > (1LL << 31) - 256)
+    return fail(MODA_ERR_UNSUPPORTED, "B*T is too large for the kernel's token index");
   if (!x || !w || !kd || !vd)
     return fail(MODA_ERR_INVALID_ARGUMENT, "x, w, kd and vd must be non-NULL");
   if (!aligned16(x) || !aligned16(w) || !aligned16(kd) || !aligned16(vd))

@@ -157,8 +157,8 @@ moda_status_t moda_decode(const void *q, const void *k, const void *v, const voi
  *           computed with fp32 accumulation and rounded to bf16; other slots are untouched.
  * Requirements: B, T, hidden, Hkv, L >= 1 and 0 <= slot < L; x, w, kd, vd non-NULL and
  * 16-byte aligned; kd and vd overlapping neither x, w nor each other
- * (MODA_ERR_INVALID_ARGUMENT otherwise).  d in {64, 128}, Hkv*d a multiple of 128 and
- * hidden a multiple of 8 (MODA_ERR_UNSUPPORTED otherwise).  One tcgen05 GEMM launch; no
+ * (MODA_ERR_INVALID_ARGUMENT otherwise).  d in {64, 128}, Hkv*d a multiple of 128,
+ * hidden a multiple of 8 and B*T < 2^31 - 256 (MODA_ERR_UNSUPPORTED otherwise).  One tcgen05 GEMM launch; no
  * workspace.
  */
 moda_status_t moda_depth_kv_write(const void *x, const void *w, void *kd, void *vd, int B,

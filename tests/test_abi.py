@@ -135,6 +135,7 @@ def test_depth_kv_write_rejects_bad_arguments():
     assert st(d=96) == moda.MODA_ERR_UNSUPPORTED
     assert st(Hkv=1) == moda.MODA_ERR_UNSUPPORTED      # Hkv*d = 64
     assert st(hidden=60) == moda.MODA_ERR_UNSUPPORTED  # rows not 16-byte multiples
+    assert st(B=1 << 16, T=1 << 15) == moda.MODA_ERR_UNSUPPORTED  # B*T = 2^31 tokens
 
 
 def test_forward_L0_allows_null_depth():
