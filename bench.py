@@ -429,7 +429,10 @@ def oracle_sample(cfg, seed_base, cpu_seconds, fwd_only):
     The sample is a window of the LAST nt query tokens (the most expensive rows of the
     causal problem) with all heads; its algorithmic FLOPs are summed row by row with the
     same per-row count as the full problem (4*d*(|visible keys| + L) forward, x2.5 for the
-    backward).  nt grows until the sample takes about cpu_seconds.
+    backward).  nt grows until the sample takes about cpu_seconds.  ``cores`` is the number
+    of threads the oracle actually ran: its forward splits rows over the host's threads, its
+    backward one (batch, KV head) unit per thread.  A second, smaller sample on one thread
+    gives ``value_1_thread``.
     """
     import oracle
     g = torch.Generator().manual_seed(seed_base)
@@ -439,7 +442,7 @@ def oracle_sample(cfg, seed_base, cpu_seconds, fwd_only):
     v = torch.randn((B, Hkv, T, d), generator=g).to(torch.bfloat16)
     threads = oracle.default_threads()
 
-    def sample(nt):
+    def sample(nt, nthreads=threads):
         t0 = T - nt
         q = torch.randn((B, Hq, nt, d), generator=g).to(torch.bfloat16)
         kd = vd = None
@@ -450,10 +453,10 @@ def oracle_sample(cfg, seed_base, cpu_seconds, fwd_only):
         fl = 4.0 * d * rows_keys
         start = time.perf_counter()
         if fwd_only:
-            oracle.forward(q, k, v, kd, vd, scale, True, t0=t0, nthreads=threads)
+            oracle.forward(q, k, v, kd, vd, scale, True, t0=t0, nthreads=nthreads)
         else:
             dout = torch.randn((B, Hq, nt, d), generator=g).to(torch.bfloat16)
-            oracle.backward(q, k, v, kd, vd, dout, scale, True, t0=t0, nthreads=threads)
+            oracle.backward(q, k, v, kd, vd, dout, scale, True, t0=t0, nthreads=nthreads)
             fl *= 1.0 + BWD_FLOP_FACTOR
         return fl, time.perf_counter() - start
 
@@ -465,9 +468,14 @@ def oracle_sample(cfg, seed_base, cpu_seconds, fwd_only):
     if sec < cpu_seconds / 2 and nt < T:
         nt = min(T, max(nt + 1, int(nt * cpu_seconds / max(sec, 1e-3))))
         fl, sec = sample(nt)
+    used = min(threads, B * Hq * nt if fwd_only else B * Hkv)
+    # one thread, on about a quarter of the time budget
+    nt1 = max(1, nt // (4 * used))
+    fl1, sec1 = sample(nt1, 1)
     what = "forward" if fwd_only else "forward+backward"
-    return {"value": round(fl / sec / 1e12, 6), "unit": UNIT, "cores": threads, "kind": "oracle",
-            "seconds": round(sec, 2),
+    return {"value": round(fl / sec / 1e12, 6), "unit": UNIT, "cores": used, "kind": "oracle",
+            "seconds": round(sec, 2), "host_threads": threads,
+            "value_1_thread": round(fl1 / sec1 / 1e12, 6), "sample_1_thread_tokens": nt1,
             "sample": f"fp64 oracle {what} on the last {nt} query tokens (all {B * Hq} "
                       f"heads) of the {cfg['T']}-token workload, L={L}; FLOPs counted "
                       f"row by row as 4*d*(visible keys + L)"
