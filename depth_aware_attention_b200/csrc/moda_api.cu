@@ -41,7 +41,10 @@ moda_status_t check_sizes(int B, int Hq, int Hkv, int T, int L, int d) {
     return fail(MODA_ERR_INVALID_ARGUMENT, "sizes must satisfy B,Hq,Hkv,T >= 1 and L >= 0");
   if (Hq % Hkv != 0) return fail(MODA_ERR_INVALID_ARGUMENT, "Hq must be a multiple of Hkv");
   if (d != 64 && d != 128) return fail(MODA_ERR_UNSUPPORTED, "head size d must be 64 or 128");
-  if (Hq / Hkv > 64) return fail(MODA_ERR_UNSUPPORTED, "query heads per KV head must be <= 64");
+  // Groups above 16 are refused: the parity tests cover G <= 16, and the forward's dense
+  // depth blocks give each row only the keys inside its warp's 32 columns, which holds a
+  // token's G entries only for G <= 32.
+  if (Hq / Hkv > 16) return fail(MODA_ERR_UNSUPPORTED, "query heads per KV head must be <= 16");
   // index arithmetic in the kernels uses 32-bit tile/row counts and 64-bit offsets
   const long long rows = 1LL * B * Hq * T;
   if (rows > (1LL << 31) || 1LL * B * Hkv > 65535 || T > (1 << 30) || L > 65535)

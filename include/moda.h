@@ -21,10 +21,10 @@
  *   k, v, dk, dv     : bf16 [B][Hkv][T][d]
  *   kd, vd, dkd, dvd : bf16 [B][Hkv][T][L][d]     (may be NULL when L == 0)
  *   lse              : fp32 [B][Hq][T]
- * Sizes: B, T >= 1; Hq, Hkv >= 1 with Hq % Hkv == 0 and Hq / Hkv <= 64; L >= 0;
+ * Sizes: B, T >= 1; Hq, Hkv >= 1 with Hq % Hkv == 0 and Hq / Hkv <= 16; L >= 0;
  * d in {64, 128}.  scale is applied to every logit (typically 1/sqrt(d)) and must be
  * finite.  Violations give MODA_ERR_INVALID_ARGUMENT, except d outside {64, 128}, a
- * group above the entry point's limit, and problems beyond the kernels' index ranges
+ * group Hq / Hkv above 16, and problems beyond the kernels' index ranges
  * (B*Hq*T > 2^31 rows, B*Hkv > 65535, T > 2^30 or L > 65535), which give
  * MODA_ERR_UNSUPPORTED.  Output buffers must not overlap any input or each other
  * (MODA_ERR_INVALID_ARGUMENT).

@@ -55,6 +55,7 @@ def fwd(**kw):
     (dict(Hq=3, Hkv=2), moda.MODA_ERR_INVALID_ARGUMENT),
     (dict(d=96), moda.MODA_ERR_UNSUPPORTED),
     (dict(Hq=256, Hkv=2), moda.MODA_ERR_UNSUPPORTED),
+    (dict(Hq=64, Hkv=2), moda.MODA_ERR_UNSUPPORTED),   # G = 32: beyond the tested groups
     (dict(q=None), moda.MODA_ERR_INVALID_ARGUMENT),
     (dict(kd=None), moda.MODA_ERR_INVALID_ARGUMENT),
     (dict(q=A + 8), moda.MODA_ERR_INVALID_ARGUMENT),
