@@ -11,7 +11,10 @@ import depth_aware_attention_b200 as moda
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "moda.h")
 
-A = 1 << 20  # a fake, 16-byte aligned "device pointer" that is never dereferenced
+# A fake, 16-byte aligned "device pointer" that is never dereferenced.  Every call in this
+# file must fail an argument check: on a machine with a GPU, a call whose arguments are all
+# valid would launch a kernel on these addresses.
+A = 1 << 20
 
 
 def declared_functions():
