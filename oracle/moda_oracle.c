@@ -52,8 +52,10 @@
  * sequence keys, S(t) = {}.  The moda_oracle_depth_* entry points run it (causal = -1
  * internally; k, v, dk, dv absent).
  *
- * Parallelism: rows (forward) or (b, kv-head) units (backward) are handed to POSIX
- * threads through an atomic counter; each unit's arithmetic is the plain loop above.
+ * Parallelism: rows (forward) or tokens of one (b, kv-head) group (backward) are handed
+ * to POSIX threads through an atomic counter; each unit's arithmetic is the plain loop
+ * above.  In the backward each thread sums its rows' sequence-key gradients into private
+ * buffers that are added into dk/dv when the group is done.
  */
 #include <math.h>
 #include <pthread.h>
@@ -149,68 +151,129 @@ static void *forward_worker(void *arg) {
     return NULL;
 }
 
-/* Backward for one (b, g) unit: the rows of the G heads of group g whose token lies in
- * the window.  Adds their contributions to dq, dk, dv, dkd, dvd. */
-static void backward_unit(job_t *J, int b, int g, double *scratch, double *o_row) {
+/* Per-thread state of the backward: row scratch and private key-gradient buffers.  The
+ * rows of one (b, g) group are dealt out token by token among the threads; every row
+ * adds to the sequence-key gradients dk/dv of every key it sees, so each thread sums
+ * those contributions into its own [nkeys][d] buffers, and the buffers are added into
+ * dk/dv once every thread has finished the group.  dq rows and the depth gradients of a
+ * token (dkd/dvd, summed over the G heads of the token's group) belong to exactly one
+ * token, so one thread writes them directly. */
+typedef struct {
+    job_t *J;
+    double *scratch, *o_row, *dk_acc, *dv_acc;
+    int b, g, tid, nthreads;
+    int64_t nkeys;
+} bwd_ctx_t;
+
+/* Backward for the G rows (heads of group g) of token t0+w: adds their contributions to
+ * dq (own rows), dkd/dvd (own token) and the thread's dk/dv buffers. */
+static void backward_token(bwd_ctx_t *C, int w) {
+    job_t *J = C->J;
+    const int b = C->b, g = C->g;
     const int d = J->d, T = J->T, L = J->L, G = J->Hq / J->Hkv;
     const int64_t kvoff = ((int64_t)b * J->Hkv + g) * T * d;
     const int has_seq = J->causal >= 0;
     const double *kb = has_seq ? J->k + kvoff : NULL, *vb = has_seq ? J->v + kvoff : NULL;
-    double *dkb = has_seq ? J->dk + kvoff : NULL, *dvb = has_seq ? J->dv + kvoff : NULL;
+    double *dkb = C->dk_acc, *dvb = C->dv_acc;
+    double *scratch = C->scratch, *o_row = C->o_row;
     for (int h = g * G; h < (g + 1) * G; ++h) {
-        for (int w = 0; w < J->nt; ++w) {
-            const int64_t r = qrow(J, b, h, w);
-            const double *qr = J->q + r * d, *dor = J->dout + r * d;
-            double *dqr = J->dq + r * d;
-            const int64_t doff = dtok(J, b, g, w) * L * d;
-            const double *kdt = L ? J->kd + doff : NULL, *vdt = L ? J->vd + doff : NULL;
-            double *dkdt = L ? J->dkd + doff : NULL, *dvdt = L ? J->dvd + doff : NULL;
-            const int ns = n_seq(J->t0 + w, T, J->causal);
-            double lse;
-            forward_row(J, b, h, w, scratch, o_row, &lse);
-            if (J->out) { memcpy(J->out + r * d, o_row, sizeof(double) * d); J->lse[r] = lse; }
-            const double D = dot(dor, J->out_given ? J->out_given + r * d : o_row, d);
-            /* sequence keys: logits are in scratch[0..ns) from forward_row */
-            for (int s = 0; s < ns; ++s) {
-                const double P = exp(scratch[s] - lse);
-                const double dP = dot(dor, vb + (int64_t)s * d, d);
-                const double dS = P * (dP - D);
-                const double *kr = kb + (int64_t)s * d;
-                double *dkr = dkb + (int64_t)s * d, *dvr = dvb + (int64_t)s * d;
-                for (int c = 0; c < d; ++c) {
-                    dqr[c] += J->scale * dS * kr[c];
-                    dkr[c] += J->scale * dS * qr[c];
-                    dvr[c] += P * dor[c];
-                }
+        const int64_t r = qrow(J, b, h, w);
+        const double *qr = J->q + r * d, *dor = J->dout + r * d;
+        double *dqr = J->dq + r * d;
+        const int64_t doff = dtok(J, b, g, w) * L * d;
+        const double *kdt = L ? J->kd + doff : NULL, *vdt = L ? J->vd + doff : NULL;
+        double *dkdt = L ? J->dkd + doff : NULL, *dvdt = L ? J->dvd + doff : NULL;
+        const int ns = n_seq(J->t0 + w, T, J->causal);
+        double lse;
+        forward_row(J, b, h, w, scratch, o_row, &lse);
+        if (J->out) { memcpy(J->out + r * d, o_row, sizeof(double) * d); J->lse[r] = lse; }
+        const double D = dot(dor, J->out_given ? J->out_given + r * d : o_row, d);
+        /* sequence keys: logits are in scratch[0..ns) from forward_row */
+        for (int s = 0; s < ns; ++s) {
+            const double P = exp(scratch[s] - lse);
+            const double dP = dot(dor, vb + (int64_t)s * d, d);
+            const double dS = P * (dP - D);
+            const double *kr = kb + (int64_t)s * d;
+            double *dkr = dkb + (int64_t)s * d, *dvr = dvb + (int64_t)s * d;
+            for (int c = 0; c < d; ++c) {
+                dqr[c] += J->scale * dS * kr[c];
+                dkr[c] += J->scale * dS * qr[c];
+                dvr[c] += P * dor[c];
             }
-            /* depth keys of the row's own token: logits in scratch[ns..ns+L) */
-            for (int j = 0; j < L; ++j) {
-                const double P = exp(scratch[ns + j] - lse);
-                const double dP = dot(dor, vdt + (int64_t)j * d, d);
-                const double dS = P * (dP - D);
-                const double *kr = kdt + (int64_t)j * d;
-                double *dkr = dkdt + (int64_t)j * d, *dvr = dvdt + (int64_t)j * d;
-                for (int c = 0; c < d; ++c) {
-                    dqr[c] += J->scale * dS * kr[c];
-                    dkr[c] += J->scale * dS * qr[c];
-                    dvr[c] += P * dor[c];
-                }
+        }
+        /* depth keys of the row's own token: logits in scratch[ns..ns+L) */
+        for (int j = 0; j < L; ++j) {
+            const double P = exp(scratch[ns + j] - lse);
+            const double dP = dot(dor, vdt + (int64_t)j * d, d);
+            const double dS = P * (dP - D);
+            const double *kr = kdt + (int64_t)j * d;
+            double *dkr = dkdt + (int64_t)j * d, *dvr = dvdt + (int64_t)j * d;
+            for (int c = 0; c < d; ++c) {
+                dqr[c] += J->scale * dS * kr[c];
+                dkr[c] += J->scale * dS * qr[c];
+                dvr[c] += P * dor[c];
             }
         }
     }
 }
 
+/* Thread `tid` of `nthreads` takes the window's tokens tid, tid + nthreads, ... (a fixed
+ * interleaving: causal rows grow in cost with t, so every thread gets a similar mix). */
 static void *backward_worker(void *arg) {
-    job_t *J = (job_t *)arg;
-    double *scratch = (double *)malloc(sizeof(double) * ((size_t)J->T + (size_t)J->L + 1));
-    double *o_row = (double *)malloc(sizeof(double) * (size_t)J->d);
-    for (int64_t u; (u = take(J)) < J->nunits;)
-        backward_unit(J, (int)(u / J->Hkv), (int)(u % J->Hkv), scratch, o_row);
-    free(o_row);
-    free(scratch);
+    bwd_ctx_t *C = (bwd_ctx_t *)arg;
+    for (int w = C->tid; w < C->J->nt; w += C->nthreads) backward_token(C, w);
     return NULL;
 }
 
+/* The whole backward: one (b, g) group after another, each group's window tokens shared
+ * out among the threads, then the threads' key-gradient buffers summed into dk/dv. */
+static void run_backward(job_t *J, int nthreads) {
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 256) nthreads = 256;
+    if (nthreads > J->nt) nthreads = J->nt;
+    const int has_seq = J->causal >= 0;
+    /* keys that window rows can see: [0, t0+nt) when causal, all T otherwise */
+    const int64_t nkeys = !has_seq ? 0 : (J->causal ? J->t0 + J->nt : J->T);
+    const size_t kbytes = sizeof(double) * (size_t)nkeys * (size_t)J->d;
+    pthread_t th[256];
+    bwd_ctx_t C[256];
+    for (int i = 0; i < nthreads; ++i) {
+        C[i].J = J;
+        C[i].scratch = (double *)malloc(sizeof(double) * ((size_t)J->T + (size_t)J->L + 1));
+        C[i].o_row = (double *)malloc(sizeof(double) * (size_t)J->d);
+        C[i].dk_acc = nkeys ? (double *)malloc(kbytes) : NULL;
+        C[i].dv_acc = nkeys ? (double *)malloc(kbytes) : NULL;
+        C[i].nkeys = nkeys;
+        C[i].tid = i;
+        C[i].nthreads = nthreads;
+    }
+    for (int b = 0; b < J->B; ++b) {
+        for (int g = 0; g < J->Hkv; ++g) {
+            for (int i = 0; i < nthreads; ++i) {
+                C[i].b = b;
+                C[i].g = g;
+                if (nkeys) { memset(C[i].dk_acc, 0, kbytes); memset(C[i].dv_acc, 0, kbytes); }
+            }
+            for (int i = 1; i < nthreads; ++i) pthread_create(&th[i], NULL, backward_worker, &C[i]);
+            backward_worker(&C[0]);
+            for (int i = 1; i < nthreads; ++i) pthread_join(th[i], NULL);
+            if (nkeys) {
+                const int64_t kvoff = ((int64_t)b * J->Hkv + g) * J->T * J->d;
+                const int64_t n = nkeys * J->d;
+                for (int i = 0; i < nthreads; ++i)
+                    for (int64_t e = 0; e < n; ++e) {
+                        J->dk[kvoff + e] += C[i].dk_acc[e];
+                        J->dv[kvoff + e] += C[i].dv_acc[e];
+                    }
+            }
+        }
+    }
+    for (int i = 0; i < nthreads; ++i) {
+        free(C[i].scratch); free(C[i].o_row); free(C[i].dk_acc); free(C[i].dv_acc);
+    }
+}
+
+/* Forward threading: rows handed out through the job's atomic counter. */
 static void run(job_t *J, void *(*fn)(void *), int nthreads) {
     if (nthreads < 1) nthreads = 1;
     if (nthreads > 256) nthreads = 256;
@@ -281,8 +344,7 @@ int moda_oracle_backward(const double *q, const double *k, const double *v,
     J.dq = dq; J.dk = dk; J.dv = dv; J.dkd = dkd; J.dvd = dvd; J.out = out; J.lse = lse;
     J.B = B; J.Hq = Hq; J.Hkv = Hkv; J.T = T; J.L = L; J.d = d; J.causal = causal;
     J.t0 = t0; J.nt = nt; J.scale = scale;
-    J.nunits = (int64_t)B * Hkv;
-    run(&J, backward_worker, nthreads);
+    run_backward(&J, nthreads);
     return 0;
 }
 
@@ -304,8 +366,7 @@ int moda_oracle_backward_given_out(const double *q, const double *k, const doubl
     J.dq = dq; J.dk = dk; J.dv = dv; J.dkd = dkd; J.dvd = dvd;
     J.B = B; J.Hq = Hq; J.Hkv = Hkv; J.T = T; J.L = L; J.d = d; J.causal = causal;
     J.t0 = t0; J.nt = nt; J.scale = scale;
-    J.nunits = (int64_t)B * Hkv;
-    run(&J, backward_worker, nthreads);
+    run_backward(&J, nthreads);
     return 0;
 }
 
@@ -372,7 +433,6 @@ int moda_oracle_depth_backward(const double *q, const double *kd, const double *
     J.dq = dq; J.dkd = dkd; J.dvd = dvd; J.out = out; J.lse = lse;
     J.B = B; J.Hq = Hq; J.Hkv = Hkv; J.T = T; J.L = L; J.d = d; J.causal = -1;
     J.t0 = t0; J.nt = nt; J.scale = scale;
-    J.nunits = (int64_t)B * Hkv;
-    run(&J, backward_worker, nthreads);
+    run_backward(&J, nthreads);
     return 0;
 }

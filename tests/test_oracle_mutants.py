@@ -43,36 +43,39 @@ MUTANTS = [
      "*lse_row = m + log(Z);", "*lse_row = log(Z);"),
     ("depth dS with the wrong sign", C,
      "const double dP = dot(dor, vdt + (int64_t)j * d, d);\n"
-     "                const double dS = P * (dP - D);",
+     "            const double dS = P * (dP - D);",
      "const double dP = dot(dor, vdt + (int64_t)j * d, d);\n"
-     "                const double dS = P * (D - dP);"),
+     "            const double dS = P * (D - dP);"),
     ("sequence dk without the scale", C,
      "double *dkr = dkb + (int64_t)s * d, *dvr = dvb + (int64_t)s * d;\n"
-     "                for (int c = 0; c < d; ++c) {\n"
-     "                    dqr[c] += J->scale * dS * kr[c];\n"
-     "                    dkr[c] += J->scale * dS * qr[c];",
+     "            for (int c = 0; c < d; ++c) {\n"
+     "                dqr[c] += J->scale * dS * kr[c];\n"
+     "                dkr[c] += J->scale * dS * qr[c];",
      "double *dkr = dkb + (int64_t)s * d, *dvr = dvb + (int64_t)s * d;\n"
-     "                for (int c = 0; c < d; ++c) {\n"
-     "                    dqr[c] += J->scale * dS * kr[c];\n"
-     "                    dkr[c] += dS * qr[c];"),
+     "            for (int c = 0; c < d; ++c) {\n"
+     "                dqr[c] += J->scale * dS * kr[c];\n"
+     "                dkr[c] += dS * qr[c];"),
     ("dvd from q instead of dO", C,
      "*dvr = dvdt + (int64_t)j * d;\n"
-     "                for (int c = 0; c < d; ++c) {\n"
-     "                    dqr[c] += J->scale * dS * kr[c];\n"
-     "                    dkr[c] += J->scale * dS * qr[c];\n"
-     "                    dvr[c] += P * dor[c];",
+     "            for (int c = 0; c < d; ++c) {\n"
+     "                dqr[c] += J->scale * dS * kr[c];\n"
+     "                dkr[c] += J->scale * dS * qr[c];\n"
+     "                dvr[c] += P * dor[c];",
      "*dvr = dvdt + (int64_t)j * d;\n"
-     "                for (int c = 0; c < d; ++c) {\n"
-     "                    dqr[c] += J->scale * dS * kr[c];\n"
-     "                    dkr[c] += J->scale * dS * qr[c];\n"
-     "                    dvr[c] += P * qr[c];"),
+     "            for (int c = 0; c < d; ++c) {\n"
+     "                dqr[c] += J->scale * dS * kr[c];\n"
+     "                dkr[c] += J->scale * dS * qr[c];\n"
+     "                dvr[c] += P * qr[c];"),
     ("dq misses the depth keys", C,
      "*dvr = dvdt + (int64_t)j * d;\n"
-     "                for (int c = 0; c < d; ++c) {\n"
-     "                    dqr[c] += J->scale * dS * kr[c];",
+     "            for (int c = 0; c < d; ++c) {\n"
+     "                dqr[c] += J->scale * dS * kr[c];",
      "*dvr = dvdt + (int64_t)j * d;\n"
-     "                for (int c = 0; c < d; ++c) {\n"
-     "                    (void)kr;"),
+     "            for (int c = 0; c < d; ++c) {\n"
+     "            (void)kr;"),
+    ("only one thread's key-gradient buffer summed", C,
+     "for (int i = 0; i < nthreads; ++i)\n                    for (int64_t e = 0; e < n; ++e) {",
+     "for (int i = 0; i < 1; ++i)\n                    for (int64_t e = 0; e < n; ++e) {"),
     ("row term D dropped", C,
      "const double D = dot(dor, J->out_given ? J->out_given + r * d : o_row, d);",
      "const double D = 0.0 * dot(dor, J->out_given ? J->out_given + r * d : o_row, d);"),
