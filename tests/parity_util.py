@@ -18,6 +18,9 @@ for it the mean-abs bound too is applied beyond the output rounding
 """
 from __future__ import annotations
 
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -65,30 +68,75 @@ def oracle_forward_window(x, t0, nt, scale, causal):
     return oracle.forward(w["q"], w["k"], w["v"], w["kd"], w["vd"], scale, causal, t0=t0)
 
 
+def log_stats(what, **fields):
+    """Appends one JSON line of measured errors to the file named by MODA_PARITY_STATS
+    (when set), so that a run can record every case's figures, passing or not."""
+    path = os.environ.get("MODA_PARITY_STATS")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps(dict(case=what, **fields)) + "\n")
+
+
+def error_stats(err, ref):
+    """max-abs, plain mean-abs, max beyond rounding and mean beyond rounding."""
+    ex = excess(err, ref)
+    return dict(max_abs=float(err.max()), mean_abs=float(err.mean()),
+                max_beyond_rounding=float(ex.max()),
+                mean_beyond_rounding=float(np.maximum(ex, 0.0).mean()))
+
+
 def compare_forward(out, lse, ref_out, ref_lse, what="", mean_beyond_rounding=False):
     o = out.detach().to("cpu", torch.float64).numpy()
     ls = lse.detach().to("cpu", torch.float64).numpy()
     err = np.abs(o - ref_out)
     lerr = np.abs(ls - ref_lse)
+    st = error_stats(err, ref_out)
+    log_stats(what, kind="out", rows=int(np.prod(ref_lse.shape)), lse_max_abs=float(lerr.max()),
+              **st)
     assert np.isfinite(o).all(), f"{what}: non-finite output"
-    ex = excess(err, ref_out)
-    assert ex.max() <= OUT_MAX, f"{what}: out max-abs {err.max():.3e} (beyond rounding {ex.max():.3e})"
-    mean = np.maximum(ex, 0.0).mean() if mean_beyond_rounding else err.mean()
-    assert mean <= OUT_MEAN, f"{what}: out mean-abs {mean:.3e}"
+    assert st["max_beyond_rounding"] <= OUT_MAX, (
+        f"{what}: out max-abs {st['max_abs']:.3e} (beyond rounding "
+        f"{st['max_beyond_rounding']:.3e})")
+    mean = st["mean_beyond_rounding"] if mean_beyond_rounding else st["mean_abs"]
+    assert mean <= OUT_MEAN, f"{what}: out mean-abs {mean:.3e} (plain {st['mean_abs']:.3e})"
     assert lerr.max() <= LSE_MAX, f"{what}: lse max-abs {lerr.max():.3e}"
-    return float(err.max()), float(err.mean()), float(lerr.max())
+    return st["max_abs"], st["mean_abs"], float(lerr.max())
 
 
 def compare_grad(g, ref, what, max_tol=OUT_MAX, mean_tol=OUT_MEAN, mean_beyond_rounding=False):
     a = g.detach().to("cpu", torch.float64).numpy()
     err = np.abs(a - ref)
-    assert np.isfinite(a).all(), f"{what}: non-finite"
-    ex = excess(err, ref)
-    assert ex.max() <= max_tol, f"{what}: max-abs {err.max():.3e} (beyond rounding {ex.max():.3e})"
-    mean = np.maximum(ex, 0.0).mean() if mean_beyond_rounding else err.mean()
-    assert mean <= mean_tol, f"{what}: mean-abs {mean:.3e}"
+    st = error_stats(err, ref)
     rms = float(np.sqrt((ref ** 2).mean()))
-    if rms > 0:
-        rel = float(np.sqrt((err ** 2).mean())) / rms
-        assert rel <= GRAD_REL_RMS, f"{what}: relative RMS error {rel:.3e}"
-    return float(err.max()), float(err.mean())
+    rel = float(np.sqrt((err ** 2).mean())) / rms if rms > 0 else 0.0
+    log_stats(what, kind="grad", elements=int(ref.size), rel_rms=rel, **st)
+    assert np.isfinite(a).all(), f"{what}: non-finite"
+    assert st["max_beyond_rounding"] <= max_tol, (
+        f"{what}: max-abs {st['max_abs']:.3e} (beyond rounding "
+        f"{st['max_beyond_rounding']:.3e})")
+    mean = st["mean_beyond_rounding"] if mean_beyond_rounding else st["mean_abs"]
+    assert mean <= mean_tol, f"{what}: mean-abs {mean:.3e} (plain {st['mean_abs']:.3e})"
+    assert rel <= GRAD_REL_RMS, f"{what}: relative RMS error {rel:.3e}"
+    return st["max_abs"], st["mean_abs"]
+
+
+def window_starts(T, nt, n_random, seed):
+    """Starts of token windows of nt tokens: the first (t = 0), the last (t = T-1) and
+    n_random more drawn uniformly from a seeded generator."""
+    rng = np.random.RandomState(seed)
+    starts = [0, T - nt] + [int(s) for s in rng.randint(0, T - nt + 1, size=n_random)]
+    return sorted(set(starts))
+
+
+def oracle_forward_windows(x, starts, nt, scale, causal):
+    """Oracle forward on several token windows of one problem.  k and v are widened to
+    fp64 once and shared by every window.  Yields (t0, ref_out, ref_lse)."""
+    k = x["k"].cpu().to(torch.float64).numpy()
+    v = x["v"].cpu().to(torch.float64).numpy()
+    for t0 in starts:
+        sl = slice(t0, t0 + nt)
+        kd = None if x.get("kd") is None else x["kd"][:, :, sl].cpu()
+        vd = None if x.get("vd") is None else x["vd"][:, :, sl].cpu()
+        ref_out, ref_lse = oracle.forward(x["q"][:, :, sl].cpu(), k, v, kd, vd, scale,
+                                          causal, t0=t0)
+        yield t0, ref_out, ref_lse

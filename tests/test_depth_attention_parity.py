@@ -4,7 +4,10 @@ through the C ABI) vs the fp64 oracle's depth-only mode, element by element.
 Small problems are compared in full over group sizes that do and do not divide 128 (the
 dense tensor-core depth path and the CUDA-core fold path), both head sizes, ragged token
 counts, L = 1 and long depth caches.  The deep-stack head layout at 4K tokens is compared
-on token windows (depth-only rows are independent per token, so a window is exact).
+on token windows (depth-only rows are independent per token, so a window is exact).  The
+gradients are compared with the oracle's exact gradient of the definition.  The mean-abs
+bound is applied beyond each element's bf16 rounding (the outputs average only L values,
+so they are O(1)); the plain mean-abs of every case is logged beside it.
 """
 import math
 
@@ -14,7 +17,7 @@ import torch
 import depth_aware_attention_b200 as moda
 import workloads
 import oracle
-from parity_util import compare_forward, compare_grad, gpu_inputs
+from parity_util import compare_forward, compare_grad, gpu_inputs, window_starts
 
 pytestmark = pytest.mark.gpu
 
@@ -43,12 +46,11 @@ def test_depth_attention_small_full(name, cfg):
     moda.check_device_errors()
     w = _sel(x, 0, cfg["T"])
     ref_out, ref_lse = oracle.depth_forward(w["q"], w["kd"], w["vd"], scale)
-    compare_forward(out, lse, ref_out, ref_lse, name, mean_beyond_rounding=True)
-    # the backward receives the forward's bf16 out: compare with the exact gradient given
-    # that out (the row terms D = <dO, out> can only be formed from it)
-    ref = oracle.depth_backward(w["q"], w["kd"], w["vd"], w["dout"], scale, out=out.cpu())
+    compare_forward(out, lse, ref_out, ref_lse, f"fda {name}", mean_beyond_rounding=True)
+    # the exact gradient of the definition (the oracle's own out and row terms)
+    ref = oracle.depth_backward(w["q"], w["kd"], w["vd"], w["dout"], scale)
     for n in ("dq", "dkd", "dvd"):
-        compare_grad(g[n], ref[n], f"{name}:{n}", mean_beyond_rounding=True)
+        compare_grad(g[n], ref[n], f"fda {name}:{n}", mean_beyond_rounding=True)
 
 
 def test_depth_attention_is_deterministic():
@@ -71,15 +73,14 @@ def test_depth_attention_deep_windows():
     out, lse = moda.depth_attention_forward(x["q"], x["kd"], x["vd"], scale)
     g = moda.depth_attention_backward(x["q"], x["kd"], x["vd"], out, lse, x["dout"], scale)
     moda.check_device_errors()
-    T, nt = cfg["T"], 24
-    for t0 in (0, T // 2 - 3, T - nt):
+    T, nt = cfg["T"], 16
+    for t0 in window_starts(T, nt, 6, seed=workloads.SEED_BASE["deep-4k"]):
         w = _sel(x, t0, nt)
         sl = slice(t0, t0 + nt)
         ref_out, ref_lse = oracle.depth_forward(w["q"], w["kd"], w["vd"], scale, t0=t0)
         compare_forward(out[:, :, sl], lse[:, :, sl], ref_out, ref_lse, f"deep-4k fda @{t0}",
                         mean_beyond_rounding=True)
-        ref = oracle.depth_backward(w["q"], w["kd"], w["vd"], w["dout"], scale,
-                                    out=out[:, :, sl].cpu(), t0=t0)
+        ref = oracle.depth_backward(w["q"], w["kd"], w["vd"], w["dout"], scale, t0=t0)
         compare_grad(g["dq"][:, :, sl], ref["dq"], f"deep-4k fda dq @{t0}",
                      mean_beyond_rounding=True)
         compare_grad(g["dkd"][:, :, sl], ref["dkd"], f"deep-4k fda dkd @{t0}",

@@ -13,7 +13,8 @@ import torch
 
 import depth_aware_attention_b200 as moda
 import workloads
-from parity_util import compare_forward, gpu_inputs, oracle_forward_window
+from parity_util import (compare_forward, gpu_inputs, oracle_forward_window,
+                         oracle_forward_windows, window_starts)
 import oracle
 
 pytestmark = pytest.mark.gpu
@@ -68,7 +69,8 @@ def test_forward_small_full_each_depth_path(name, cfg, causal, path):
 @pytest.mark.parametrize("path", [1, 2], ids=["fold", "dense"])
 def test_forward_deep_windows_each_depth_path(path):
     """The deep-stack head layout (L = 128) at 4K tokens through each depth path, on
-    token windows at the start, middle and end; the dense path is also deterministic."""
+    16-token windows at the start, the end and seeded random positions (every head: at
+    least 4096 rows); each path is also deterministic."""
     cfg = workloads.CONFIGS["deep-4k"]
     x = gpu_inputs(cfg, workloads.SEED_BASE["deep-4k"])
     scale = workloads.default_scale(cfg["d"])
@@ -78,9 +80,9 @@ def test_forward_deep_windows_each_depth_path(path):
                               depth_path=path)
     moda.check_device_errors()
     assert torch.equal(out, out2) and torch.equal(lse, lse2)
-    T, nt = cfg["T"], 48
-    for t0 in (0, T // 2 - 5, T - nt):
-        ref_out, ref_lse = oracle_forward_window(x, t0, nt, scale, True)
+    T, nt = cfg["T"], 16
+    starts = window_starts(T, nt, 6, seed=workloads.SEED_BASE["deep-4k"])
+    for t0, ref_out, ref_lse in oracle_forward_windows(x, starts, nt, scale, True):
         sl = slice(t0, t0 + nt)
         compare_forward(out[:, :, sl], lse[:, :, sl], ref_out, ref_lse,
                         f"deep-4k path {path} @{t0}")
@@ -134,17 +136,26 @@ def test_L0_matches_torch_causal_attention():
 BIG = ["layer-4k", "long-64k", "long-64k-L0", "deep-stack", "fwd-bwd-16k"]
 
 
+SAMPLE_ROWS = 4096
+
+
 @pytest.mark.parametrize("name", BIG)
 def test_forward_benchmark_workloads_windows(name):
+    """A stratified sample of at least 4096 rows of each benchmark workload, in the launch
+    configuration the benchmark times: every head of every batch entry on 8-token windows
+    at t = 0, at t = T-1 and at seeded random positions.  Rows are independent, so each
+    sampled row is compared with its exact oracle value."""
     cfg = workloads.CONFIGS[name]
     x = gpu_inputs(cfg, workloads.SEED_BASE[name])
     scale = workloads.default_scale(cfg["d"])
     out, lse = moda.forward(x["q"], x["k"], x["v"], x["kd"], x["vd"], scale, True)
     moda.check_device_errors()
-    T = cfg["T"]
-    nt = 32 if T >= 16384 else 64
-    for t0 in (0, T // 2 - 17, T - nt):
-        ref_out, ref_lse = oracle_forward_window(x, t0, nt, scale, True)
+    T, nt = cfg["T"], 8
+    per_window = cfg["B"] * cfg["Hq"] * nt
+    n_windows = max(8, -(-SAMPLE_ROWS // per_window))
+    starts = window_starts(T, nt, n_windows - 2, seed=workloads.SEED_BASE[name])
+    assert len(starts) * per_window >= SAMPLE_ROWS and starts[0] == 0 and starts[-1] == T - nt
+    for t0, ref_out, ref_lse in oracle_forward_windows(x, starts, nt, scale, True):
         sl = slice(t0, t0 + nt)
         compare_forward(out[:, :, sl], lse[:, :, sl], ref_out, ref_lse, f"{name}@{t0}")
     del x, out, lse
