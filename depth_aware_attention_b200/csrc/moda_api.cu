@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <mutex>
@@ -74,6 +75,36 @@ moda_status_t check_device() {
   return MODA_OK;
 }
 
+// Host-side fault injection, for testing how callers handle the library's errors; no
+// kernel is launched in either mode.  The environment variable MODA_FAULT_INJECT is read
+// on every call (so a test can set and clear it in-process):
+//   validate  every compute entry point returns MODA_ERR_INVALID_ARGUMENT before its
+//             argument checks;
+//   launch    it returns MODA_ERR_CUDA once its argument checks have passed, in place of
+//             the device query and the launch.
+// Any other value, or none, injects nothing.
+enum { kInjectNone = 0, kInjectValidate = 1, kInjectLaunch = 2 };
+
+int fault_injection() {
+  const char* e = getenv("MODA_FAULT_INJECT");
+  if (e == nullptr) return kInjectNone;
+  if (strcmp(e, "validate") == 0) return kInjectValidate;
+  if (strcmp(e, "launch") == 0) return kInjectLaunch;
+  return kInjectNone;
+}
+
+moda_status_t injected_at_validate() {
+  if (fault_injection() == kInjectValidate)
+    return fail(MODA_ERR_INVALID_ARGUMENT, "injected failure (MODA_FAULT_INJECT=validate)");
+  return MODA_OK;
+}
+
+moda_status_t injected_at_launch() {
+  if (fault_injection() == kInjectLaunch)
+    return fail(MODA_ERR_CUDA, "injected failure (MODA_FAULT_INJECT=launch)");
+  return MODA_OK;
+}
+
 moda::EncodeTiledFn get_encoder() {
   static std::once_flag once;
   static moda::EncodeTiledFn fn = nullptr;
@@ -112,7 +143,9 @@ static moda_status_t forward_entry(const void* q, const void* k, const void* v,
                                    int causal, int depth_path, int depth_only,
                                    moda_stream_t stream) {
   g_msg[0] = 0;
-  moda_status_t s = check_sizes(B, Hq, Hkv, T, L, d);
+  moda_status_t s = injected_at_validate();
+  if (s != MODA_OK) return s;
+  s = check_sizes(B, Hq, Hkv, T, L, d);
   if (s != MODA_OK) return s;
   if (depth_only) {
     if (L < 1) return fail(MODA_ERR_INVALID_ARGUMENT, "depth-only attention needs L >= 1");
@@ -143,6 +176,8 @@ static moda_status_t forward_entry(const void* q, const void* k, const void* v,
   p.depth_only = depth_only ? 1 : 0;
   if (depth_path == moda::kDepthPathDense && !moda::dense_depth_supported(p))
     return fail(MODA_ERR_UNSUPPORTED, "dense depth blocks need Hq/Hkv to divide 128");
+  s = injected_at_launch();
+  if (s != MODA_OK) return s;
   s = check_device();
   if (s != MODA_OK) return s;
   moda::EncodeTiledFn enc = get_encoder();
@@ -193,7 +228,9 @@ moda_status_t moda_decode(const void* q, const void* k, const void* v, const voi
                           size_t workspace_bytes, int B, int Hq, int Hkv, int S, int L, int d,
                           float scale, moda_stream_t stream) {
   g_msg[0] = 0;
-  moda_status_t s = check_sizes(B, Hq, Hkv, S, L, d);
+  moda_status_t s = injected_at_validate();
+  if (s != MODA_OK) return s;
+  s = check_sizes(B, Hq, Hkv, S, L, d);
   if (s != MODA_OK) return s;
   if (Hq / Hkv > 16)
     return fail(MODA_ERR_UNSUPPORTED, "decode supports at most 16 query heads per KV head");
@@ -227,6 +264,8 @@ moda_status_t moda_decode(const void* q, const void* k, const void* v, const voi
       if (overlaps(outs[o], outsz[o], outs[o2], outsz[o2]))
         return fail(MODA_ERR_INVALID_ARGUMENT, "out, lse and workspace must not overlap");
   }
+  s = injected_at_launch();
+  if (s != MODA_OK) return s;
   s = check_device();
   if (s != MODA_OK) return s;
   moda::EncodeTiledFn enc = get_encoder();
@@ -245,6 +284,7 @@ moda_status_t moda_depth_kv_write(const void* x, const void* w, void* kd, void* 
                                   int T, int hidden, int Hkv, int d, int L, int slot,
                                   moda_stream_t stream) {
   g_msg[0] = 0;
+  if (injected_at_validate() != MODA_OK) return MODA_ERR_INVALID_ARGUMENT;
   if (B < 1 || T < 1 || hidden < 1 || Hkv < 1 || L < 1)
     return fail(MODA_ERR_INVALID_ARGUMENT, "B, T, hidden, Hkv and L must be positive");
   if (slot < 0 || slot >= L) return fail(MODA_ERR_INVALID_ARGUMENT, "slot must lie in [0, L)");
@@ -265,7 +305,9 @@ moda_status_t moda_depth_kv_write(const void* x, const void* w, void* kd, void* 
   if (overlaps(kd, nd, x, nx) || overlaps(kd, nd, w, nw) || overlaps(vd, nd, x, nx) ||
       overlaps(vd, nd, w, nw) || overlaps(kd, nd, vd, nd))
     return fail(MODA_ERR_INVALID_ARGUMENT, "kd/vd must not overlap x, w or each other");
-  moda_status_t s = check_device();
+  moda_status_t s = injected_at_launch();
+  if (s != MODA_OK) return s;
+  s = check_device();
   if (s != MODA_OK) return s;
   moda::EncodeTiledFn enc = get_encoder();
   if (!enc) return fail(MODA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
@@ -290,14 +332,19 @@ size_t moda_backward_workspace_size(int B, int Hq, int Hkv, int T, int L, int d)
 
 namespace {
 
+// validate_only: run the argument checks that need neither the workspace nor the device
+// and return (no device query, no launch); the workspace may then be NULL.
 moda_status_t backward_entry(const void* q, const void* k, const void* v, const void* kd,
                              const void* vd, const void* out, const float* lse,
                              const void* dout, void* dq, void* dk, void* dv, void* dkd,
                              void* dvd, void* workspace, size_t workspace_bytes, int B,
                              int Hq, int Hkv, int T, int L, int d, float scale, int causal,
-                             unsigned stages, int depth_only, moda_stream_t stream) {
+                             unsigned stages, int depth_only, moda_stream_t stream,
+                             bool validate_only = false) {
   g_msg[0] = 0;
-  moda_status_t s = check_sizes(B, Hq, Hkv, T, L, d);
+  moda_status_t s = injected_at_validate();
+  if (s != MODA_OK) return s;
+  s = check_sizes(B, Hq, Hkv, T, L, d);
   if (s != MODA_OK) return s;
   if (depth_only) {
     if (L < 1) return fail(MODA_ERR_INVALID_ARGUMENT, "depth-only attention needs L >= 1");
@@ -305,7 +352,8 @@ moda_status_t backward_entry(const void* q, const void* k, const void* v, const 
     dk = dv = nullptr;
     stages = moda::kStageDepth | moda::kStageConvert;
   }
-  if (!q || !out || !lse || !dout || !dq || !workspace || (!depth_only && (!k || !v || !dk || !dv)))
+  if (!q || !out || !lse || !dout || !dq || (!workspace && !validate_only) ||
+      (!depth_only && (!k || !v || !dk || !dv)))
     return fail(MODA_ERR_INVALID_ARGUMENT,
                 "q, k, v, out, lse, dout, dq, dk, dv and workspace must be non-NULL");
   if (L > 0 && (!kd || !vd || !dkd || !dvd))
@@ -322,6 +370,24 @@ moda_status_t backward_entry(const void* q, const void* k, const void* v, const 
     return fail(MODA_ERR_UNSUPPORTED, "the backward supports at most 16 query heads per KV head");
   moda::Problem p{B, Hq, Hkv, T, L, d, Hq / Hkv, causal ? 1 : 0, scale};
   p.depth_only = depth_only ? 1 : 0;
+  if (validate_only) {
+    // the checks of the gradient buffers against the inputs and each other
+    const size_t nq = size_t(B) * Hq * T * d * 2, nk = size_t(B) * Hkv * T * d * 2;
+    const size_t nd = nk * size_t(L), nl = size_t(B) * Hq * T * 4;
+    const void* ins[8] = {q, k, v, kd, vd, out, lse, dout};
+    const size_t insz[8] = {nq, nk, nk, nd, nd, nq, nl, nq};
+    void* outs[5] = {dq, dk, dv, dkd, dvd};
+    const size_t outsz[5] = {nq, nk, nk, nd, nd};
+    for (int o = 0; o < 5; ++o) {
+      for (int i = 0; i < 8; ++i)
+        if (overlaps(outs[o], outsz[o], ins[i], insz[i]))
+          return fail(MODA_ERR_INVALID_ARGUMENT, "gradient buffers must not overlap an input");
+      for (int o2 = o + 1; o2 < 5; ++o2)
+        if (overlaps(outs[o], outsz[o], outs[o2], outsz[o2]))
+          return fail(MODA_ERR_INVALID_ARGUMENT, "gradient buffers must not overlap each other");
+    }
+    return MODA_OK;
+  }
   const size_t need = moda::backward_workspace_bytes(p);
   if (workspace_bytes < need)
     return fail(MODA_ERR_INVALID_ARGUMENT, "workspace is smaller than moda_backward_workspace_size()");
@@ -339,6 +405,8 @@ moda_status_t backward_entry(const void* q, const void* k, const void* v, const 
       if (overlaps(outs[o], outsz[o], outs[o2], outsz[o2]))
         return fail(MODA_ERR_INVALID_ARGUMENT, "gradient/workspace buffers must not overlap each other");
   }
+  s = injected_at_launch();
+  if (s != MODA_OK) return s;
   s = check_device();
   if (s != MODA_OK) return s;
   moda::EncodeTiledFn enc = get_encoder();

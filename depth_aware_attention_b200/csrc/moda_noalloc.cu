@@ -32,7 +32,9 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 namespace {
 
 // Device address of g_noalloc_scratch on the calling thread's current device, looked up
-// on the first call for that device and cached.  NULL (with *err set) on failure.
+// on the first call for that device and cached for the life of the process.  The cache
+// is not invalidated: a cudaDeviceReset() (which unloads the module, so the array may come
+// back elsewhere) between calls is not supported.  NULL (with *err set) on failure.
 void* noalloc_scratch(int dev, cudaError_t* err) {
   static std::mutex mu;
   static void* addr[64] = {nullptr};
@@ -57,7 +59,12 @@ extern "C" moda_status_t moda_backward_noalloc(
     const void* out, const float* lse, const void* dout, void* dq, void* dk, void* dv,
     void* dkd, void* dvd, int B, int Hq, int Hkv, int T, int L, int d, float scale,
     int causal, moda_stream_t stream) {
-  // Invalid sizes report 0 here; moda_backward then returns the precise error for them.
+  // Every argument check that needs neither the workspace nor the device runs first, so
+  // a bad call is refused before anything touches the GPU.
+  moda_status_t s = backward_entry(q, k, v, kd, vd, out, lse, dout, dq, dk, dv, dkd, dvd,
+                                   nullptr, 0, B, Hq, Hkv, T, L, d, scale, causal,
+                                   moda::kStagesAll, 0, stream, /*validate_only=*/true);
+  if (s != MODA_OK) return s;
   const size_t need = moda_backward_workspace_size(B, Hq, Hkv, T, L, d);
   if (need > moda::kNoAllocScratchBytes) {
     snprintf(g_msg, sizeof(g_msg),
@@ -66,6 +73,10 @@ extern "C" moda_status_t moda_backward_noalloc(
              need, moda::kNoAllocScratchBytes);
     return MODA_ERR_UNSUPPORTED;
   }
+  s = injected_at_launch();
+  if (s != MODA_OK) return s;
+  s = check_device();
+  if (s != MODA_OK) return s;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
     snprintf(g_msg, sizeof(g_msg), "moda_backward_noalloc: no usable current CUDA device");

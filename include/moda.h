@@ -39,6 +39,12 @@
  * No entry point aborts or throws.  Kernels that detect an internal failure (a bounded
  * wait that ran out, an index check) record it in a per-device error word that
  * moda_check_device_errors() reads and clears.
+ *
+ * Fault injection (for testing a caller's error handling; not on the paper): when the
+ * environment variable MODA_FAULT_INJECT is "validate", every compute entry point returns
+ * MODA_ERR_INVALID_ARGUMENT before its argument checks; when it is "launch", it returns
+ * MODA_ERR_CUDA once its argument checks have passed, in place of the device query and
+ * the launch.  Nothing is launched in either case.  The variable is read on every call.
  */
 #ifndef MODA_H_
 #define MODA_H_
@@ -221,9 +227,13 @@ moda_status_t moda_backward_stages(const void *q, const void *k, const void *v,
  * the process exits.  Neither the caller nor the library allocates anything.
  *   - Sizes whose moda_backward_workspace_size() exceeds 64 MiB are rejected with
  *     MODA_ERR_UNSUPPORTED (about B*Hq*T <= 130000 rows at d = 128).
+ *   - Argument checks come first and need no device: a bad pointer or size is refused
+ *     (MODA_ERR_INVALID_ARGUMENT, or MODA_ERR_UNSUPPORTED for sizes beyond 64 MiB)
+ *     before anything touches the GPU.
  *   - The first call on a device (the calling thread's current device) looks up the
- *     array's device address with cudaGetSymbolAddress; make that first call before any
- *     stream capture begins.
+ *     array's device address with cudaGetSymbolAddress and caches it for the process;
+ *     make that first call before any stream capture begins.  A cudaDeviceReset()
+ *     between calls is not supported (the cached address would be stale).
  *   - Every call on a device shares the one array and leaves its contents behind.  The
  *     backward writes every workspace element it reads before reading it, so nothing has
  *     to be cleared between calls, but calls that may overlap on the GPU (different

@@ -185,3 +185,32 @@ def test_backward_stages_rejects_bad_masks(stages):
 def test_binding_has_no_fallback():
     src = open(os.path.join(ROOT, "depth_aware_attention_b200", "__init__.py")).read()
     assert "oracle" not in src.lower().replace("no cpu", "")
+
+
+NOALLOC_LIMIT = 64 << 20  # bytes of the no-allocation backward's static scratch
+
+
+def _noalloc(ptrs, B, Hq, Hkv, T, L, d, scale=0.088):
+    return moda.moda_backward_noalloc(*[None if p is None else ctypes.c_void_p(p) for p in ptrs],
+                                      B, Hq, Hkv, T, L, d, scale, 1, None)
+
+
+def test_noalloc_rejects_sizes_beyond_its_scratch_before_touching_the_gpu():
+    # 13 buffers 4 GiB apart, so that no size check sees an overlap.  The sizes must need
+    # more workspace than the static scratch holds: the call is then refused by that check
+    # and nothing is launched on the fake addresses.
+    sizes = (1, 16, 4, 16384, 4, 128)
+    assert moda.moda_backward_workspace_size(*sizes) > NOALLOC_LIMIT, \
+        "these sizes must exceed the no-allocation scratch, or the call would launch"
+    ptrs = [(i + 1) << 32 for i in range(13)]
+    assert _noalloc(ptrs, *sizes) == moda.MODA_ERR_UNSUPPORTED
+    assert "static scratch" in moda.moda_last_error_message()
+
+
+def test_noalloc_rejects_bad_pointers_before_touching_the_gpu():
+    sizes = (1, 4, 2, 64, 2, 64)
+    ptrs = [A * (i + 1) for i in range(13)]
+    assert _noalloc([None] + ptrs[1:], *sizes) == moda.MODA_ERR_INVALID_ARGUMENT
+    assert _noalloc([A * 1 + 8] + ptrs[1:], *sizes) == moda.MODA_ERR_INVALID_ARGUMENT
+    assert _noalloc(ptrs[:8] + [A * 2] + ptrs[9:], *sizes) == moda.MODA_ERR_INVALID_ARGUMENT
+    assert _noalloc(ptrs, *sizes, scale=float("inf")) == moda.MODA_ERR_INVALID_ARGUMENT
