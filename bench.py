@@ -234,7 +234,7 @@ def kernel_roofline(name, cfg, avg_ms, pk, workload):
         else:
             bound, work = "tensor", flops
             what = "4*B*Hq*d*(T^2/2 + T*L) FLOPs"
-    elif name == "moda_bwd_seq_kernel":
+    elif name in ("moda_bwd_seq_kernel", "moda_bwd_seq_h_kernel"):
         bound, work = "tensor", BWD_FLOP_FACTOR * 4.0 * B * Hq * d * T * T / 2.0
         what = "2.5 x 4*B*Hq*d*T^2/2 FLOPs (sequence part of the backward)"
     elif name == "moda_bwd_depth_kernel":
@@ -282,8 +282,10 @@ def run_moda(args, world, rank, local):
     # Every launch of the step is bracketed by CUDA events on the launching stream: the
     # forward kernel, then the backward's three stages (row terms + depth part, sequence
     # part, dq convert), each launched on its own through moda_backward_stages.
+    # the sequence stage runs the half-tile kernel at d = 128, the plain one at d = 64
+    seq_kernel = "moda_bwd_seq_h_kernel" if d == 128 else "moda_bwd_seq_kernel"
     names = ["moda_fwd_kernel"] + ([] if args.fwd_only else
-                                   ["moda_bwd_depth_kernel", "moda_bwd_seq_kernel",
+                                   ["moda_bwd_depth_kernel", seq_kernel,
                                     "moda_dq_convert_kernel"])
     events = {n: [] for n in names}
 
@@ -373,53 +375,92 @@ def run_moda(args, world, rank, local):
 
 def run_e2e(args, moda, cfg, x, scale, dev, stream, world):
     """Same metric through the public API from pinned HOST buffers: every step copies its
-    inputs host->device, runs the operator and reads the results back to the host."""
+    inputs host->device, runs the operator and reads every result back to the host.
+
+    The steps are pipelined on three streams with two device buffer sets: while step i
+    runs its kernels, step i+1's inputs are uploaded into the other set and step i-1's
+    results are read back (the two copy directions use separate copy engines).  A set's
+    inputs are overwritten only after the kernels that read them finished, and its
+    outputs only after their read-back finished.  The timed region covers K steps
+    including the pipeline's fill and drain."""
     names = ["q", "k", "v", "kd", "vd"] + ([] if args.fwd_only else ["dout"])
     host = {n: torch.empty(x[n].shape, dtype=x[n].dtype, pin_memory=True)
             for n in names if x[n] is not None}
     for n, h in host.items():
         h.copy_(x[n])
-    dbuf = {n: torch.empty_like(x[n]) for n in host}
     h2d = sum(h.numel() * h.element_size() for h in host.values())
     B, Hq, T, d = x["q"].shape
-    L = cfg["L"]
-    out_h = torch.empty(x["q"].shape, dtype=torch.bfloat16, pin_memory=True)
-    lse_h = torch.empty((B, Hq, T), dtype=torch.float32, pin_memory=True)
+    Hkv, L = x["k"].shape[1], cfg["L"]
+    res_names = ["out", "lse"] + ([] if args.fwd_only else
+                                  ["dq", "dk", "dv"] + (["dkd", "dvd"] if L else []))
+    like = dict(out=x["q"], dq=x["q"], dk=x["k"], dv=x["v"], dkd=x["kd"], dvd=x["vd"])
     res_h = {}
-    if not args.fwd_only:
-        for n in ["q", "k", "v"] + (["kd", "vd"] if L else []):
-            res_h["d" + n] = torch.empty(x[n].shape, dtype=torch.bfloat16, pin_memory=True)
-    d2h = out_h.numel() * 2 + lse_h.numel() * 4 + sum(r.numel() * 2 for r in res_h.values())
+    for n in res_names:
+        if n == "lse":
+            res_h[n] = torch.empty((B, Hq, T), dtype=torch.float32, pin_memory=True)
+        else:
+            res_h[n] = torch.empty(like[n].shape, dtype=torch.bfloat16, pin_memory=True)
+    d2h = sum(r.numel() * r.element_size() for r in res_h.values())
+    sets = []
+    for _ in range(2):
+        ins = {n: torch.empty_like(x[n]) for n in host}
+        outs = {n: torch.empty(r.shape, dtype=r.dtype, device=dev) for n, r in res_h.items()}
+        sets.append((ins, outs))
+    ws = None if args.fwd_only else torch.empty(
+        moda.moda_backward_workspace_size(B, Hq, Hkv, T, L, d), device=dev, dtype=torch.uint8)
+    s_up, s_run, s_down = (torch.cuda.Stream(dev) for _ in range(3))
+    ran = [torch.cuda.Event() for _ in range(2)]   # kernels that read set i finished
+    read = [torch.cuda.Event() for _ in range(2)]  # set i's results are on the host
+    for e in ran + read:
+        e.record(stream)
 
-    def step():
-        for n, h in host.items():
-            dbuf[n].copy_(h, non_blocking=True)
-        out, lse = moda.forward(dbuf["q"], dbuf["k"], dbuf["v"], dbuf.get("kd"), dbuf.get("vd"),
-                                scale, True)
-        out_h.copy_(out, non_blocking=True)
-        lse_h.copy_(lse, non_blocking=True)
-        if not args.fwd_only:
-            g = moda.backward(dbuf["q"], dbuf["k"], dbuf["v"], dbuf.get("kd"), dbuf.get("vd"),
-                              out, lse, dbuf["dout"], scale, True)
+    def step(i):
+        ins, outs = sets[i % 2]
+        up = torch.cuda.Event()
+        with torch.cuda.stream(s_up):
+            s_up.wait_event(ran[i % 2])
+            for n, h in host.items():
+                ins[n].copy_(h, non_blocking=True)
+            up.record(s_up)
+        with torch.cuda.stream(s_run):
+            s_run.wait_event(up)
+            s_run.wait_event(read[i % 2])
+            moda.forward(ins["q"], ins["k"], ins["v"], ins.get("kd"), ins.get("vd"), scale,
+                         True, out=outs["out"], lse=outs["lse"])
+            if not args.fwd_only:
+                grads = {n: outs.get(n) for n in ("dq", "dk", "dv", "dkd", "dvd")}
+                moda.backward(ins["q"], ins["k"], ins["v"], ins.get("kd"), ins.get("vd"),
+                              outs["out"], outs["lse"], ins["dout"], scale, True,
+                              workspace=ws, grads=grads)
+            ran[i % 2].record(s_run)
+        with torch.cuda.stream(s_down):
+            s_down.wait_event(ran[i % 2])
             for n, r in res_h.items():
-                r.copy_(g[n], non_blocking=True)
+                r.copy_(outs[n], non_blocking=True)
+            read[i % 2].record(s_down)
 
-    steps = max(1, min(args.steps, 3))
-    step()
-    torch.cuda.synchronize(dev)
+    def run(k):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for st in (s_up, s_run, s_down):
+            st.wait_event(e0)
+        for i in range(k):
+            step(i)
+        for st in (s_up, s_run, s_down):
+            stream.wait_stream(st)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1)
+
+    run(2)  # warm-up: both buffer sets once
     barrier(world)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(steps):
-        step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier(world)
-    ms = max_over_ranks(e0.elapsed_time(e1) / steps, world)
+    steps = max(1, args.steps)
+    ms = max_over_ranks(run(steps) / steps, world)
     value = job_value(step_flops(cfg, args.fwd_only), world, ms)
-    del host, dbuf, out_h, lse_h, res_h
+    del host, sets, res_h, ws
     return {"value": round(value, 2), "unit": UNIT, "ms_per_step": round(ms, 3),
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "pipeline": "three streams (upload, kernels, read-back), two device buffer sets"}
 
 
 # ----------------------------------------------------------------------------- CPU oracle
@@ -430,9 +471,9 @@ def oracle_sample(cfg, seed_base, cpu_seconds, fwd_only):
     causal problem) with all heads; its algorithmic FLOPs are summed row by row with the
     same per-row count as the full problem (4*d*(|visible keys| + L) forward, x2.5 for the
     backward).  nt grows until the sample takes about cpu_seconds.  ``cores`` is the number
-    of threads the oracle actually ran: its forward splits rows over the host's threads, its
-    backward one (batch, KV head) unit per thread.  A second, smaller sample on one thread
-    gives ``value_1_thread``.
+    of threads the oracle actually ran: its forward splits rows, its backward the window's
+    tokens, over the host's threads.  A second, smaller sample on one thread gives
+    ``value_1_thread``.
     """
     import oracle
     g = torch.Generator().manual_seed(seed_base)
@@ -468,13 +509,13 @@ def oracle_sample(cfg, seed_base, cpu_seconds, fwd_only):
     if sec < cpu_seconds / 2 and nt < T:
         nt = min(T, max(nt + 1, int(nt * cpu_seconds / max(sec, 1e-3))))
         fl, sec = sample(nt)
-    used = min(threads, B * Hq * nt if fwd_only else B * Hkv)
+    used = min(threads, B * Hq * nt if fwd_only else nt)
     # one thread, on about a quarter of the time budget
     nt1 = max(1, nt // (4 * used))
     fl1, sec1 = sample(nt1, 1)
     what = "forward" if fwd_only else "forward+backward"
     return {"value": round(fl / sec / 1e12, 6), "unit": UNIT, "cores": used, "kind": "oracle",
-            "seconds": round(sec, 2), "host_threads": threads,
+            "seconds": round(sec, 2), "host_threads": threads, "sample_tokens": nt,
             "value_1_thread": round(fl1 / sec1 / 1e12, 6), "sample_1_thread_tokens": nt1,
             "sample": f"fp64 oracle {what} on the last {nt} query tokens (all {B * Hq} "
                       f"heads) of the {cfg['T']}-token workload, L={L}; FLOPs counted "
