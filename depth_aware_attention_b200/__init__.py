@@ -33,8 +33,8 @@ EXPORTED = ("moda_forward", "moda_forward_depth_path", "moda_depth_attention_for
             "moda_depth_attention_backward", "moda_decode", "moda_decode_workspace_size",
             "moda_depth_kv_write",
             "moda_backward", "moda_backward_workspace_size",
-            "moda_backward_stages", "moda_backward_noalloc", "moda_check_device_errors", "moda_status_string",
-            "moda_last_error_message")
+            "moda_backward_stages", "moda_backward_noalloc", "moda_check_device_errors",
+            "moda_test_set_device_fault", "moda_status_string", "moda_last_error_message")
 
 
 class ModaError(RuntimeError):
@@ -72,6 +72,8 @@ def _load():
     lib.moda_backward_stages.restype = I
     lib.moda_backward_noalloc.argtypes = [P] * 13 + [I] * 6 + [F, I, P]
     lib.moda_backward_noalloc.restype = I
+    lib.moda_test_set_device_fault.argtypes = [I, ctypes.c_uint64]
+    lib.moda_test_set_device_fault.restype = I
     lib.moda_check_device_errors.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
     lib.moda_check_device_errors.restype = I
     lib.moda_status_string.argtypes = [I]
@@ -169,6 +171,12 @@ def moda_check_device_errors(stream=None):
     flags = ctypes.c_uint32(0)
     st = lib.moda_check_device_errors(stream, ctypes.byref(flags))
     return st, int(flags.value)
+
+
+def moda_test_set_device_fault(fault, wait_limit_ns=0):
+    """TEST ONLY: set the kernels' injected fault and bounded-wait limit on the current
+    device (0, 0 restores the normal state).  Returns the status."""
+    return lib.moda_test_set_device_fault(int(fault), int(wait_limit_ns))
 
 
 def moda_status_string(status):

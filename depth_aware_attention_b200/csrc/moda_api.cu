@@ -464,6 +464,22 @@ moda_status_t moda_depth_attention_backward(const void* q, const void* kd, const
                         moda::kStagesAll, 1, stream);
 }
 
+moda_status_t moda_test_set_device_fault(int fault, uint64_t wait_limit_ns) {
+  g_msg[0] = 0;
+  if (fault < 0 || fault > moda::kFaultForwardNoLoads)
+    return fail(MODA_ERR_INVALID_ARGUMENT, "fault must be 0 (none) or 1 (forward issues no loads)");
+  if (wait_limit_ns != 0 && (wait_limit_ns < 100000ull || wait_limit_ns > 10000000000ull))
+    return fail(MODA_ERR_INVALID_ARGUMENT, "wait_limit_ns must be 0 or lie in [1e5, 1e10]");
+  moda_status_t s = check_device();
+  if (s != MODA_OK) return s;
+  const uint64_t limit = wait_limit_ns ? wait_limit_ns : moda::kWaitLimitNs;
+  cudaError_t e = cudaMemcpyToSymbol(moda::g_wait_limit_ns, &limit, sizeof(limit));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(moda::g_device_fault, &fault, sizeof(fault));
+  if (e != cudaSuccess)
+    return fail(MODA_ERR_CUDA, "setting the test knobs failed: %s", cudaGetErrorString(e));
+  return MODA_OK;
+}
+
 moda_status_t moda_check_device_errors(moda_stream_t stream, uint32_t* flags) {
   g_msg[0] = 0;
   if (flags) *flags = 0;

@@ -52,6 +52,10 @@ struct BwdDepthArgs {
   float* drow;   // [B][Hq][T] fp32: D = <dO, out>
   long long ntok;  // B * Hkv * T
   int T, L, G;
+  // 1 (depth-only attention): the row terms are formed from the depth logits themselves,
+  // D = sum_j P_j <dO, vd_j>, in a first pass over the token's entries, instead of from
+  // the rounded out.  Every key of such a row is a depth key, so this is the exact D.
+  int exact_rows;
   float scale, scale_log2;
 };
 
@@ -140,6 +144,67 @@ __global__ void __launch_bounds__(kDepthThreads, GM <= 4 ? 3 : 1)
       for (int e = 0; e < 8; ++e) dq[h][e] = 0.f;
 
     const long long tok_off = (bg * a.T + t) * L * D + cs * 8;
+    if (a.exact_rows) {
+      // D_h = sum_j P_hj <dO_h, vd_j> with P_hj = 2^(y_hj * scale * log2(e) - lse_h * log2(e)),
+      // the same weights the gradient loop below recomputes; kd and vd are read once more.
+      float dsum[GM];
+#pragma unroll
+      for (int h = 0; h < GM; ++h) dsum[h] = 0.f;
+#pragma unroll 4
+      for (long long j = 0; j < L; ++j) {
+        uint4 kw = make_uint4(0, 0, 0, 0), vw = make_uint4(0, 0, 0, 0);
+        if (valid) {
+          kw = ldg_nc_v4(a.kd + tok_off + j * D);
+          vw = ldg_nc_v4(a.vd + tok_off + j * D);
+        }
+        float kf[8], vf[8];
+        unpack8(kw, kf);
+        unpack8(vw, vf);
+        float y[GM], p[GM];
+#pragma unroll
+        for (int h = 0; h < GM; ++h) {
+          y[h] = p[h] = 0.f;
+          if (h < G) {
+            float qf[8], df[8];
+            if constexpr (kReg) {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                qf[e] = qreg[h][e];
+                df[e] = dreg[h][e];
+              }
+            } else {
+              unpack8(lds128(q_s + uint32_t((h * D + cs * 8) * 2)), qf);
+              unpack8(lds128(do_s + uint32_t((h * D + cs * 8) * 2)), df);
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              y[h] = fmaf(qf[e], kf[e], y[h]);
+              p[h] = fmaf(df[e], vf[e], p[h]);
+            }
+          }
+        }
+#pragma unroll
+        for (int o = NT / 2; o > 0; o >>= 1) {
+#pragma unroll
+          for (int h = 0; h < GM; ++h) {
+            if (h < G) {
+              y[h] += __shfl_xor_sync(0xffffffffu, y[h], o);
+              p[h] += __shfl_xor_sync(0xffffffffu, p[h], o);
+            }
+          }
+        }
+#pragma unroll
+        for (int h = 0; h < GM; ++h)
+          if (h < G) dsum[h] = fmaf(ex2(y[h] * a.scale_log2 - lse2[h]), p[h], dsum[h]);
+      }
+#pragma unroll
+      for (int h = 0; h < GM; ++h) {
+        if (h < G) {
+          drw[h] = dsum[h];
+          if (valid && cs == 0) a.drow[(bg * G + h) * a.T + t] = dsum[h];
+        }
+      }
+    }
     const long long nbat = (L + kU - 1) / kU;
     // batch b's copies (an empty group past the last batch keeps the group count uniform)
     auto issue = [&](long long b) {
@@ -681,7 +746,18 @@ struct SeqHBars {
   uint64_t kv_done;
   uint32_t tmem_base;
   int abort;
+  int lo_tile[2];  // half h of tile i needs its lo passes iff lo_tile[h] == i + 1
 };
+
+// The lo halves of P and dS (x - bf16(x)) enter the dV and dK products only for the half
+// tiles where some of them exceeds this size.  A dropped lo value is at most 2^-9 of its
+// element, so below it the element is small (P or dS under about 2^-6), and a half tile's
+// 64 such terms move a dV or dK entry by far less than the output's own bf16 rounding.
+// Large weights (short sequences, the first rows of long ones) keep both passes.
+#ifndef MODA_BWD_LO_KEEP
+#define MODA_BWD_LO_KEEP 3.0517578125e-05f  // 2^-15
+#endif
+constexpr float kLoKeep = MODA_BWD_LO_KEEP;
 
 // dQ warps of moda_bwd_seq_h_kernel.  Thread = TMEM lane = head-dimension index c of
 // dQ^T_h: per half it reads its 64 row values, frees the TMEM region at once and adds
@@ -786,6 +862,7 @@ __global__ void __launch_bounds__(kSeqHThreads, 1)
     }
     mbar_init(bar(bars->kv_done), 1);
     bars->abort = 0;
+    bars->lo_tile[0] = bars->lo_tile[1] = 0;
     fence_barrier_init();
   }
   // Q/dO rows past TQ*G (G not dividing 128) never receive TMA data: zero them once.
@@ -800,6 +877,7 @@ __global__ void __launch_bounds__(kSeqHThreads, 1)
       }
     fence_proxy_async_smem();
   }
+  volatile int* lo_tile = bars->lo_tile;
   if (warp == 13) {
     tmem_alloc(smem_u32(&bars->tmem_base), 512);
     tmem_relinquish();
@@ -884,19 +962,21 @@ __global__ void __launch_bounds__(kSeqHThreads, 1)
         mbar_wait(bar(bars->pds_full[h]), i & 1, abort_flag);
         tc_fence_after();
         const int st = i & 1;
+        // the P/dS warps marked this half before arriving on pds_full
+        const bool lo = lo_tile[h] == i + 1;
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
           const uint32_t col = (ks >> 1) * 32 + (ks & 1) * 8;
           const uint64_t bd = make_sdesc_sw128(sDO(st) + (4 * h + ks) * 2048, kBwdRegion, 1024);
           mma_ts(tDV, tA(h) + col, bd, idesc_g, (i > 0 || h > 0 || ks > 0) ? 1u : 0u);
-          mma_ts(tDV, tA(h) + col + 16, bd, idesc_g, 1u);
+          if (lo) mma_ts(tDV, tA(h) + col + 16, bd, idesc_g, 1u);
         }
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
           const uint32_t col = (ks >> 1) * 32 + (ks & 1) * 8;
           const uint64_t bd = make_sdesc_sw128(sQ(st) + (4 * h + ks) * 2048, kBwdRegion, 1024);
           mma_ts(tDK, tB(h) + col, bd, idesc_g, (i > 0 || h > 0 || ks > 0) ? 1u : 0u);
-          mma_ts(tDK, tB(h) + col + 16, bd, idesc_g, 1u);
+          if (lo) mma_ts(tDK, tB(h) + col + 16, bd, idesc_g, 1u);
         }
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
@@ -983,6 +1063,7 @@ __global__ void __launch_bounds__(kSeqHThreads, 1)
         const bool masked = r_min > c * 32;
         // dS for the dQ^T product: region h, this key's row, rows 32g..32g+31 of the half
         const uint32_t reg = sDS + h * kBwdRegion + uint32_t(kt) * 128;
+        float mlo = 0.f;  // largest lo value of this thread's P and dS elements
 #pragma unroll
         for (int k = 0; k < 2; ++k) {  // 16-row sub-chunks
           uint32_t pp[8], pl[8], pd[8], dl[8];
@@ -1007,6 +1088,8 @@ __global__ void __launch_bounds__(kSeqHThreads, 1)
             const float2 plo =
                 ffma2(make_float2(bf16lo(ph), bf16hi(ph)), neg1, make_float2(P0, P1));
             const float2 dlo = ffma2(make_float2(bf16lo(dh), bf16hi(dh)), neg1, dS);
+            mlo = fmax3(mlo, fabsf(plo.x), fabsf(plo.y));
+            mlo = fmax3(mlo, fabsf(dlo.x), fabsf(dlo.y));
             pp[e2 / 2] = ph;
             pl[e2 / 2] = pack_bf16x2(plo.x, plo.y);
             pd[e2 / 2] = dh;
@@ -1024,6 +1107,9 @@ __global__ void __launch_bounds__(kSeqHThreads, 1)
                    make_uint4(pd[qd * 4], pd[qd * 4 + 1], pd[qd * 4 + 2], pd[qd * 4 + 3]));
           }
         }
+        // mark the half for its lo passes (ordered before this lane's arrival below)
+        if (__any_sync(0xffffffffu, mlo > kLoKeep) && (threadIdx.x & 31) == 0)
+          lo_tile[h] = i + 1;
         tmem_wait_st();
         fence_proxy_async_smem();
         tc_fence_before();
@@ -1162,6 +1248,7 @@ cudaError_t launch_backward_d(const Problem& p, const void* q, const void* k, co
   da.T = p.T;
   da.L = p.L;
   da.G = p.G;
+  da.exact_rows = p.depth_only;
   da.scale = p.scale;
   da.scale_log2 = p.scale * kLog2eBwd;
   cudaError_t e = cudaSuccess;

@@ -91,37 +91,51 @@ struct Bars {
   uint64_t s_full[2];     // S_t(j) in TMEM
   uint64_t p_full[2];     // P_t(j) in TMEM (and O_t rescaled)
   uint64_t o_final[2];    // last PV_t done
+  uint64_t drain;         // abort path: every product issued so far has finished
   uint32_t tmem_base;
   int abort;
 };
 
-// Order of a tile pair's steps.  With ND depth steps and NB0 sequence blocks in tile 0,
-// the first 2K steps (K = min(ND, NB0)) alternate depth step, sequence block; then come
-// the remaining depth steps, then the remaining sequence blocks.  Spreading the depth
-// steps (HBM-bound) among the sequence blocks (tensor-bound) keeps both busy.  Tile 1
-// shares the mapping of every common step (its at most one extra block comes last), and
-// every depth step comes before step ND + NB0.  ND = 0: step j is sequence block j.
+// Sequence blocks between two interleaved depth steps of the dense depth path.  At 64K
+// tokens (G = 4, L = 32) a depth step brings 128 KB from HBM, about twice the time of a
+// sequence block's tensor work at one SM's share of the bandwidth; spacings 1 / 2 / 3 / 4
+// measured 18.0 / 17.5 / 17.2 / 17.5 ms there (L = 0: 16.2 ms).
+constexpr int kDepthSpacing = 3;
+
+// Order of a tile pair's steps.  With ND depth steps, NB0 sequence blocks in tile 0 and a
+// spacing R >= 1, the first K(R+1) steps (K = min(ND, NB0 / R)) repeat the pattern: one
+// depth step, then R sequence blocks; then come the remaining depth steps, then the
+// remaining sequence blocks.  Spreading the depth steps (HBM-bound) among the sequence
+// blocks (tensor-bound) keeps both busy.  Tile 1 shares the mapping of every common step
+// (its at most one extra block comes last), and every depth step comes before step
+// ND + NB0.  ND = 0: step j is sequence block j.
 struct StepMap {
-  int ND, K;
+  int ND, K, R;
   __device__ __forceinline__ bool is_depth(int j) const {
-    return j < 2 * K ? (j & 1) == 0 : (j - 2 * K) < ND - K;
+    const int P = R + 1;
+    return j < K * P ? j % P == 0 : (j - K * P) < ND - K;
   }
   // depth step index or sequence block index of step j
   __device__ __forceinline__ int index(int j) const {
-    if (j < 2 * K) return j >> 1;
-    const int jj = j - 2 * K;
-    return jj < ND - K ? K + jj : K + (jj - (ND - K));
+    const int P = R + 1;
+    if (j < K * P) {
+      const int q = j / P, m = j - q * P;
+      return m == 0 ? q : q * R + (m - 1);
+    }
+    const int jj = j - K * P;
+    return jj < ND - K ? K + jj : K * R + (jj - (ND - K));
   }
   // ring entries loaded before step j (4 per depth step, 2 per sequence block)
   __device__ __forceinline__ int entry(int j) const {
+    const int P = R + 1;
     int nd, ns;
-    if (j < 2 * K) {
-      nd = (j + 1) >> 1;
-      ns = j >> 1;
+    if (j < K * P) {
+      nd = (j + P - 1) / P;
+      ns = j - nd;
     } else {
-      const int jj = j - 2 * K;
+      const int jj = j - K * P;
       nd = K + min(jj, ND - K);
-      ns = K + max(0, jj - (ND - K));
+      ns = K * R + max(0, jj - (ND - K));
     }
     return 4 * nd + 2 * ns;
   }
@@ -177,7 +191,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const int ND = kDense ? nchunk : 0;  // tensor-core depth steps (ahead of the sequence)
   const int N0 = ND + NB0, N1 = ND + NB1;  // steps of tile 0 / tile 1
   constexpr int kDUses = 2 * Cfg::kRegions;   // depth stage uses per chunk: kd, vd regions
-  const StepMap sm{ND, min(ND, NB0)};
+  const StepMap sm{ND, min(ND, NB0 / kDepthSpacing), kDepthSpacing};
   // Ring entries in load order.  Depth step: kd of tile 0, kd of tile 1, vd of tile 0,
   // vd of tile 1; sequence block: K then V, shared by both tiles.
   auto kidx = [&](int t, int j) { return sm.entry(j) + (sm.is_depth(j) ? t : 0); };
@@ -198,6 +212,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_init(bar(bars->p_full[t]), 1);
       mbar_init(bar(bars->o_final[t]), 1);
     }
+    mbar_init(bar(bars->drain), 1);
     bars->abort = 0;
     fence_barrier_init();
   }
@@ -224,7 +239,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer lanes
     const int lane = threadIdx.x & 31;
-    if (lane == 0) {
+    // test-only fault: issue no loads, so that every wait for them runs out
+    const bool no_loads = g_device_fault == kFaultForwardNoLoads;
+    if (lane == 0 && !no_loads) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
@@ -234,27 +251,32 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           tma_load_4d(sQ(t) + rg * kRegion, &tmQ, bar(bars->q_full), rg * 64, 0,
                       t ? tq1 : tq0, bg);
       int e = 0;  // ring entry
+      // next ring stage, or -1 once a wait for a free stage has failed (the CTA aborts)
       auto acquire = [&](int bytes) {
         const int s = e % NKV;
-        if (e >= NKV) mbar_wait(bar(bars->empty[s]), ((e / NKV) - 1) & 1, abort_flag);
+        if (e >= NKV && !mbar_wait(bar(bars->empty[s]), ((e / NKV) - 1) & 1, abort_flag))
+          return -1;
         mbar_expect_tx(bar(bars->full[s]), uint32_t(bytes));
         ++e;
         return s;
       };
-      for (int j = 0; j < N1; ++j) {
+      bool stop = false;
+      for (int j = 0; j < N1 && !stop; ++j) {
         const int ix = sm.index(j);
         if (sm.is_depth(j)) {
           // depth chunk ix of each tile: entries [ix*JC, ix*JC+JC) of its TQ tokens
-          for (int u = 0; u < 4; ++u) {
+          for (int u = 0; u < 4 && !stop; ++u) {
             const int s = acquire(Cfg::kTileBytes);
+            if (s < 0) { stop = true; break; }
             const CUtensorMap* map = (u < 2) ? &tmKD : &tmVD;
             for (int rg = 0; rg < Cfg::kRegions; ++rg)
               tma_load_4d(sKV(s) + rg * kRegion, map, bar(bars->full[s]), rg * 64,
                           ix * a.JC, (u & 1) ? tq1 : tq0, bg);
           }
         } else {
-          for (int u = 0; u < 2; ++u) {
+          for (int u = 0; u < 2 && !stop; ++u) {
             const int s = acquire(Cfg::kTileBytes);
+            if (s < 0) { stop = true; break; }
             const CUtensorMap* map = u ? &tmV : &tmK;
             for (int rg = 0; rg < Cfg::kRegions; ++rg)
               tma_load_3d(sKV(s) + rg * kRegion, map, bar(bars->full[s]), rg * 64, ix * kBN,
@@ -262,7 +284,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           }
         }
       }
-    } else if constexpr (!kDense) if ((lane == 1 || lane == 2) && NC > 0) {
+      if (*abort_flag) {
+        // abort path: the loads issued so far still land in shared memory; wait for them
+        // (Q, and the last NKV ring entries: every earlier one was consumed) before exit
+        mbar_wait_drain(bar(bars->q_full), 0);
+        for (int i = (e > NKV ? e - NKV : 0); i < e; ++i)
+          mbar_wait_drain(bar(bars->full[i % NKV]), (i / NKV) & 1);
+      }
+    } else if constexpr (!kDense) if ((lane == 1 || lane == 2) && NC > 0 && !no_loads) {
       // Depth chunk ci of tile t: entries [ci*JC, ci*JC+JC) of the tile's TQ tokens as
       // rows (token, entry), one 64-column region per stage: kd regions, then vd regions.
       const int t = lane - 1;
@@ -286,6 +315,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         box(idx, map, x, y);
         tma_prefetch_l2_4d(map, x, y, t ? tq1 : tq0, bg);
       }
+      int issued = 0;
       for (int idx = 0; idx < nuse; ++idx) {
         if (idx + kDPrefetch < nuse) {
           const CUtensorMap* pmap; int px, py;
@@ -293,14 +323,21 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           tma_prefetch_l2_4d(pmap, px, py, t ? tq1 : tq0, bg);
         }
         const int s = idx % NDS;
-        if (idx >= NDS)
-          mbar_wait(bar(bars->dempty[t][s]), ((idx / NDS) - 1) & 1, abort_flag);
+        if (idx >= NDS &&
+            !mbar_wait(bar(bars->dempty[t][s]), ((idx / NDS) - 1) & 1, abort_flag))
+          break;
         const int u = idx % kDUses;
         const CUtensorMap* map = (u < Cfg::kRegions) ? &tmKD : &tmVD;
         const int rg = u % Cfg::kRegions;
         mbar_expect_tx(bar(bars->dfull[t][s]), dbytes);
         tma_load_4d(sDS(t, s), map, bar(bars->dfull[t][s]), rg * 64, (idx / kDUses) * a.JC,
                     t ? tq1 : tq0, bg);
+        issued = idx + 1;
+      }
+      if (*abort_flag) {
+        // abort path: wait for this ring's loads still in flight before exit
+        for (int i = (issued > NDS ? issued - NDS : 0); i < issued; ++i)
+          mbar_wait_drain(bar(bars->dfull[t][i % NDS]), (i / NDS) & 1);
       }
     }
     __syncwarp();
@@ -357,6 +394,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         issue_pv(1, j);
         if (j == N1 - 1) tc_commit(bar(bars->o_final[1]));
         if (j + 1 < N1) issue_s(1, j + 1);
+      }
+      if (*abort_flag) {
+        // abort path: let every product issued so far finish before TMEM is released
+        tc_commit(bar(bars->drain));
+        mbar_wait_drain(bar(bars->drain), 0);
       }
     }
     __syncwarp();

@@ -24,6 +24,14 @@ __device__ uint32_t g_error_word = 0;
 // A wait that has not completed after this many nanoseconds is treated as a failure.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
+// Test knobs, set only through moda_test_set_device_fault(): the limit every bounded wait
+// uses (kWaitLimitNs unless a test shortens it), and a fault the kernels inject on purpose
+// so that a test can watch the waits run out (0: none; kFaultForwardNoLoads: the forward
+// kernel's TMA producer issues no loads, so every wait for its data runs out).
+constexpr int kFaultForwardNoLoads = 1;
+__device__ uint64_t g_wait_limit_ns = kWaitLimitNs;
+__device__ int g_device_fault = 0;
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -97,18 +105,35 @@ __device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t par
 }
 
 // Waits until the phase with the given parity has completed.  Bounded: returns false
-// (and records kErrTimeout) if it has not after kWaitLimitNs, or at once if *abort is
+// (and records kErrTimeout) if it has not after g_wait_limit_ns, or at once if *abort is
 // already set by another thread of the CTA; sets *abort itself on a timeout.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
                                           volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
+  const uint64_t limit = *reinterpret_cast<volatile uint64_t*>(&g_wait_limit_ns);
   while (true) {
     if (mbar_try_wait_suspend(bar, parity)) return true;
     if (*abort) return false;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > limit) {
       atomicOr(&g_error_word, kErrTimeout);
       *abort = 1;
+      return false;
+    }
+  }
+}
+
+// The wait of the abort path: the CTA has given up (*abort is set) and now lets its own
+// asynchronous operations in flight (TMA loads, tensor-core products) finish before it
+// releases TMEM and exits.  Bounded by the same limit, but not cut short by the abort flag.
+__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  const uint64_t limit = *reinterpret_cast<volatile uint64_t*>(&g_wait_limit_ns);
+  while (true) {
+    if (mbar_try_wait_suspend(bar, parity)) return true;
+    if (globaltimer() - t0 > limit) {
+      atomicOr(&g_error_word, kErrTimeout);
       return false;
     }
   }

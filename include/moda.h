@@ -255,6 +255,23 @@ moda_status_t moda_backward_noalloc(const void *q, const void *k, const void *v,
  */
 moda_status_t moda_check_device_errors(moda_stream_t stream, uint32_t *flags);
 
+/*
+ * TEST ONLY: exercises the kernels' failure detection without a real fault.  Sets, on the
+ * calling thread's current device, the limit every bounded kernel wait uses and a fault
+ * the kernels inject on purpose:
+ *   fault 0  none (the normal state);
+ *   fault 1  the forward kernel's TMA producer issues no loads, so every wait for that
+ *            data runs out after wait_limit_ns: each CTA records the timeout in the
+ *            device error word, lets the operations it has in flight finish, releases its
+ *            tensor memory and exits (its out and lse are then meaningless), and
+ *            moda_check_device_errors() returns MODA_ERR_TIMEOUT.
+ * wait_limit_ns: 0 restores the default limit (2 s), otherwise 1e5..1e10 ns.  Call it
+ * with no kernel of this library in flight on the device, and call it again with (0, 0)
+ * afterwards.  MODA_ERR_INVALID_ARGUMENT for other values, MODA_ERR_CUDA or
+ * MODA_ERR_UNSUPPORTED from the device check.  Not part of the paper's operator.
+ */
+moda_status_t moda_test_set_device_fault(int fault, uint64_t wait_limit_ns);
+
 /* Static English description of a status code.  Never NULL. */
 const char *moda_status_string(moda_status_t status);
 

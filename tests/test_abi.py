@@ -214,3 +214,10 @@ def test_noalloc_rejects_bad_pointers_before_touching_the_gpu():
     assert _noalloc([A * 1 + 8] + ptrs[1:], *sizes) == moda.MODA_ERR_INVALID_ARGUMENT
     assert _noalloc(ptrs[:8] + [A * 2] + ptrs[9:], *sizes) == moda.MODA_ERR_INVALID_ARGUMENT
     assert _noalloc(ptrs, *sizes, scale=float("inf")) == moda.MODA_ERR_INVALID_ARGUMENT
+
+
+def test_test_fault_knob_rejects_bad_values_before_touching_the_gpu():
+    assert moda.moda_test_set_device_fault(2, 0) == moda.MODA_ERR_INVALID_ARGUMENT
+    assert moda.moda_test_set_device_fault(-1, 0) == moda.MODA_ERR_INVALID_ARGUMENT
+    assert moda.moda_test_set_device_fault(0, 5) == moda.MODA_ERR_INVALID_ARGUMENT
+    assert moda.moda_test_set_device_fault(0, 20_000_000_000) == moda.MODA_ERR_INVALID_ARGUMENT
