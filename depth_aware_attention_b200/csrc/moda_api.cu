@@ -42,10 +42,9 @@ moda_status_t check_sizes(int B, int Hq, int Hkv, int T, int L, int d) {
     return fail(MODA_ERR_INVALID_ARGUMENT, "sizes must satisfy B,Hq,Hkv,T >= 1 and L >= 0");
   if (Hq % Hkv != 0) return fail(MODA_ERR_INVALID_ARGUMENT, "Hq must be a multiple of Hkv");
   if (d != 64 && d != 128) return fail(MODA_ERR_UNSUPPORTED, "head size d must be 64 or 128");
-  // Groups above 16 are refused: the parity tests cover G <= 16, and the forward's dense
-  // depth blocks give each row only the keys inside its warp's 32 columns, which holds a
-  // token's G entries only for G <= 32.
-  if (Hq / Hkv > 16) return fail(MODA_ERR_UNSUPPORTED, "query heads per KV head must be <= 16");
+  // Groups above 64 are refused: a query tile holds 128 / G tokens, and the parity tests
+  // cover groups up to 64.
+  if (Hq / Hkv > 64) return fail(MODA_ERR_UNSUPPORTED, "query heads per KV head must be <= 64");
   // index arithmetic in the kernels uses 32-bit tile/row counts and 64-bit offsets
   const long long rows = 1LL * B * Hq * T;
   if (rows > (1LL << 31) || 1LL * B * Hkv > 65535 || T > (1 << 30) || L > 65535)
@@ -218,7 +217,7 @@ moda_status_t moda_forward_depth_path(const void* q, const void* k, const void* 
 }
 
 size_t moda_decode_workspace_size(int B, int Hq, int Hkv, int S, int L, int d) {
-  if (check_sizes(B, Hq, Hkv, S, L, d) != MODA_OK || Hq / Hkv > 16) return 0;
+  if (check_sizes(B, Hq, Hkv, S, L, d) != MODA_OK) return 0;
   moda::Problem p{B, Hq, Hkv, S, L, d, Hq / Hkv, 1, 1.f};
   return moda::decode_workspace_bytes(p);
 }
@@ -232,8 +231,6 @@ moda_status_t moda_decode(const void* q, const void* k, const void* v, const voi
   if (s != MODA_OK) return s;
   s = check_sizes(B, Hq, Hkv, S, L, d);
   if (s != MODA_OK) return s;
-  if (Hq / Hkv > 16)
-    return fail(MODA_ERR_UNSUPPORTED, "decode supports at most 16 query heads per KV head");
   if (!q || !k || !v || !out || !lse || !workspace)
     return fail(MODA_ERR_INVALID_ARGUMENT, "q, k, v, out, lse and workspace must be non-NULL");
   if (L > 0 && (!kd || !vd))
@@ -366,8 +363,6 @@ moda_status_t backward_entry(const void* q, const void* k, const void* v, const 
     return fail(MODA_ERR_INVALID_ARGUMENT, "workspace must be 256-byte aligned");
   if (!(scale == scale) || scale == INFINITY || scale == -INFINITY)
     return fail(MODA_ERR_INVALID_ARGUMENT, "scale must be finite");
-  if (Hq / Hkv > 16)
-    return fail(MODA_ERR_UNSUPPORTED, "the backward supports at most 16 query heads per KV head");
   moda::Problem p{B, Hq, Hkv, T, L, d, Hq / Hkv, causal ? 1 : 0, scale};
   p.depth_only = depth_only ? 1 : 0;
   if (validate_only) {

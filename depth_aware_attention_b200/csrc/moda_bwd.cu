@@ -40,6 +40,7 @@ constexpr float kLog2eBwd = 1.4426950408889634f;
 
 // ============================================================ 1. depth + row terms
 constexpr int kDepthThreads = 128;
+constexpr int kDepthMaxG = 16;  // heads of one depth-kernel launch (registers hold their dq)
 constexpr int kDepthU = 2;     // depth entries per load batch
 constexpr int kDepthRing = 8;  // per-thread cp.async ring stages (batches in flight: 7)
 constexpr int kDepthRingBytes = kDepthRing * kDepthU * 2 * kDepthThreads * 16;
@@ -56,6 +57,13 @@ struct BwdDepthArgs {
   // D = sum_j P_j <dO, vd_j>, in a first pass over the token's entries, instead of from
   // the rounded out.  Every key of such a row is a depth key, so this is the exact D.
   int exact_rows;
+  // Groups above kDepthMaxG heads run as several launches, one per chunk of at most
+  // kDepthMaxG heads: G is this chunk's head count, head0 its first head, Gfull the group
+  // size.  dkd/dvd sum over all the group's heads, so the chunks add their contributions
+  // into fp32 accumulators in the workspace (acc_mode 1: write, 2: add, 3: add and store
+  // the bf16 result); acc_mode 0: the whole group in one launch, bf16 stored directly.
+  int head0, Gfull, acc_mode;
+  float *dkd_acc, *dvd_acc;  // [B][Hkv][T][L][D] fp32 (acc_mode != 0)
   float scale, scale_log2;
 };
 
@@ -108,7 +116,7 @@ __global__ void __launch_bounds__(kDepthThreads, GM <= 4 ? 3 : 1)
         for (int e = 0; e < 8; ++e) qreg[h][e] = dreg[h][e] = 0.f;
       }
       if (h < G) {
-        const long long row = (bg * G + h) * a.T + t;
+        const long long row = (bg * a.Gfull + a.head0 + h) * a.T + t;
         float part = 0.f;
         if (valid) {
           const uint4 qw = ldg_nc_v4(a.q + row * D + cs * 8);
@@ -201,7 +209,7 @@ __global__ void __launch_bounds__(kDepthThreads, GM <= 4 ? 3 : 1)
       for (int h = 0; h < GM; ++h) {
         if (h < G) {
           drw[h] = dsum[h];
-          if (valid && cs == 0) a.drow[(bg * G + h) * a.T + t] = dsum[h];
+          if (valid && cs == 0) a.drow[(bg * a.Gfull + a.head0 + h) * a.T + t] = dsum[h];
         }
       }
     }
@@ -315,8 +323,31 @@ __global__ void __launch_bounds__(kDepthThreads, GM <= 4 ? 3 : 1)
         }
       }
       if (valid) {
-        *reinterpret_cast<uint4*>(a.dvd + tok_off + j * D) = pack8(dv, 1.f);
-        *reinterpret_cast<uint4*>(a.dkd + tok_off + j * D) = pack8(dk, a.scale);
+        const long long o = tok_off + j * D;
+        if (a.acc_mode == 0) {
+          *reinterpret_cast<uint4*>(a.dvd + o) = pack8(dv, 1.f);
+          *reinterpret_cast<uint4*>(a.dkd + o) = pack8(dk, a.scale);
+        } else {
+          // this chunk's heads' share, summed with the other chunks' in fp32
+          float4* av = reinterpret_cast<float4*>(a.dvd_acc + o);
+          float4* ak = reinterpret_cast<float4*>(a.dkd_acc + o);
+          if (a.acc_mode != 1) {
+            const float4 v0 = av[0], v1 = av[1], k0 = ak[0], k1 = ak[1];
+            dv[0] += v0.x; dv[1] += v0.y; dv[2] += v0.z; dv[3] += v0.w;
+            dv[4] += v1.x; dv[5] += v1.y; dv[6] += v1.z; dv[7] += v1.w;
+            dk[0] += k0.x; dk[1] += k0.y; dk[2] += k0.z; dk[3] += k0.w;
+            dk[4] += k1.x; dk[5] += k1.y; dk[6] += k1.z; dk[7] += k1.w;
+          }
+          if (a.acc_mode == 3) {
+            *reinterpret_cast<uint4*>(a.dvd + o) = pack8(dv, 1.f);
+            *reinterpret_cast<uint4*>(a.dkd + o) = pack8(dk, a.scale);
+          } else {
+            av[0] = make_float4(dv[0], dv[1], dv[2], dv[3]);
+            av[1] = make_float4(dv[4], dv[5], dv[6], dv[7]);
+            ak[0] = make_float4(dk[0], dk[1], dk[2], dk[3]);
+            ak[1] = make_float4(dk[4], dk[5], dk[6], dk[7]);
+          }
+        }
       }
       }
     }
@@ -326,7 +357,7 @@ __global__ void __launch_bounds__(kDepthThreads, GM <= 4 ? 3 : 1)
 #pragma unroll
       for (int h = 0; h < GM; ++h) {
         if (h < G) {
-          const long long row = (bg * G + h) * a.T + t;
+          const long long row = (bg * a.Gfull + a.head0 + h) * a.T + t;
           float4* dst = reinterpret_cast<float4*>(a.dqacc + row * D + cs * 8);
           dst[0] = make_float4(dq[h][0] * a.scale, dq[h][1] * a.scale, dq[h][2] * a.scale,
                                dq[h][3] * a.scale);
@@ -1248,21 +1279,39 @@ cudaError_t launch_backward_d(const Problem& p, const void* q, const void* k, co
   da.T = p.T;
   da.L = p.L;
   da.G = p.G;
+  da.head0 = 0;
+  da.Gfull = p.G;
+  da.acc_mode = 0;
+  da.dkd_acc = da.dvd_acc = nullptr;
   da.exact_rows = p.depth_only;
   da.scale = p.scale;
   da.scale_log2 = p.scale * kLog2eBwd;
   cudaError_t e = cudaSuccess;
   if (stages & kStageDepth) {
-    if (p.G <= 1)
-      e = launch_depth<D, 1>(da, stream, why);
-    else if (p.G <= 2)
-      e = launch_depth<D, 2>(da, stream, why);
-    else if (p.G <= 4)
-      e = launch_depth<D, 4>(da, stream, why);
-    else if (p.G <= 8)
-      e = launch_depth<D, 8>(da, stream, why);
-    else
-      e = launch_depth<D, 16>(da, stream, why);
+    auto launch = [&]() {
+      if (da.G <= 1) return launch_depth<D, 1>(da, stream, why);
+      if (da.G <= 2) return launch_depth<D, 2>(da, stream, why);
+      if (da.G <= 4) return launch_depth<D, 4>(da, stream, why);
+      if (da.G <= 8) return launch_depth<D, 8>(da, stream, why);
+      return launch_depth<D, 16>(da, stream, why);
+    };
+    if (p.G <= kDepthMaxG) {
+      e = launch();
+    } else {
+      // one launch per chunk of kDepthMaxG heads; dkd/dvd summed in fp32 in the workspace
+      // after the dq accumulator and the row terms
+      const size_t off = (size_t(rows) * D * 4 + size_t(rows) * 4 + 255) & ~size_t(255);
+      const size_t nd = size_t(p.B) * p.Hkv * p.T * size_t(p.L) * D;
+      da.dkd_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + off);
+      da.dvd_acc = da.dkd_acc + nd;
+      const int nchunk = (p.G + kDepthMaxG - 1) / kDepthMaxG;
+      for (int c = 0; c < nchunk && e == cudaSuccess; ++c) {
+        da.head0 = c * kDepthMaxG;
+        da.G = min(kDepthMaxG, p.G - da.head0);
+        da.acc_mode = p.L == 0 ? 0 : (c == 0 ? 1 : (c == nchunk - 1 ? 3 : 2));
+        e = launch();
+      }
+    }
     if (e != cudaSuccess) return e;
   }
   // 2. sequence part (none for depth-only attention)
@@ -1366,7 +1415,10 @@ cudaError_t launch_backward_d(const Problem& p, const void* q, const void* k, co
 
 size_t backward_workspace_bytes(const Problem& p) {
   const size_t rows = size_t(p.B) * p.Hq * p.T;
-  return rows * p.d * 4 + rows * 4 + 256;
+  size_t bytes = rows * p.d * 4 + rows * 4 + 256;
+  // groups above kDepthMaxG heads: fp32 dkd and dvd accumulators for the chunked depth part
+  if (p.G > kDepthMaxG) bytes += 2 * size_t(p.B) * p.Hkv * p.T * size_t(p.L) * p.d * 4;
+  return bytes;
 }
 
 cudaError_t launch_backward(const Problem& p, const void* q, const void* k, const void* v,

@@ -58,6 +58,10 @@ struct DecArgs {
   float* ws_acc;           // [BG][nsplit][G][D]
   float* ws_ml;            // [BG][nsplit][G][2]: m (log2 units), l
   int B, Hq, Hkv, S, L, G, nsplit, bps;  // bps: sequence blocks per split
+  // Groups above kDecMaxG heads run the split kernel once per chunk of at most kDecMaxG
+  // heads (each launch reads the K/V cache again): G is the chunk's head count, head0 its
+  // first head, Gfull the group size, which the workspace and the combine kernel index by.
+  int head0, Gfull;
   float scale_log2;
 };
 
@@ -111,7 +115,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   const int b = bg / a.Hkv, g = bg - (bg / a.Hkv) * a.Hkv;
   for (int i = threadIdx.x; i < G * D / 8; i += kDecThreads) {
     const int h = i / (D / 8), c = i - h * (D / 8);
-    const uint4 w = ldg_nc_v4(a.q + ((size_t(b) * a.Hq + g * G + h) * D + c * 8));
+    const uint4 w = ldg_nc_v4(a.q + ((size_t(b) * a.Hq + g * a.Gfull + a.head0 + h) * D + c * 8));
     sts128(s0 + Cfg::kOffQ + uint32_t((h * D + c * 8) * 2), w);
   }
   __syncthreads();
@@ -257,7 +261,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     named_bar_sync(1, 128);
   }
   if (kg == 0) {
-    const size_t base = (size_t(bg) * a.nsplit + split) * G;
+    const size_t base = (size_t(bg) * a.nsplit + split) * a.Gfull + a.head0;
 #pragma unroll
     for (int h = 0; h < GM; ++h) {
       if (h < G) {
@@ -281,12 +285,12 @@ template <int D>
 __global__ void __launch_bounds__(D) moda_decode_combine_kernel(const DecArgs a) {
   __shared__ float wgt[kDecMaxSplit], lsp[kDecMaxSplit];
   __shared__ float mmax;
-  const int bg = blockIdx.x / a.G, h = blockIdx.x - (blockIdx.x / a.G) * a.G;
+  const int bg = blockIdx.x / a.Gfull, h = blockIdx.x - (blockIdx.x / a.Gfull) * a.Gfull;
   const int d = threadIdx.x;
-  const size_t base = size_t(bg) * a.nsplit * a.G;
+  const size_t base = size_t(bg) * a.nsplit * a.Gfull;
   const int ns = a.nsplit;
   for (int s = d; s < ns; s += D) {
-    const size_t r = base + size_t(s) * a.G + h;
+    const size_t r = base + size_t(s) * a.Gfull + h;
     wgt[s] = a.ws_ml[r * 2];
     lsp[s] = a.ws_ml[r * 2 + 1];
   }
@@ -304,7 +308,7 @@ __global__ void __launch_bounds__(D) moda_decode_combine_kernel(const DecArgs a)
   __syncthreads();
   float den = 0.f, n0 = 0.f, n1 = 0.f, n2 = 0.f, n3 = 0.f;
   const float* accp = a.ws_acc + base * D + size_t(h) * D + d;  // split s at + s * G * D
-  const size_t stride = size_t(a.G) * D;
+  const size_t stride = size_t(a.Gfull) * D;
   int s = 0;
   for (; s + 4 <= ns; s += 4) {
     const float x0 = accp[size_t(s) * stride], x1 = accp[size_t(s + 1) * stride];
@@ -317,7 +321,7 @@ __global__ void __launch_bounds__(D) moda_decode_combine_kernel(const DecArgs a)
   for (; s < ns; ++s) n0 = fmaf(wgt[s], accp[size_t(s) * stride], n0);
   for (int t = 0; t < ns; ++t) den = fmaf(wgt[t], lsp[t], den);
   const int b = bg / a.Hkv, g = bg - (bg / a.Hkv) * a.Hkv;
-  const size_t row = size_t(b) * a.Hq + g * a.G + h;
+  const size_t row = size_t(b) * a.Hq + g * a.Gfull + h;
   a.out[row * D + d] = __float2bfloat16_rn(((n0 + n1) + (n2 + n3)) / den);
   if (d == 0) a.lse[row] = (Mu + __log2f(den)) * kLn2Dec;
 }
@@ -369,6 +373,8 @@ cudaError_t launch_decode_d(const Problem& p, const DecodeSplit& sp, const void*
   a.S = p.T;
   a.L = p.L;
   a.G = p.G;
+  a.head0 = 0;
+  a.Gfull = p.G;
   a.nsplit = sp.nsplit;
   a.bps = sp.blocks_per_split;
   a.scale_log2 = p.scale * kLog2eDec;
@@ -380,23 +386,26 @@ cudaError_t launch_decode_d(const Problem& p, const DecodeSplit& sp, const void*
                                                                             mVD, a);
     return cudaGetLastError();
   };
-  cudaError_t e;
-  switch (p.G) {
-    case 1: e = run(moda_decode_split_kernel<D, 1, true>); break;
-    case 2: e = run(moda_decode_split_kernel<D, 2, true>); break;
-    case 3: e = run(moda_decode_split_kernel<D, 4, false>); break;
-    case 4: e = run(moda_decode_split_kernel<D, 4, true>); break;
-    case 8: e = run(moda_decode_split_kernel<D, 8, true>); break;
-    case 16: e = run(moda_decode_split_kernel<D, 16, true>); break;
-    default:
-      e = p.G < 8 ? run(moda_decode_split_kernel<D, 8, false>)
-                  : run(moda_decode_split_kernel<D, 16, false>);
+  cudaError_t e = cudaSuccess;
+  for (a.head0 = 0; a.head0 < p.G && e == cudaSuccess; a.head0 += kDecMaxG) {
+    a.G = min(kDecMaxG, p.G - a.head0);  // heads of this chunk
+    switch (a.G) {
+      case 1: e = run(moda_decode_split_kernel<D, 1, true>); break;
+      case 2: e = run(moda_decode_split_kernel<D, 2, true>); break;
+      case 3: e = run(moda_decode_split_kernel<D, 4, false>); break;
+      case 4: e = run(moda_decode_split_kernel<D, 4, true>); break;
+      case 8: e = run(moda_decode_split_kernel<D, 8, true>); break;
+      case 16: e = run(moda_decode_split_kernel<D, 16, true>); break;
+      default:
+        e = a.G < 8 ? run(moda_decode_split_kernel<D, 8, false>)
+                    : run(moda_decode_split_kernel<D, 16, false>);
+    }
   }
   if (e != cudaSuccess) {
     *why = "decode split kernel launch failed";
     return e;
   }
-  moda_decode_combine_kernel<D><<<unsigned(BG) * p.G, D, 0, stream>>>(a);
+  moda_decode_combine_kernel<D><<<unsigned(BG) * a.Gfull, D, 0, stream>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) *why = "decode combine kernel launch failed";
   return e;

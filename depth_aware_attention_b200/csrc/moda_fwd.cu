@@ -756,7 +756,9 @@ cudaError_t launch_forward_d(const Problem& p, const void* q, const void* k, con
 
 }  // namespace
 
-bool dense_depth_supported(const Problem& p) { return 128 % p.G == 0; }
+// A dense depth block gives row r only the 32 columns of its own warp, which hold the G
+// entries of the row's token only when G <= 32 (and the block is whole when G divides 128).
+bool dense_depth_supported(const Problem& p) { return 128 % p.G == 0 && p.G <= 32; }
 
 bool dense_depth_default(const Problem& p) {
   return dense_depth_supported(p) && p.L >= kDenseDepthMinL;

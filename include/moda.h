@@ -21,10 +21,10 @@
  *   k, v, dk, dv     : bf16 [B][Hkv][T][d]
  *   kd, vd, dkd, dvd : bf16 [B][Hkv][T][L][d]     (may be NULL when L == 0)
  *   lse              : fp32 [B][Hq][T]
- * Sizes: B, T >= 1; Hq, Hkv >= 1 with Hq % Hkv == 0 and Hq / Hkv <= 16; L >= 0;
+ * Sizes: B, T >= 1; Hq, Hkv >= 1 with Hq % Hkv == 0 and Hq / Hkv <= 64; L >= 0;
  * d in {64, 128}.  scale is applied to every logit (typically 1/sqrt(d)) and must be
  * finite.  Violations give MODA_ERR_INVALID_ARGUMENT, except d outside {64, 128}, a
- * group Hq / Hkv above 16, and problems beyond the kernels' index ranges
+ * group Hq / Hkv above 64, and problems beyond the kernels' index ranges
  * (B*Hq*T > 2^31 rows, B*Hkv > 65535, T > 2^30 or L > 65535), which give
  * MODA_ERR_UNSUPPORTED.  Output buffers must not overlap any input or each other
  * (MODA_ERR_INVALID_ARGUMENT).
@@ -120,8 +120,7 @@ moda_status_t moda_depth_attention_forward(const void *q, const void *kd, const 
 /*
  * Depth-only attention backward: dq (bf16), dkd, dvd (bf16) of moda_depth_attention_forward
  * given dout, from its out and lse.  Workspace as for moda_backward (size from
- * moda_backward_workspace_size with the same sizes).  L >= 1; Hq/Hkv <= 16 as for
- * moda_backward (MODA_ERR_UNSUPPORTED beyond).  Two launches: the depth
+ * moda_backward_workspace_size with the same sizes).  L >= 1.  Two launches: the depth
  * part (row terms, dkd, dvd, fp32 dq) and the dq conversion; dq is deterministic here.
  */
 moda_status_t moda_depth_attention_backward(const void *q, const void *kd, const void *vd,
@@ -141,7 +140,8 @@ moda_status_t moda_depth_attention_backward(const void *q, const void *kd, const
  *   q, out: [B, Hq, d]    k, v: [B, Hkv, S, d]    kd, vd: [B, Hkv, L, d] (NULL iff L == 0)
  *   lse: [B, Hq] fp32     workspace: >= moda_decode_workspace_size(...) bytes, 256-byte
  *   aligned, owned by the caller, contents irrelevant between calls.
- * Hq/Hkv <= 16 (MODA_ERR_UNSUPPORTED otherwise).  The sequence is split over CTAs
+ * Groups above 16 heads run the split launch once per 16 heads (each reading the cache
+ * again).  The sequence is split over CTAs
  * (a function of the sizes only) and the partial softmax states are combined by a second
  * launch.  Other argument rules as moda_forward.
  */
@@ -173,7 +173,9 @@ moda_status_t moda_depth_kv_write(const void *x, const void *w, void *kd, void *
 
 /*
  * Bytes of device workspace moda_backward needs for these sizes (fp32 dQ accumulator
- * [B][Hq][T][d] plus the fp32 row terms D = <dO, out> [B][Hq][T]).
+ * [B][Hq][T][d] plus the fp32 row terms D = <dO, out> [B][Hq][T]; for groups Hq / Hkv
+ * above 16 also fp32 dkd and dvd accumulators, 2 x [B][Hkv][T][L][d]).  0 for invalid
+ * sizes.
  */
 size_t moda_backward_workspace_size(int B, int Hq, int Hkv, int T, int L, int d);
 
@@ -183,7 +185,8 @@ size_t moda_backward_workspace_size(int B, int Hq, int Hkv, int T, int L, int d)
  * D = <dout, out> per row and dS = P * (<dout, value> - D):
  *   dq = scale * sum dS * key,  dk/dkd = scale * sum dS * q,  dv/dvd = sum P * dout.
  * The pages give no backward design; this is the exact gradient of the definition.
- * Supports Hq / Hkv <= 16 (MODA_ERR_UNSUPPORTED beyond).  dq is summed with fp32 atomics,
+ * Groups above 16 heads run the depth part once per 16 heads, summing dkd and dvd in fp32
+ * accumulators that the workspace then also holds.  dq is summed with fp32 atomics,
  * so its last bits may differ between runs; dk, dv, dkd and dvd are deterministic.
  * `out` and `lse` must be the forward's outputs for the same inputs.  `workspace`
  * (device, >= moda_backward_workspace_size bytes, 256-byte aligned) is scratch owned

@@ -58,7 +58,7 @@ def fwd(**kw):
     (dict(Hq=3, Hkv=2), moda.MODA_ERR_INVALID_ARGUMENT),
     (dict(d=96), moda.MODA_ERR_UNSUPPORTED),
     (dict(Hq=256, Hkv=2), moda.MODA_ERR_UNSUPPORTED),
-    (dict(Hq=64, Hkv=2), moda.MODA_ERR_UNSUPPORTED),   # G = 32: beyond the tested groups
+    (dict(Hq=130, Hkv=1), moda.MODA_ERR_UNSUPPORTED),  # G = 130: beyond groups of 64
     (dict(q=None), moda.MODA_ERR_INVALID_ARGUMENT),
     (dict(kd=None), moda.MODA_ERR_INVALID_ARGUMENT),
     (dict(q=A + 8), moda.MODA_ERR_INVALID_ARGUMENT),
@@ -81,6 +81,7 @@ def test_forward_rejects_bad_arguments_before_launch(kw, status):
     (dict(), 3, moda.MODA_ERR_INVALID_ARGUMENT),
     (dict(), -1, moda.MODA_ERR_INVALID_ARGUMENT),
     (dict(Hq=6, Hkv=2), 2, moda.MODA_ERR_UNSUPPORTED),  # group of 3 does not divide 128
+    (dict(Hq=128, Hkv=2), 2, moda.MODA_ERR_UNSUPPORTED),  # group of 64: beyond a warp's columns
     (dict(q=None), 2, moda.MODA_ERR_INVALID_ARGUMENT),
 ])
 def test_forward_depth_path_rejects_bad_arguments(kw, path, status):
@@ -118,10 +119,10 @@ def test_decode_rejects_bad_arguments():
     assert st(workspace_bytes=16) == moda.MODA_ERR_INVALID_ARGUMENT
     assert st(workspace=A * 256 + 16) == moda.MODA_ERR_INVALID_ARGUMENT
     assert st(out=A * 2) == moda.MODA_ERR_INVALID_ARGUMENT  # out aliases k
-    assert st(Hq=64, Hkv=2) == moda.MODA_ERR_UNSUPPORTED
+    assert st(Hq=130, Hkv=1) == moda.MODA_ERR_UNSUPPORTED
     assert st(d=96) == moda.MODA_ERR_UNSUPPORTED
     assert moda.moda_decode_workspace_size(1, 16, 4, 65536, 32, 128) > 0
-    assert moda.moda_decode_workspace_size(1, 64, 2, 100, 1, 128) == 0
+    assert moda.moda_decode_workspace_size(1, 130, 1, 100, 1, 128) == 0
 
 
 def test_depth_kv_write_rejects_bad_arguments():
@@ -171,7 +172,7 @@ def test_backward_rejects_small_workspace_and_aliasing():
     assert st == moda.MODA_ERR_INVALID_ARGUMENT
     st = moda.moda_backward(**args, **dict(base, workspace=A * 64 + 16))  # not 256-aligned
     assert st == moda.MODA_ERR_INVALID_ARGUMENT
-    st = moda.moda_backward(**args, **dict(base, Hq=64, Hkv=2))  # group of 32 heads
+    st = moda.moda_backward(**args, **dict(base, Hq=256, Hkv=2))  # group of 128 heads
     assert st == moda.MODA_ERR_UNSUPPORTED
 
 

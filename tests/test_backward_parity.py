@@ -37,6 +37,11 @@ SMALL = [
     # that shift stays under 2e-3)
     ("g16-d64", dict(B=1, T=200, Hq=16, Hkv=1, d=64, L=8), True),
     ("L0-d128", dict(B=1, T=333, Hq=8, Hkv=2, d=128, L=0), True),
+    # groups above 16: the depth part runs per 16-head chunk with fp32 dkd/dvd sums.  The
+    # shapes keep the outputs' own bf16 rounding well inside the mean-abs bound: entries of
+    # dk and dv grow with the G*T rows a key collects (rounding alone: mean 6-8e-4 here)
+    ("g32-d128", dict(B=1, T=384, Hq=32, Hkv=1, d=128, L=16), True),
+    ("g64-d64", dict(B=1, T=512, Hq=64, Hkv=1, d=64, L=16), True),
     ("T1", dict(B=2, T=1, Hq=4, Hkv=2, d=128, L=6), True),
     ("longL-d128", dict(B=1, T=64, Hq=4, Hkv=1, d=128, L=130), True),
     ("noncausal-g4", dict(B=1, T=190, Hq=4, Hkv=1, d=128, L=4), False),

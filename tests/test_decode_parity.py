@@ -24,6 +24,8 @@ CASES = [
     ("g3-d128", dict(B=1, S=130, Hq=6, Hkv=2, d=128, L=7)),
     ("g8-d128-L0", dict(B=1, S=257, Hq=16, Hkv=2, d=128, L=0)),
     ("g16-d64", dict(B=1, S=100, Hq=16, Hkv=1, d=64, L=2)),
+    ("g32-d128", dict(B=2, S=300, Hq=32, Hkv=1, d=128, L=5)),    # two 16-head chunks
+    ("g64-d64", dict(B=1, S=150, Hq=128, Hkv=2, d=64, L=3)),     # four 16-head chunks
     ("S1", dict(B=3, S=1, Hq=4, Hkv=2, d=128, L=6)),
     ("longL", dict(B=1, S=64, Hq=4, Hkv=1, d=128, L=130)),
     ("many-splits", dict(B=1, S=20000, Hq=8, Hkv=2, d=128, L=24)),

@@ -28,6 +28,8 @@ CASES = [
     ("g8-d128", dict(B=1, T=257, Hq=16, Hkv=2, d=128, L=9)),
     ("g16-d64", dict(B=1, T=100, Hq=16, Hkv=1, d=64, L=2)),
     ("L1", dict(B=1, T=77, Hq=4, Hkv=2, d=128, L=1)),
+    ("g32-d128", dict(B=1, T=90, Hq=64, Hkv=2, d=128, L=6)),
+    ("g64-d64", dict(B=1, T=70, Hq=64, Hkv=1, d=64, L=4)),
     ("longL", dict(B=1, T=64, Hq=4, Hkv=1, d=128, L=130)),
 ]
 

@@ -26,6 +26,8 @@ SMALL = [
     ("g3-d128", dict(B=1, T=130, Hq=6, Hkv=2, d=128, L=7), True),
     ("g8-d128", dict(B=1, T=257, Hq=16, Hkv=2, d=128, L=9), True),
     ("g16-d64", dict(B=1, T=100, Hq=16, Hkv=1, d=64, L=2), True),
+    ("g32-d128", dict(B=1, T=150, Hq=32, Hkv=1, d=128, L=5), True),
+    ("g64-d64", dict(B=1, T=90, Hq=64, Hkv=1, d=64, L=3), True),
     ("L0-d128", dict(B=1, T=333, Hq=8, Hkv=2, d=128, L=0), True),
     ("T1", dict(B=2, T=1, Hq=4, Hkv=2, d=128, L=6), True),
     ("longL-d128", dict(B=1, T=64, Hq=4, Hkv=1, d=128, L=130), True),
@@ -49,11 +51,12 @@ def test_forward_small_full(name, cfg, causal):
 @pytest.mark.parametrize("name,cfg,causal", SMALL, ids=[s[0] for s in SMALL])
 def test_forward_small_full_each_depth_path(name, cfg, causal, path):
     """Both depth paths (CUDA-core fold, dense tensor-core depth blocks) on every case;
-    the dense path refuses groups that do not divide 128."""
+    the dense path refuses groups that do not divide 128 or exceed 32 (a row sees only its
+    warp's 32 columns of a depth block)."""
     x = gpu_inputs(cfg, seed_base=100 + SMALL.index((name, cfg, causal)))
     scale = 1.0 / math.sqrt(cfg["d"])
     G = cfg["Hq"] // cfg["Hkv"]
-    if path == 2 and 128 % G != 0:
+    if path == 2 and (128 % G != 0 or G > 32):
         with pytest.raises(moda.ModaError) as e:
             moda.forward(x["q"], x["k"], x["v"], x["kd"], x["vd"], scale, causal,
                          depth_path=path)
