@@ -33,7 +33,8 @@ namespace {
 
 constexpr int kDecKeys = 128;      // keys per block
 constexpr int kDecStages = 3;      // K+V ring stages
-constexpr int kDecThreads = 160;   // warps 0-3 compute, warp 4 TMA producer
+constexpr int kDecCompute = 256;   // compute threads (warps 0-7)
+constexpr int kDecThreads = kDecCompute + 32;  // and warp 8, the TMA producer
 constexpr int kDecMaxG = 16;
 constexpr float kLog2eDec = 1.4426950408889634f;
 constexpr float kLn2Dec = 0.6931471805599453f;
@@ -44,11 +45,13 @@ struct DecCfg {
   static constexpr int kTile = kRegions * 16384;      // 128 keys x D bf16, 128B-swizzled
   static constexpr int kStage = 2 * kTile;            // K then V
   static constexpr int kOffQ = kDecStages * kStage;   // [G][D] bf16, row-major
-  static constexpr int kOffP = kOffQ + kDecMaxG * D * 2;           // [G][128] fp32
-  static constexpr int kOffRed = kOffP + kDecMaxG * kDecKeys * 4;  // [2][4][G] fp32
-  static constexpr int kOffAcc = kOffRed + 2 * 4 * kDecMaxG * 4;   // [G][D] fp32 (D = 64)
-  static constexpr int kOffBar = kOffAcc + (D == 64 ? kDecMaxG * D * 4 : 0);
+  static constexpr int kOffP = kOffQ + kDecMaxG * D * 2;  // [8 warps][G][16 keys] fp32
+  static constexpr int kOffBar = kOffP + 8 * kDecMaxG * 16 * 4;
   static constexpr int kSmemBytes = 1024 + kOffBar + 128;
+  static constexpr int kPairs = D / 64;  // column pairs per thread in the P.V phase
+  // the warps' states, [8][G][D] accumulators and [8][G][2] (m, l), reuse the ring after
+  // the last block
+  static_assert(8 * kDecMaxG * (D + 2) * 4 <= kDecStages * kStage, "ring too small");
 };
 
 struct DecArgs {
@@ -75,7 +78,23 @@ __device__ __forceinline__ uint32_t dec_sw(int r, int c) {
   return uint32_t(r) * 128u + ((uint32_t(c) ^ (uint32_t(r) & 7u)) << 4);
 }
 
+__device__ __forceinline__ uint32_t lds_b32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
 // GM: group size rounded up to a power of two (loop bound); kExact: G == GM.
+// Warp 8 streams each block's K and V tiles through the TMA ring.  Compute warp w owns keys
+// [16w, 16w + 16) of every block and keeps its own online-softmax state (running max m,
+// normaliser l, fp32 accumulator) for the G heads over the whole split, so the eight
+// warps never wait for each other within a block:
+//   logits: two lanes per key, each over half the head dimension (q from shared memory,
+//           bf16 x bf16 products accumulated in fp32), finished with one shuffle;
+//   P.V:    each lane owns column pairs (2 lane, 2 lane + 64 for D = 128) and reads V as
+//           packed bf16 pairs, with packed f32x2 FMAs, over the warp's 16 keys.
+// After the last block the eight states are merged exactly (each rescaled to the largest
+// max) and written to the workspace.
 template <int D, int GM, bool kExact>
 __global__ void __launch_bounds__(kDecThreads, 1)
     moda_decode_split_kernel(const __grid_constant__ CUtensorMap tmK,
@@ -90,8 +109,6 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   DecBars* bars = reinterpret_cast<DecBars*>(smem + Cfg::kOffBar);
   volatile int* abort_flag = &bars->abort;
   auto bar = [&](uint64_t& b) { return smem_u32(&b); };
-  float* P = reinterpret_cast<float*>(smem + Cfg::kOffP);
-  float* red = reinterpret_cast<float*>(smem + Cfg::kOffRed);
 
   const int bg = blockIdx.x / a.nsplit;
   const int split = blockIdx.x - bg * a.nsplit;
@@ -106,12 +123,12 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kDecStages; ++s) {
       mbar_init(bar(bars->full[s]), 1);
-      mbar_init(bar(bars->empty[s]), 128);
+      mbar_init(bar(bars->empty[s]), kDecCompute);
     }
     bars->abort = 0;
     fence_barrier_init();
   }
-  // the G query rows of this group (bf16) into shared memory
+  // the G query rows of this chunk (bf16) into shared memory
   const int b = bg / a.Hkv, g = bg - (bg / a.Hkv) * a.Hkv;
   for (int i = threadIdx.x; i < G * D / 8; i += kDecThreads) {
     const int h = i / (D / 8), c = i - h * (D / 8);
@@ -120,15 +137,16 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   }
   __syncthreads();
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (elect_one()) {
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       for (int i = 0; i < nblk; ++i) {
         const int s = i % kDecStages;
-        if (i >= kDecStages)
-          mbar_wait(bar(bars->empty[s]), ((i / kDecStages) - 1) & 1, abort_flag);
+        if (i >= kDecStages &&
+            !mbar_wait(bar(bars->empty[s]), ((i / kDecStages) - 1) & 1, abort_flag))
+          break;
         mbar_expect_tx(bar(bars->full[s]), Cfg::kStage);
         const bool dep = i < ndep;
         const int row0 = dep ? i * kDecKeys : (sb0 + i - ndep) * kDecKeys;
@@ -145,17 +163,22 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     return;  // the producer warp takes no part in the compute warps' barriers
   }
 
-  // ------------------------------------------------------------ compute warps 0-3
-  const int tid = threadIdx.x;              // key of the block (logit phase)
-  constexpr int KG = 128 / D;               // key groups in the P.V phase
-  const int dcol = tid % D, kg = tid / D;   // head-dimension column, key group
-  const int lane = tid & 31;
-  float m[GM], l[GM], acc[GM];
+  // ------------------------------------------------------------ compute warps 0-7
+  const int lane = threadIdx.x & 31;
+  const int kl = lane >> 1, part = lane & 1;  // the lane's key among the warp's 16, half of D
+  const int key = 16 * warp + kl;             // key of the block
+  constexpr int kChunks = D / 16;             // 16-byte chunks of a lane's half row
+  constexpr int NP = Cfg::kPairs;
+  const uint32_t pw = s0 + Cfg::kOffP + uint32_t(warp * kDecMaxG * 16 * 4);  // [G][16] fp32
+  float* Pw = reinterpret_cast<float*>(smem + Cfg::kOffP) + warp * kDecMaxG * 16;
+  float m[GM], l[GM];
+  float2 acc[GM][NP];
 #pragma unroll
   for (int h = 0; h < GM; ++h) {
     m[h] = -INFINITY;
     l[h] = 0.f;
-    acc[h] = 0.f;
+#pragma unroll
+    for (int j = 0; j < NP; ++j) acc[h][j] = make_float2(0.f, 0.f);
   }
   for (int i = 0; i < nblk; ++i) {
     const int s = i % kDecStages;
@@ -163,115 +186,116 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     const uint32_t kst = s0 + uint32_t(s) * Cfg::kStage;
     const uint32_t vst = kst + Cfg::kTile;
     const bool dep = i < ndep;
-    const int kabs = (dep ? i : sb0 + i - ndep) * kDecKeys + tid;
+    const int kabs = (dep ? i : sb0 + i - ndep) * kDecKeys + key;
     const bool kvalid = kabs < (dep ? a.L : a.S);
-    // logits of this key for the G heads
+    // logits of this key for the G heads (this lane's half of the dot products)
     float y[GM];
 #pragma unroll
     for (int h = 0; h < GM; ++h) y[h] = 0.f;
 #pragma unroll
-    for (int rg = 0; rg < Cfg::kRegions; ++rg) {
+    for (int cc = 0; cc < kChunks; ++cc) {
+      const int ch = part * kChunks + cc;  // 16-byte chunk of the row
+      const uint4 kw = lds128(kst + (ch / 8) * 16384 + dec_sw(key, ch % 8));
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint4 kw = lds128(kst + rg * 16384 + dec_sw(tid, c));
-#pragma unroll
-        for (int h = 0; h < GM; ++h)
-          if (h < G)
-            y[h] = dot8_bf16(lds128(s0 + Cfg::kOffQ + uint32_t((h * D + rg * 64 + c * 8) * 2)),
-                             kw, y[h]);
-      }
+      for (int h = 0; h < GM; ++h)
+        if (h < G)
+          y[h] = dot8_bf16(lds128(s0 + Cfg::kOffQ + uint32_t((h * D + ch * 8) * 2)), kw, y[h]);
     }
-    // block max per head: warp max, then across the four warps
+    // the warp's online-softmax step over its 16 keys
 #pragma unroll
     for (int h = 0; h < GM; ++h) {
       if (h < G) {
-        y[h] = kvalid ? y[h] * a.scale_log2 : -INFINITY;
-        float v = y[h];
+        y[h] += __shfl_xor_sync(0xffffffffu, y[h], 1);
+        const float yv = kvalid ? y[h] * a.scale_log2 : -INFINITY;
+        float bmax = yv;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-        if (lane == 0) red[warp * kDecMaxG + h] = v;
-      }
-    }
-    named_bar_sync(1, 128);
-    float alpha[GM];
-#pragma unroll
-    for (int h = 0; h < GM; ++h) {
-      alpha[h] = 1.f;
-      if (h < G) {
-        const float bmax = fmaxf(fmaxf(red[h], red[kDecMaxG + h]),
-                                 fmaxf(red[2 * kDecMaxG + h], red[3 * kDecMaxG + h]));
+        for (int o = 16; o > 1; o >>= 1) bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, o));
         const float m_new = fmaxf(m[h], bmax);
         const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-        alpha[h] = ex2(m[h] - m_use);
-        const float p = ex2(y[h] - m_use);
-        P[h * kDecKeys + tid] = p;
-        float v = p;
+        const float alpha = ex2(m[h] - m_use);
+        const float p = ex2(yv - m_use);
+        if (part == 0) Pw[h * 16 + kl] = p;
+        float sum = part == 0 ? p : 0.f;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == 0) red[(4 + warp) * kDecMaxG + h] = v;
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        l[h] = l[h] * alpha + sum;
         m[h] = m_new;
-      }
-    }
-    named_bar_sync(1, 128);
-    // P.V: column dcol over this thread's key group
 #pragma unroll
-    for (int h = 0; h < GM; ++h) {
-      if (h < G) {
-        const float bsum = (red[4 * kDecMaxG + h] + red[5 * kDecMaxG + h]) +
-                           (red[6 * kDecMaxG + h] + red[7 * kDecMaxG + h]);
-        l[h] = l[h] * alpha[h] + bsum;
-        acc[h] *= alpha[h];
+        for (int j = 0; j < NP; ++j) acc[h][j] = fmul2(acc[h][j], make_float2(alpha, alpha));
       }
     }
-    {
-      const int rg = dcol / 64, col = dcol % 64;
-      const uint32_t vcol = vst + rg * 16384 + uint32_t(col % 8) * 2;
-      const uint32_t pbase = s0 + Cfg::kOffP;
-      constexpr int NK = kDecKeys / KG;  // keys of this thread's group
+    __syncwarp();  // P of the warp's keys written
+    // P.V over the warp's 16 keys: column pairs 2 lane + 64 j
 #pragma unroll 2
-      for (int k4 = 0; k4 < NK; k4 += 4) {
-        const int k = kg * NK + k4;
-        float vv[4];
+    for (int k4 = 0; k4 < 16; k4 += 4) {
+      float2 vv[4][NP];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) vv[u] = bf16lo(lds_u16(vcol + dec_sw(k + u, col / 8)));
+      for (int u = 0; u < 4; ++u)
 #pragma unroll
-        for (int h = 0; h < GM; ++h) {
-          if (h < G) {
-            const uint4 pw = lds128(pbase + uint32_t(h * kDecKeys + k) * 4u);
-            acc[h] = fmaf(__uint_as_float(pw.x), vv[0], acc[h]);
-            acc[h] = fmaf(__uint_as_float(pw.y), vv[1], acc[h]);
-            acc[h] = fmaf(__uint_as_float(pw.z), vv[2], acc[h]);
-            acc[h] = fmaf(__uint_as_float(pw.w), vv[3], acc[h]);
-          }
+        for (int j = 0; j < NP; ++j) {
+          const int col = 2 * lane + 64 * j;
+          const uint32_t w = lds_b32(vst + uint32_t((col / 64) * 16384 + (col % 8) * 2) +
+                                     dec_sw(16 * warp + k4 + u, (col % 64) / 8));
+          vv[u][j] = make_float2(bf16lo(w), bf16hi(w));
+        }
+#pragma unroll
+      for (int h = 0; h < GM; ++h) {
+        if (h < G) {
+          const uint4 pq = lds128(pw + uint32_t((h * 16 + k4) * 4));
+          const float pk[4] = {__uint_as_float(pq.x), __uint_as_float(pq.y),
+                               __uint_as_float(pq.z), __uint_as_float(pq.w)};
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int j = 0; j < NP; ++j)
+              acc[h][j] = ffma2(make_float2(pk[u], pk[u]), vv[u][j], acc[h][j]);
         }
       }
     }
-    named_bar_sync(1, 128);  // P and the reduction slots are rewritten by the next block
+    __syncwarp();  // the warp's P is rewritten by the next block
     mbar_arrive(bar(bars->empty[s]));
   }
 
-  // partial results of this split
-  float* accs = reinterpret_cast<float*>(smem + Cfg::kOffAcc);
-  if (KG == 2) {
-    if (kg == 1) {
+  // merge the eight warps' states in the ring's memory: free once every warp has finished
+  // reading its last block (every block's loads were waited for)
+  named_bar_sync(1, kDecCompute);
+  float* wacc = reinterpret_cast<float*>(smem);          // [8][G][D]
+  float* wml = wacc + 8 * kDecMaxG * D;                   // [8][G][2]
 #pragma unroll
-      for (int h = 0; h < GM; ++h)
-        if (h < G) accs[h * D + dcol] = acc[h];
-    }
-    named_bar_sync(1, 128);
-  }
-  if (kg == 0) {
-    const size_t base = (size_t(bg) * a.nsplit + split) * a.Gfull + a.head0;
+  for (int h = 0; h < GM; ++h) {
+    if (h < G) {
 #pragma unroll
-    for (int h = 0; h < GM; ++h) {
-      if (h < G) {
-        const float v = (KG == 2) ? acc[h] + accs[h * D + dcol] : acc[h];
-        a.ws_acc[(base + h) * D + dcol] = v;
-        if (dcol == 0) {
-          a.ws_ml[(base + h) * 2] = m[h];
-          a.ws_ml[(base + h) * 2 + 1] = l[h];
-        }
+      for (int j = 0; j < NP; ++j)
+        *reinterpret_cast<float2*>(wacc + (warp * kDecMaxG + h) * D + 2 * lane + 64 * j) =
+            acc[h][j];
+      if (lane == 0) {
+        wml[(warp * kDecMaxG + h) * 2] = m[h];
+        wml[(warp * kDecMaxG + h) * 2 + 1] = l[h];
       }
+    }
+  }
+  named_bar_sync(1, kDecCompute);
+  const size_t base = (size_t(bg) * a.nsplit + split) * a.Gfull + a.head0;
+  for (int e = threadIdx.x; e < G * (D / 2); e += kDecCompute) {
+    const int h = e / (D / 2), col = 2 * (e - h * (D / 2));
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) M = fmaxf(M, wml[(w * kDecMaxG + h) * 2]);
+    const float Mu = (M == -INFINITY) ? 0.f : M;
+    float2 v = make_float2(0.f, 0.f);
+    float lsum = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      const float f = ex2(wml[(w * kDecMaxG + h) * 2] - Mu);
+      const float2 x = *reinterpret_cast<const float2*>(wacc + (w * kDecMaxG + h) * D + col);
+      v.x = fmaf(f, x.x, v.x);
+      v.y = fmaf(f, x.y, v.y);
+      lsum = fmaf(f, wml[(w * kDecMaxG + h) * 2 + 1], lsum);
+    }
+    *reinterpret_cast<float2*>(a.ws_acc + (base + h) * D + col) = v;
+    if (col == 0) {
+      a.ws_ml[(base + h) * 2] = M;
+      a.ws_ml[(base + h) * 2 + 1] = lsum;
     }
   }
 }
@@ -414,16 +438,34 @@ cudaError_t launch_decode_d(const Problem& p, const DecodeSplit& sp, const void*
 }  // namespace
 
 DecodeSplit decode_split(const Problem& p) {
+  // One CTA (about 206 KB of shared memory) per SM of a B200 (148 SMs).  The split count
+  // is chosen so that the CTAs fill whole waves: among splits of up to 8 waves the one with
+  // the least idle SM time, each wave beyond the first charged 1% (every CTA refills its
+  // load pipeline).  The choice depends on the sizes alone, so the workspace size is a
+  // function of the sizes.
+  constexpr int kSMs = 148, kMaxWaves = 8;
   DecodeSplit sp;
   const int nseq = (p.T + kDecKeys - 1) / kDecKeys;
-  const int bg = p.B * p.Hkv;
-  // at most one wave: one CTA (211 KB of shared memory) per SM of a B200 (148 SMs); a
-  // fixed target keeps the workspace size a function of the sizes alone (nsplit <= 148)
-  int want = 148 / bg;
-  if (want < 1) want = 1;
-  if (want > nseq) want = nseq;
-  sp.blocks_per_split = (nseq + want - 1) / want;
-  sp.nsplit = (nseq + sp.blocks_per_split - 1) / sp.blocks_per_split;  // none empty
+  const long long bg = (long long)p.B * p.Hkv;
+  int best_ns = 1;
+  double best_eff = -1.0;
+  long long best_waves = 0;
+  const int max_ns = min(nseq, kDecMaxSplit);
+  for (int want = 1; want <= max_ns; ++want) {
+    const int bps = (nseq + want - 1) / want;
+    const int ns = (nseq + bps - 1) / bps;  // no empty split
+    const long long ctas = bg * ns;
+    const long long waves = (ctas + kSMs - 1) / kSMs;
+    if (waves > kMaxWaves && want > 1) break;
+    const double eff = double(ctas) / double(waves * kSMs) - 0.01 * double(waves - 1);
+    if (eff > best_eff + 1e-9 || (eff > best_eff - 1e-9 && waves < best_waves)) {
+      best_eff = eff;
+      best_ns = ns;
+      best_waves = waves;
+    }
+  }
+  sp.blocks_per_split = (nseq + best_ns - 1) / best_ns;
+  sp.nsplit = (nseq + sp.blocks_per_split - 1) / sp.blocks_per_split;
   return sp;
 }
 
