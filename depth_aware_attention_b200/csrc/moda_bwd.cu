@@ -72,6 +72,29 @@ struct BwdDepthArgs {
 // time.  The G query rows of the token keep q and dO unpacked to fp32 in registers when
 // GM <= 4, else in shared memory (bf16); the dq partial sums of up to GM heads stay in
 // registers.
+// Butterfly reduce-scatter of the 2*GM partial dot products (y_0..y_{GM-1}, then
+// p_0..p_{GM-1}) over the NT lanes of a token slot.  In each round a lane sends half of its
+// values to the partner lane (xor o), keeps the other half and adds the partner's copy, so
+// the count halves; once a lane holds one value the remaining rounds are plain all-reduce
+// steps.  The first round splits the y values from the p values, so the partner across
+// the first bit holds p_h for the same heads h.  bf_count: values a lane holds at the end;
+// bf_head(lane, i): the head of its i-th value (lanes whose first bit is 0 hold y values).
+template <int NT, int NV>
+__host__ __device__ constexpr int bf_count() {
+  int c = NV;
+  for (int o = NT / 2; o > 0 && c > 1; o >>= 1) c /= 2;
+  return c;
+}
+template <int NT, int NV>
+__host__ __device__ constexpr int bf_head(int lane, int i) {
+  int c = NV, base = 0;
+  for (int o = NT / 2; o > 0 && c > 1; o >>= 1) {
+    c /= 2;
+    if (lane & o) base += c;
+  }
+  return (base + i) % (NV / 2);
+}
+
 template <int D, int GM>
 // (GM <= 4: at most 168 registers, three CTAs per SM; measured faster than 188 registers
 // and two CTAs)
@@ -155,10 +178,19 @@ __global__ void __launch_bounds__(kDepthThreads, GM <= 4 ? 3 : 1)
     if (a.exact_rows) {
       // D_h = sum_j P_hj <dO_h, vd_j> with P_hj = 2^(y_hj * scale * log2(e) - lse_h * log2(e)),
       // the same weights the gradient loop below recomputes; kd and vd are read once more.
-      float dsum[GM];
+      // The dot products are finished by the butterfly of the gradient loop (below), each
+      // lane summing P * p for the heads it ends up holding; one broadcast per token.
+      constexpr int kNV0 = 2 * GM, kBC0 = bf_count<NT, kNV0>();
+      float lse_mine[kBC0], dsum[kBC0];
 #pragma unroll
-      for (int h = 0; h < GM; ++h) dsum[h] = 0.f;
-#pragma unroll 4
+      for (int i = 0; i < kBC0; ++i) {
+        lse_mine[i] = dsum[i] = 0.f;
+#pragma unroll
+        for (int h = 0; h < GM; ++h)
+          if (h == bf_head<NT, kNV0>(cs, i)) lse_mine[i] = lse2[h];
+      }
+      const bool is_y = (cs & (NT / 2)) == 0;
+#pragma unroll 2
       for (long long j = 0; j < L; ++j) {
         uint4 kw = make_uint4(0, 0, 0, 0), vw = make_uint4(0, 0, 0, 0);
         if (valid) {
@@ -168,10 +200,10 @@ __global__ void __launch_bounds__(kDepthThreads, GM <= 4 ? 3 : 1)
         float kf[8], vf[8];
         unpack8(kw, kf);
         unpack8(vw, vf);
-        float y[GM], p[GM];
+        float bv[kNV0];
 #pragma unroll
         for (int h = 0; h < GM; ++h) {
-          y[h] = p[h] = 0.f;
+          bv[h] = bv[GM + h] = 0.f;
           if (h < G) {
             float qf[8], df[8];
             if constexpr (kReg) {
@@ -186,32 +218,64 @@ __global__ void __launch_bounds__(kDepthThreads, GM <= 4 ? 3 : 1)
             }
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-              y[h] = fmaf(qf[e], kf[e], y[h]);
-              p[h] = fmaf(df[e], vf[e], p[h]);
+              bv[h] = fmaf(qf[e], kf[e], bv[h]);
+              bv[GM + h] = fmaf(df[e], vf[e], bv[GM + h]);
             }
           }
         }
+        int c = kNV0;
 #pragma unroll
         for (int o = NT / 2; o > 0; o >>= 1) {
+          if (c > 1) {
+            const bool up = (cs & o) != 0;
 #pragma unroll
-          for (int h = 0; h < GM; ++h) {
-            if (h < G) {
-              y[h] += __shfl_xor_sync(0xffffffffu, y[h], o);
-              p[h] += __shfl_xor_sync(0xffffffffu, p[h], o);
+            for (int i = 0; i < kNV0 / 2; ++i) {
+              if (i < c / 2) {
+                const float send = up ? bv[i] : bv[c / 2 + i];
+                const float keep = up ? bv[c / 2 + i] : bv[i];
+                bv[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+              }
             }
+            c /= 2;
+          } else {
+            bv[0] += __shfl_xor_sync(0xffffffffu, bv[0], o);
           }
         }
 #pragma unroll
-        for (int h = 0; h < GM; ++h)
-          if (h < G) dsum[h] = fmaf(ex2(y[h] * a.scale_log2 - lse2[h]), p[h], dsum[h]);
-      }
-#pragma unroll
-      for (int h = 0; h < GM; ++h) {
-        if (h < G) {
-          drw[h] = dsum[h];
-          if (valid && cs == 0) a.drow[(bg * a.Gfull + a.head0 + h) * a.T + t] = dsum[h];
+        for (int i = 0; i < kBC0; ++i) {
+          const float other = __shfl_xor_sync(0xffffffffu, bv[i], NT / 2);
+          const float yy = is_y ? bv[i] : other, pp = is_y ? other : bv[i];
+          dsum[i] = fmaf(ex2(yy * a.scale_log2 - lse_mine[i]), pp, dsum[i]);
         }
       }
+      const int slot0 = (threadIdx.x & 31) & ~(NT - 1);
+#pragma unroll
+      for (int h = 0; h < GM; ++h) {
+        int src = 0, si = 0;
+#pragma unroll
+        for (int l2 = NT / 2 - 1; l2 >= 0; --l2)
+#pragma unroll
+          for (int i = 0; i < kBC0; ++i)
+            if (bf_head<NT, kNV0>(l2, i) == h) { src = l2; si = i; }
+        const float dh = __shfl_sync(0xffffffffu, dsum[si], slot0 + src);
+        if (h < G) {
+          drw[h] = dh;
+          if (valid && cs == 0) a.drow[(bg * a.Gfull + a.head0 + h) * a.T + t] = dh;
+        }
+      }
+    }
+    // (after the exact row terms above, when they apply) row terms of the heads whose P and dS this lane computes (see the butterfly below)
+    constexpr int kNV = 2 * GM, kBC = bf_count<NT, kNV>();
+    float my_lse2[kBC], my_drw[kBC];
+#pragma unroll
+    for (int i = 0; i < kBC; ++i) {
+      my_lse2[i] = my_drw[i] = 0.f;
+#pragma unroll
+      for (int h = 0; h < GM; ++h)
+        if (h == bf_head<NT, kNV>(cs, i) % GM) {
+          my_lse2[i] = lse2[h];
+          my_drw[i] = drw[h];
+        }
     }
     const long long nbat = (L + kU - 1) / kU;
     // batch b's copies (an empty group past the last batch keeps the group count uniform)
@@ -278,24 +342,62 @@ __global__ void __launch_bounds__(kDepthThreads, GM <= 4 ? 3 : 1)
           p[h] = p2.x + p2.y;
         }
       }
+      // finish the token's dot products: butterfly reduce-scatter over the slot's lanes
+      float bv[kNV];
 #pragma unroll
-      for (int o = NT / 2; o > 0; o >>= 1) {
+      for (int h = 0; h < GM; ++h) {
+        bv[h] = y[h];
+        bv[GM + h] = p[h];
+      }
+      {
+        int c = kNV;
 #pragma unroll
-        for (int h = 0; h < GM; ++h) {
-          if (h < G) {
-            y[h] += __shfl_xor_sync(0xffffffffu, y[h], o);
-            p[h] += __shfl_xor_sync(0xffffffffu, p[h], o);
+        for (int o = NT / 2; o > 0; o >>= 1) {
+          if (c > 1) {
+            const bool up = (cs & o) != 0;
+#pragma unroll
+            for (int i = 0; i < kNV / 2; ++i) {
+              if (i < c / 2) {
+                const float send = up ? bv[i] : bv[c / 2 + i];
+                const float keep = up ? bv[c / 2 + i] : bv[i];
+                bv[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+              }
+            }
+            c /= 2;
+          } else {
+            bv[0] += __shfl_xor_sync(0xffffffffu, bv[0], o);
           }
         }
       }
+      // bv[0..kBC) are now full sums; the partner across the first bit holds the other
+      // kind (y or p) of the same heads: P and dS of those heads, then broadcast
+      float bP[kBC], bS[kBC];
+      {
+        const bool is_y = (cs & (NT / 2)) == 0;
+#pragma unroll
+        for (int i = 0; i < kBC; ++i) {
+          const float other = __shfl_xor_sync(0xffffffffu, bv[i], NT / 2);
+          const float yy = is_y ? bv[i] : other, pp = is_y ? other : bv[i];
+          bP[i] = ex2(yy * a.scale_log2 - my_lse2[i]);
+          bS[i] = bP[i] * (pp - my_drw[i]);
+        }
+      }
+      const int slot0 = (threadIdx.x & 31) & ~(NT - 1);  // first lane of this token slot
       float dv[8], dk[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) dv[e] = dk[e] = 0.f;
 #pragma unroll
       for (int h = 0; h < GM; ++h) {
         if (h < G) {
-          const float P = ex2(y[h] * a.scale_log2 - lse2[h]);
-          const float dS = P * (p[h] - drw[h]);
+          // the value of head h sits in slot i of the y lanes l with bf_head(l, i) == h
+          int src = 0, si = 0;
+#pragma unroll
+          for (int l2 = NT / 2 - 1; l2 >= 0; --l2)
+#pragma unroll
+            for (int i = 0; i < kBC; ++i)
+              if (bf_head<NT, kNV>(l2, i) == h) { src = l2; si = i; }
+          const float P = __shfl_sync(0xffffffffu, bP[si], slot0 + src);
+          const float dS = __shfl_sync(0xffffffffu, bS[si], slot0 + src);
           float qf[8], df[8];
           if constexpr (kReg) {
 #pragma unroll
