@@ -10,8 +10,9 @@
 //
 // Three launches:
 //  1. moda_bwd_depth_kernel (token-major, CUDA cores, bandwidth-bound): per token of one
-//     KV group, D for the G query rows, dkd/dvd for the token's L depth entries, and the
-//     depth share of dq, which initialises the fp32 dq accumulator.  Threads split the
+//     KV group, D for the G query rows (with -lse*log2e, as the per-tile records the d =
+//     128 sequence kernel loads), dkd/dvd for the token's L depth entries, and the depth
+//     share of dq, which initialises the fp32 dq accumulator.  Threads split the
 //     head dimension into 16-byte column chunks; dot products are finished with warp
 //     shuffles, so every depth byte is read from HBM once, with 16-byte coalesced loads.
 //  2. moda_bwd_seq_kernel (KV-block-major, tcgen05): one CTA owns 128 sequence keys of
@@ -27,6 +28,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math.h>
+
+#include <type_traits>
 
 #include "moda_internal.h"
 #include "sm100.cuh"
@@ -50,7 +53,13 @@ struct BwdDepthArgs {
   const float* lse;
   __nv_bfloat16 *dkd, *dvd;
   float* dqacc;  // [B][Hq][T][D] fp32, written (not accumulated) here
-  float* drow;   // [B][Hq][T] fp32: D = <dO, out>
+  float* drow;   // [B][Hq][T] fp32: D = <dO, out> (null: not written)
+  // Row terms of each query tile of the d = 128 sequence kernel, which loads them with one
+  // bulk copy per tile: [B*Hkv][nqt][2][128] fp32, record r of tile qt = tile row
+  // (t - qt*TQ)*G + head; first -lse*log2(e), then -D*scale.  Rows past the last token or
+  // past TQ*G get -inf and 0 (P = 0, dS = 0).  Null: not written.
+  float* rt;
+  int TQ, nqt;
   long long ntok;  // B * Hkv * T
   int T, L, G;
   // 1 (depth-only attention): the row terms are formed from the depth logits themselves,
@@ -127,6 +136,9 @@ __global__ void __launch_bounds__(kDepthThreads, GM <= 4 ? 3 : 1)
     const long long tkc = valid ? tk : a.ntok - 1;
     const long long bg = tkc / a.T;
     const int t = int(tkc - bg * a.T);
+    const int qt = a.rt ? t / a.TQ : 0, tq = t - qt * a.TQ;
+    float* const rt_tile = a.rt ? a.rt + ((bg * a.nqt + qt) << 8) : nullptr;
+    const int r0 = tq * a.Gfull + a.head0;  // tile row of this chunk's head 0
 
     float lse2[GM], drw[GM];
     float qreg[kReg ? GM : 1][8], dreg[kReg ? GM : 1][8];
@@ -163,7 +175,19 @@ __global__ void __launch_bounds__(kDepthThreads, GM <= 4 ? 3 : 1)
 #pragma unroll
         for (int o = NT / 2; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
         drw[h] = part;
-        if (valid && cs == 0) a.drow[row] = part;
+        if (valid && cs == 0 && a.drow) a.drow[row] = part;
+        if (valid && cs == (h & (NT - 1)) && a.rt) {
+          rt_tile[r0 + h] = -lse2[h];
+          rt_tile[128 + r0 + h] = -part * a.scale;
+        }
+      }
+    }
+    // the last token of a tile fills the tile's records past its rows (once, in the first
+    // head chunk)
+    if (valid && a.rt && a.head0 == 0 && (tq == a.TQ - 1 || t == a.T - 1)) {
+      for (int r = r0 + a.Gfull + cs; r < 128; r += NT) {
+        rt_tile[r] = -INFINITY;
+        rt_tile[128 + r] = 0.f;
       }
     }
     __syncwarp();
@@ -260,7 +284,7 @@ __global__ void __launch_bounds__(kDepthThreads, GM <= 4 ? 3 : 1)
         const float dh = __shfl_sync(0xffffffffu, dsum[si], slot0 + src);
         if (h < G) {
           drw[h] = dh;
-          if (valid && cs == 0) a.drow[(bg * a.Gfull + a.head0 + h) * a.T + t] = dh;
+          if (valid && cs == 0 && a.drow) a.drow[(bg * a.Gfull + a.head0 + h) * a.T + t] = dh;
         }
       }
     }
@@ -501,7 +525,8 @@ struct SeqBars {
 struct SeqArgs {
   __nv_bfloat16 *dk, *dv;
   float* dqacc;
-  const float *lse, *drow;
+  const float *lse, *drow;  // d = 64 kernel: [B][Hq][T] each
+  const float* rt;          // d = 128 kernel: tiled row terms (BwdDepthArgs::rt)
   int Hkv, T, G, TQ, nqt, BG, causal;
   float scale, scale_log2;
 };
@@ -864,31 +889,38 @@ __global__ void __launch_bounds__(kSeqThreads, 1)
 // either way (TMA bulk reduce-add or per-thread reductions), so the readout is bound by
 // that outbound rate; reductions from registers keep it off the tensor pipe's critical
 // path: no shared-memory staging, no wait for the TMA unit before TMEM is released.
+// Each tile's row terms (-lse*log2e, -D*scale per row) arrive with its Q in one bulk copy
+// from records the depth kernel wrote, so the P/dS warps issue no global loads.
 //
-// Tensor-core issue order per tile i (primes: tile i+1):
-//   [pds0] dV0 dK0 dQ0 dP0' [dqfree0] S0'   [pds1] dV1 dK1 dQ1 dP1' [dqfree1] S1'
-// so that the softmax warps work on half 0 of tile i+1 while the tensor cores run the
-// products of half 1 of tile i (and the reverse), instead of waiting on each other.
-constexpr int kSeqHThreads = 448;  // warps 0-7 P/dS, 8-11 dQ, 12 TMA, 13 tcgen05
+// Tensor-core issue order of half h's issuer per tile i (primes: tile i+1; brackets: the
+// barrier waited for):
+//   [pds_h] dV_h dK_h dQ_h dP_h'  [dqfree_h] S_h'
+// The two issuers share the tensor pipe, so one half's products run while the P/dS warps
+// work on the other half, and neither issuer waits behind the other half's barriers.
+// warps 0-7 P/dS, 8-11 dQ, 12 TMA, 13 and 14 tcgen05 issuers of halves 0 and 1
+constexpr int kSeqHThreads = 480;
+constexpr uint32_t kRowTermBytes = 2 * 128 * 4;  // one tile's -lse*log2e and -D records
 
 struct SeqHBars {
   uint64_t kv_full;
   uint64_t q_full[2], q_empty[2];
   uint64_t do_full[2], do_empty[2];
   uint64_t s_full[2], dp_full[2], pds_full[2], dq_full[2], dq_free[2];
-  uint64_t kv_done;
+  uint64_t kv_done, acc_zero;
   uint32_t tmem_base;
   int abort;
   int lo_tile[2];  // half h of tile i needs its lo passes iff lo_tile[h] == i + 1
 };
 
 // The lo halves of P and dS (x - bf16(x)) enter the dV and dK products only for the half
-// tiles where some of them exceeds this size.  A dropped lo value is at most 2^-9 of its
-// element, so below it the element is small (P or dS under about 2^-6), and a half tile's
-// 64 such terms move a dV or dK entry by far less than the output's own bf16 rounding.
-// Large weights (short sequences, the first rows of long ones) keep both passes.
+// tiles where some P or |dS| exceeds kLoKeep.  A lo value is at most 2^-8 of its element
+// (bf16 keeps 8 significant bits), so every lo value dropped is under 2^-15, and a half
+// tile's 64 such terms move a dV or dK entry by far less than the output's own bf16
+// rounding.  Large weights (short sequences, the first rows of long ones) keep both passes.
+// A warp computes the lo halves of its elements only when one of them is that large, and
+// writes zeros otherwise, for the half tiles whose lo passes another warp asked for.
 #ifndef MODA_BWD_LO_KEEP
-#define MODA_BWD_LO_KEEP 3.0517578125e-05f  // 2^-15
+#define MODA_BWD_LO_KEEP 0.0078125f  // 2^-7
 #endif
 constexpr float kLoKeep = MODA_BWD_LO_KEEP;
 
@@ -910,7 +942,7 @@ __device__ __forceinline__ void dq_readout(const SeqArgs& a, SeqHBars* bars, uin
     const int ntok = min(a.TQ, a.T - t0q);  // valid tokens of this tile
 #pragma unroll 1
     for (int h = 0; h < 2; ++h) {
-      const uint32_t tA = tmem + uint32_t(64 * h);
+      const uint32_t tA = tmem + uint32_t(64 * h);  // region A_h
       mbar_wait(smem_u32(&bars->dq_full[h]), i & 1, abort_flag);
       tc_fence_after();
       uint32_t o[64];
@@ -968,7 +1000,8 @@ __global__ void __launch_bounds__(kSeqHThreads, 1)
   const uint32_t sK = s0 + Cfg::kOffK, sV = s0 + Cfg::kOffV, sDS = s0 + Cfg::kOffDS;
   auto sQ = [&](int st) { return s0 + Cfg::kOffQ + uint32_t(st) * Cfg::kTile; };
   auto sDO = [&](int st) { return s0 + Cfg::kOffDO + uint32_t(st) * Cfg::kTile; };
-  float* ld_s = reinterpret_cast<float*>(smem + Cfg::kOffLD);
+  auto sLD = [&](int st) { return s0 + Cfg::kOffLD + uint32_t(st) * kRowTermBytes; };
+  const float* ld_s = reinterpret_cast<const float*>(smem + Cfg::kOffLD);
   SeqHBars* bars = reinterpret_cast<SeqHBars*>(smem + Cfg::kOffBar);
   volatile int* abort_flag = &bars->abort;
   auto bar = [&](uint64_t& b) { return smem_u32(&b); };
@@ -984,16 +1017,17 @@ __global__ void __launch_bounds__(kSeqHThreads, 1)
     mbar_init(bar(bars->kv_full), 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(bars->q_full[i]), 1);
-      mbar_init(bar(bars->q_empty[i]), 1);
+      mbar_init(bar(bars->q_empty[i]), 2);  // one commit from each issuer
       mbar_init(bar(bars->do_full[i]), 1);
-      mbar_init(bar(bars->do_empty[i]), 1);
+      mbar_init(bar(bars->do_empty[i]), 2);
       mbar_init(bar(bars->s_full[i]), 1);
       mbar_init(bar(bars->dp_full[i]), 1);
       mbar_init(bar(bars->pds_full[i]), 256);
       mbar_init(bar(bars->dq_full[i]), 1);
       mbar_init(bar(bars->dq_free[i]), 128);
     }
-    mbar_init(bar(bars->kv_done), 1);
+    mbar_init(bar(bars->kv_done), 2);
+    mbar_init(bar(bars->acc_zero), 256);
     bars->abort = 0;
     bars->lo_tile[0] = bars->lo_tile[1] = 0;
     fence_barrier_init();
@@ -1039,8 +1073,11 @@ __global__ void __launch_bounds__(kSeqHThreads, 1)
       for (int i = 0; i < ntiles; ++i) {
         const int st = i & 1;
         const int t0 = (first_qt + i) * a.TQ;
+        // q_empty also means every P/dS warp is done with tile i-2's row terms
         if (i >= 2) mbar_wait(bar(bars->q_empty[st]), ((i >> 1) - 1) & 1, abort_flag);
-        mbar_expect_tx(bar(bars->q_full[st]), qbytes);
+        mbar_expect_tx(bar(bars->q_full[st]), qbytes + kRowTermBytes);
+        bulk_load(sLD(st), a.rt + ((long long)bg * a.nqt + first_qt + i) * 256, kRowTermBytes,
+                  bar(bars->q_full[st]));
         for (int rg = 0; rg < Cfg::kRegions; ++rg)
           tma_load_4d(sQ(st) + rg * kBwdRegion, &tmQ, bar(bars->q_full[st]), rg * 64, 0, t0,
                       bg);
@@ -1052,8 +1089,12 @@ __global__ void __launch_bounds__(kSeqHThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 13) {
-    // ------------------------------------------------------------ tcgen05 issuer
+  } else if (warp == 13 || warp == 14) {
+    // ------------------------------------------------------------ tcgen05 issuers
+    // One issuer per 64-row half, so that neither half's products wait behind a barrier
+    // of the other half; both feed the SM's one tensor pipe.  dV and dK accumulate the
+    // products of both issuers: the P/dS warps zero them first, and every product adds.
+    const int h = warp - 13;
     if (elect_one()) {
       constexpr uint32_t idesc_t = make_idesc_bf16(128, 64, 0, 0);  // S^T_h, dP^T_h
       constexpr uint32_t idesc_g = make_idesc_bf16(128, D, 0, 1);   // dV, dK (A in TMEM)
@@ -1061,10 +1102,8 @@ __global__ void __launch_bounds__(kSeqHThreads, 1)
       mbar_wait(bar(bars->kv_full), 0, abort_flag);
       // S^T_h(i) = K Q_h(i)^T, dP^T_h(i) = V dO_h(i)^T : B = the half's 64 rows, K-major
       auto issue_s = [&](int i, int h) {
-        if (h == 0) {
-          mbar_wait(bar(bars->q_full[i & 1]), (i >> 1) & 1, abort_flag);
-          tc_fence_after();
-        }
+        mbar_wait(bar(bars->q_full[i & 1]), (i >> 1) & 1, abort_flag);
+        tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t off = (ks / 4) * kBwdRegion + (ks % 4) * 32;
@@ -1075,10 +1114,8 @@ __global__ void __launch_bounds__(kSeqHThreads, 1)
         tc_commit(bar(bars->s_full[h]));
       };
       auto issue_dp = [&](int i, int h) {
-        if (h == 0) {
-          mbar_wait(bar(bars->do_full[i & 1]), (i >> 1) & 1, abort_flag);
-          tc_fence_after();
-        }
+        mbar_wait(bar(bars->do_full[i & 1]), (i >> 1) & 1, abort_flag);
+        tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t off = (ks / 4) * kBwdRegion + (ks % 4) * 32;
@@ -1090,26 +1127,27 @@ __global__ void __launch_bounds__(kSeqHThreads, 1)
       };
       // dV += P_h^T dO_h, dK += dS_h^T Q_h (hi then lo; K-step ks covers the half's rows
       // 16ks..16ks+15: packed columns 32(ks/2) + 8(ks%2) of the region, lo +16), then
-      // dQ^T_h = K^T dS_h^T into region A_h.
+      // dQ^T_h = K^T dS_h^T into region A_h, after dV has read P^T_h from it.
       auto issue_grads = [&](int i, int h) {
         mbar_wait(bar(bars->pds_full[h]), i & 1, abort_flag);
         tc_fence_after();
-        const int st = i & 1;
-        // the P/dS warps marked this half before arriving on pds_full
+        // the P/dS warps marked the half before arriving on pds_full
         const bool lo = lo_tile[h] == i + 1;
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
           const uint32_t col = (ks >> 1) * 32 + (ks & 1) * 8;
-          const uint64_t bd = make_sdesc_sw128(sDO(st) + (4 * h + ks) * 2048, kBwdRegion, 1024);
-          mma_ts(tDV, tA(h) + col, bd, idesc_g, (i > 0 || h > 0 || ks > 0) ? 1u : 0u);
+          const uint64_t bd =
+              make_sdesc_sw128(sDO(i & 1) + (4 * h + ks) * 2048, kBwdRegion, 1024);
+          mma_ts(tDV, tA(h) + col, bd, idesc_g, 1u);
           if (lo) mma_ts(tDV, tA(h) + col + 16, bd, idesc_g, 1u);
         }
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
           const uint32_t col = (ks >> 1) * 32 + (ks & 1) * 8;
-          const uint64_t bd = make_sdesc_sw128(sQ(st) + (4 * h + ks) * 2048, kBwdRegion, 1024);
-          mma_ts(tDK, tB(h) + col, bd, idesc_g, (i > 0 || h > 0 || ks > 0) ? 1u : 0u);
-          if (lo) mma_ts(tDK, tB(h) + col + 16, bd, idesc_g, 1u);
+          const uint64_t bq =
+              make_sdesc_sw128(sQ(i & 1) + (4 * h + ks) * 2048, kBwdRegion, 1024);
+          mma_ts(tDK, tB(h) + col, bq, idesc_g, 1u);
+          if (lo) mma_ts(tDK, tB(h) + col + 16, bq, idesc_g, 1u);
         }
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
@@ -1118,25 +1156,18 @@ __global__ void __launch_bounds__(kSeqHThreads, 1)
                  ks > 0 ? 1u : 0u);
         tc_commit(bar(bars->dq_full[h]));
       };
-      issue_s(0, 0);
-      issue_dp(0, 0);
-      issue_s(0, 1);
-      issue_dp(0, 1);
+      issue_s(0, h);
+      issue_dp(0, h);
+      mbar_wait(bar(bars->acc_zero), 0, abort_flag);
+      tc_fence_after();
       for (int i = 0; i < ntiles; ++i) {
-        const bool more = i + 1 < ntiles;
-        issue_grads(i, 0);
-        if (more) {
-          issue_dp(i + 1, 0);
-          mbar_wait(bar(bars->dq_free[0]), i & 1, abort_flag);
-          issue_s(i + 1, 0);
-        }
-        issue_grads(i, 1);
-        tc_commit(bar(bars->do_empty[i & 1]));
-        tc_commit(bar(bars->q_empty[i & 1]));
-        if (more) {
-          issue_dp(i + 1, 1);
-          mbar_wait(bar(bars->dq_free[1]), i & 1, abort_flag);
-          issue_s(i + 1, 1);
+        issue_grads(i, h);
+        tc_commit(bar(bars->do_empty[i & 1]));  // dO(i): dP and dV of this half read
+        tc_commit(bar(bars->q_empty[i & 1]));   // Q(i): S and dK of this half read
+        if (i + 1 < ntiles) {
+          issue_dp(i + 1, h);  // region B_h: dK has read dS^T_h
+          mbar_wait(bar(bars->dq_free[h]), i & 1, abort_flag);
+          issue_s(i + 1, h);
         }
       }
       tc_commit(bar(bars->kv_done));
@@ -1150,38 +1181,32 @@ __global__ void __launch_bounds__(kSeqHThreads, 1)
     const int kt = threadIdx.x & 127;  // TMEM lane = key key0 + kt
     const int key = key0 + kt;
     const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
-    // Row terms (lse, D) of the next tile, loaded by group 0 (row = kt) one tile ahead and
-    // transformed only when stored, so that the loads' latency stays hidden.
-    const int hl = kt % a.G, tok = kt / a.G;
-    float raw_l = 0.f, raw_d = 0.f;
-    bool raw_valid = false;
-    auto load_rowterms = [&](int i) {
-      const int t = (first_qt + i) * a.TQ + tok;
-      raw_valid = i < ntiles && tok < a.TQ && t < a.T;
-      const long long idx = ((long long)bg * a.G + hl) * a.T + (raw_valid ? t : 0);
-      raw_l = a.lse[idx];
-      raw_d = a.drow[idx];
-    };
-    if (g == 0) load_rowterms(0);
     const float2 sl2 = make_float2(a.scale_log2, a.scale_log2);
     const float2 sc2 = make_float2(a.scale, a.scale);
     const float2 neg1 = make_float2(-1.f, -1.f);
+    {
+      // this lane's row of the dV (group 0) or dK (group 1) accumulator starts at zero
+      const uint32_t zero8[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+      const uint32_t dst = (g ? tDK : tDV) + lane_base;
+#pragma unroll
+      for (int cc = 0; cc < D / 8; ++cc) tmem_st8(dst + 8 * cc, zero8);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(bars->acc_zero));
+    }
     for (int i = 0; i < ntiles; ++i) {
       const int qt = first_qt + i;
       const int b = i & 1;
-      if (g == 0) {
-        ld_s[b * 256 + kt] = raw_valid ? -raw_l * kLog2eBwd : -INFINITY;  // stored negated
-        ld_s[b * 256 + 128 + kt] = raw_valid ? -raw_d : 0.f;              // stored negated
-      }
-      named_bar_sync(1, 256);
-      if (g == 0) load_rowterms(i + 1);
+      // the tile's row terms, bulk-loaded with its Q (the wait orders their bytes before the
+      // reads below; the phase completed before S was computed)
+      mbar_wait(bar(bars->q_full[b]), (i >> 1) & 1, abort_flag);
       int r_min = 0;
       if (key >= a.T)
         r_min = 1 << 30;
       else if (a.causal)
         r_min = a.G * (key - qt * a.TQ);
-      const float* nlse2 = ld_s + b * 256;
-      const float* ndr = ld_s + b * 256 + 128;
+      const float* nlse2 = ld_s + b * 256;       // -lse * log2e per tile row
+      const float* ndr = ld_s + b * 256 + 128;   // -D * scale per tile row
 #pragma unroll 1
       for (int h = 0; h < 2; ++h) {
         mbar_wait(bar(bars->s_full[h]), i & 1, abort_flag);
@@ -1196,53 +1221,87 @@ __global__ void __launch_bounds__(kSeqHThreads, 1)
         const bool masked = r_min > c * 32;
         // dS for the dQ^T product: region h, this key's row, rows 32g..32g+31 of the half
         const uint32_t reg = sDS + h * kBwdRegion + uint32_t(kt) * 128;
-        float mlo = 0.f;  // largest lo value of this thread's P and dS elements
+        const uint32_t tP = tA(h) + lane_base + g * 32, tS = tB(h) + lane_base + g * 32;
+        // One pass over this thread's 32 elements: P = 2^(s*scale*log2e - lse*log2e) and
+        // dS = P * scale*(dP - D) (both row terms stored negated, D pre-scaled).  The first
+        // pass stores the bf16 P^T / dS^T words (hi, chunk columns 8k..) and returns the
+        // largest P or |dS|; kLo passes store what the rounding dropped (lo, 16 columns
+        // further).  kMask applies the causal / past-the-end mask: r_min <= 32c for a
+        // thread that has no masked row, so the test is exact for every thread.
+        auto pass = [&](auto mask_c, auto lo_c) {
+          constexpr bool kMask = decltype(mask_c)::value, kLo = decltype(lo_c)::value;
+          float mx = 0.f;
 #pragma unroll
-        for (int k = 0; k < 2; ++k) {  // 16-row sub-chunks
-          uint32_t pp[8], pl[8], pd[8], dl[8];
+          for (int k = 0; k < 2; ++k) {  // 16-row sub-chunks
+            uint32_t hp[8], hd[8], lp[8], ld[8];
 #pragma unroll
-          for (int e2 = 0; e2 < 16; e2 += 2) {
-            const int e = 16 * k + e2;
-            const int r = c * 32 + e;
-            const float2 arg = ffma2(
-                make_float2(__uint_as_float(s[e]), __uint_as_float(s[e + 1])), sl2,
-                make_float2(nlse2[r], nlse2[r + 1]));
-            float P0 = ex2(arg.x), P1 = ex2(arg.y);
-            if (masked) {
-              if (r < r_min) P0 = 0.f;
-              if (r + 1 < r_min) P1 = 0.f;
+            for (int e4 = 0; e4 < 16; e4 += 4) {
+              const int r4 = c * 32 + 16 * k + e4;
+              const float4 nl = *reinterpret_cast<const float4*>(nlse2 + r4);
+              const float4 nd = *reinterpret_cast<const float4*>(ndr + r4);
+#pragma unroll
+              for (int u = 0; u < 2; ++u) {
+                const int e = 16 * k + e4 + 2 * u, r = r4 + 2 * u, w = (e4 >> 1) + u;
+                const float2 arg = ffma2(
+                    make_float2(__uint_as_float(s[e]), __uint_as_float(s[e + 1])), sl2,
+                    u ? make_float2(nl.z, nl.w) : make_float2(nl.x, nl.y));
+                float P0 = ex2(arg.x), P1 = ex2(arg.y);
+                if constexpr (kMask) {
+                  if (r < r_min) P0 = 0.f;
+                  if (r + 1 < r_min) P1 = 0.f;
+                }
+                const float2 dd = ffma2(
+                    make_float2(__uint_as_float(dp[e]), __uint_as_float(dp[e + 1])), sc2,
+                    u ? make_float2(nd.z, nd.w) : make_float2(nd.x, nd.y));
+                const float2 dS = fmul2(make_float2(P0, P1), dd);
+                const uint32_t ph = pack_bf16x2(P0, P1), dh = pack_bf16x2(dS.x, dS.y);
+                if constexpr (kLo) {
+                  const float2 plo =
+                      ffma2(make_float2(bf16lo(ph), bf16hi(ph)), neg1, make_float2(P0, P1));
+                  const float2 dlo = ffma2(make_float2(bf16lo(dh), bf16hi(dh)), neg1, dS);
+                  lp[w] = pack_bf16x2(plo.x, plo.y);
+                  ld[w] = pack_bf16x2(dlo.x, dlo.y);
+                } else {
+                  hp[w] = ph;
+                  hd[w] = dh;
+                  mx = fmax3(mx, P0, P1);
+                  mx = fmax3(mx, fabsf(dS.x), fabsf(dS.y));
+                }
+              }
             }
-            const float2 Ps = fmul2(make_float2(P0, P1), sc2);
-            const float2 dd = fadd2(
-                make_float2(__uint_as_float(dp[e]), __uint_as_float(dp[e + 1])),
-                make_float2(ndr[r], ndr[r + 1]));
-            const float2 dS = fmul2(Ps, dd);
-            const uint32_t ph = pack_bf16x2(P0, P1), dh = pack_bf16x2(dS.x, dS.y);
-            const float2 plo =
-                ffma2(make_float2(bf16lo(ph), bf16hi(ph)), neg1, make_float2(P0, P1));
-            const float2 dlo = ffma2(make_float2(bf16lo(dh), bf16hi(dh)), neg1, dS);
-            mlo = fmax3(mlo, fabsf(plo.x), fabsf(plo.y));
-            mlo = fmax3(mlo, fabsf(dlo.x), fabsf(dlo.y));
-            pp[e2 / 2] = ph;
-            pl[e2 / 2] = pack_bf16x2(plo.x, plo.y);
-            pd[e2 / 2] = dh;
-            dl[e2 / 2] = pack_bf16x2(dlo.x, dlo.y);
-          }
-          // packed P^T / dS^T words: hi at chunk column 8k.., lo 16 columns further
-          tmem_st8(tA(h) + lane_base + g * 32 + 8 * k, pp);
-          tmem_st8(tA(h) + lane_base + g * 32 + 16 + 8 * k, pl);
-          tmem_st8(tB(h) + lane_base + g * 32 + 8 * k, pd);
-          tmem_st8(tB(h) + lane_base + g * 32 + 16 + 8 * k, dl);
+            if constexpr (kLo) {
+              tmem_st8(tP + 16 + 8 * k, lp);
+              tmem_st8(tS + 16 + 8 * k, ld);
+            } else {
+              tmem_st8(tP + 8 * k, hp);
+              tmem_st8(tS + 8 * k, hd);
 #pragma unroll
-          for (int qd = 0; qd < 2; ++qd) {
-            const uint32_t chunk = g * 4 + 2 * k + qd;
-            sts128(reg + ((chunk ^ (uint32_t(kt) & 7u)) << 4),
-                   make_uint4(pd[qd * 4], pd[qd * 4 + 1], pd[qd * 4 + 2], pd[qd * 4 + 3]));
+              for (int qd = 0; qd < 2; ++qd) {
+                const uint32_t chunk = g * 4 + 2 * k + qd;
+                sts128(reg + ((chunk ^ (uint32_t(kt) & 7u)) << 4),
+                       make_uint4(hd[qd * 4], hd[qd * 4 + 1], hd[qd * 4 + 2], hd[qd * 4 + 3]));
+              }
+            }
+          }
+          return mx;
+        };
+        using kNo = std::integral_constant<bool, false>;
+        using kYes = std::integral_constant<bool, true>;
+        // warp-uniform choice: most warps of a causal pass hold no masked row
+        const float mx = __any_sync(0xffffffffu, masked) ? pass(kYes{}, kNo{}) : pass(kNo{}, kNo{});
+        if (__any_sync(0xffffffffu, mx > kLoKeep)) {
+          pass(kYes{}, kYes{});
+          // mark the half for its lo passes (ordered before this lane's arrival below)
+          if ((threadIdx.x & 31) == 0) lo_tile[h] = i + 1;
+        } else {
+          // zeros: the lo passes, if another warp's rows need them, add nothing for these
+          const uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            tmem_st8(tP + 16 + 8 * k, z);
+            tmem_st8(tS + 16 + 8 * k, z);
           }
         }
-        // mark the half for its lo passes (ordered before this lane's arrival below)
-        if (__any_sync(0xffffffffu, mlo > kLoKeep) && (threadIdx.x & 31) == 0)
-          lo_tile[h] = i + 1;
         tmem_wait_st();
         fence_proxy_async_smem();
         tc_fence_before();
@@ -1353,6 +1412,24 @@ cudaError_t launch_depth(const BwdDepthArgs& a, cudaStream_t stream, const char*
   return e;
 }
 
+// Byte offsets of the backward's workspace regions: the fp32 dq accumulator [B][Hq][T][d]
+// at 0, the head-major row terms D [B][Hq][T] (d = 64), the tiled row-term records
+// [B*Hkv][nqt][2][128] (d = 128), then the fp32 dkd/dvd accumulators of groups above
+// kDepthMaxG heads.
+struct BwdLayout {
+  size_t drow, rt, acc;
+};
+inline BwdLayout bwd_layout(const Problem& p) {
+  const size_t rows = size_t(p.B) * p.Hq * p.T;
+  BwdLayout l;
+  l.drow = rows * p.d * 4;
+  l.rt = (l.drow + rows * 4 + 255) & ~size_t(255);
+  const size_t rt_bytes =
+      p.d == 128 ? size_t(p.B) * p.Hkv * tile_geom(p).nqt * kRowTermBytes : 0;
+  l.acc = l.rt + rt_bytes;
+  return l;
+}
+
 template <int D>
 cudaError_t launch_backward_d(const Problem& p, const void* q, const void* k, const void* v,
                               const void* kd, const void* vd, const void* out,
@@ -1362,8 +1439,11 @@ cudaError_t launch_backward_d(const Problem& p, const void* q, const void* k, co
                               const char** why) {
   const TileGeom tg = tile_geom(p);
   const long long rows = (long long)p.B * p.Hq * p.T;
-  float* dqacc = static_cast<float*>(workspace);
-  float* drow = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + rows * D * 4);
+  const BwdLayout lay = bwd_layout(p);
+  uint8_t* const ws = static_cast<uint8_t*>(workspace);
+  float* dqacc = reinterpret_cast<float*>(ws);
+  float* drow = reinterpret_cast<float*>(ws + lay.drow);
+  float* rt = reinterpret_cast<float*>(ws + lay.rt);
 
   // 1. depth part, row terms, dq accumulator initialisation
   BwdDepthArgs da;
@@ -1376,7 +1456,12 @@ cudaError_t launch_backward_d(const Problem& p, const void* q, const void* k, co
   da.dkd = static_cast<__nv_bfloat16*>(dkd);
   da.dvd = static_cast<__nv_bfloat16*>(dvd);
   da.dqacc = dqacc;
-  da.drow = drow;
+  // the d = 64 sequence kernel reads head-major row terms, the d = 128 one tiled records;
+  // depth-only attention has no sequence part
+  da.drow = (D == 64 && !p.depth_only) ? drow : nullptr;
+  da.rt = (D == 128 && !p.depth_only) ? rt : nullptr;
+  da.TQ = tg.TQ;
+  da.nqt = tg.nqt;
   da.ntok = (long long)p.B * p.Hkv * p.T;
   da.T = p.T;
   da.L = p.L;
@@ -1402,9 +1487,8 @@ cudaError_t launch_backward_d(const Problem& p, const void* q, const void* k, co
     } else {
       // one launch per chunk of kDepthMaxG heads; dkd/dvd summed in fp32 in the workspace
       // after the dq accumulator and the row terms
-      const size_t off = (size_t(rows) * D * 4 + size_t(rows) * 4 + 255) & ~size_t(255);
       const size_t nd = size_t(p.B) * p.Hkv * p.T * size_t(p.L) * D;
-      da.dkd_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + off);
+      da.dkd_acc = reinterpret_cast<float*>(ws + lay.acc);
       da.dvd_acc = da.dkd_acc + nd;
       const int nchunk = (p.G + kDepthMaxG - 1) / kDepthMaxG;
       for (int c = 0; c < nchunk && e == cudaSuccess; ++c) {
@@ -1442,8 +1526,34 @@ cudaError_t launch_backward_d(const Problem& p, const void* q, const void* k, co
         return cudaErrorInvalidValue;
       }
     }
-    CUtensorMap mDQ;
-    {
+    SeqArgs sa;
+    sa.dk = static_cast<__nv_bfloat16*>(dk);
+    sa.dv = static_cast<__nv_bfloat16*>(dv);
+    sa.dqacc = dqacc;
+    sa.lse = lse;
+    sa.drow = drow;
+    sa.rt = rt;
+    sa.Hkv = p.Hkv;
+    sa.T = p.T;
+    sa.G = p.G;
+    sa.TQ = tg.TQ;
+    sa.nqt = tg.nqt;
+    sa.BG = int(BG);
+    sa.causal = p.causal;
+    sa.scale = p.scale;
+    sa.scale_log2 = p.scale * kLog2eBwd;
+    const int nkb = (p.T + 127) / 128;
+    if constexpr (D == 128) {
+      e = cudaFuncSetAttribute(moda_bwd_seq_h_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               SeqCfg<128>::kSmemBytes);
+      if (e != cudaSuccess) {
+        *why = "cudaFuncSetAttribute(sequence backward, halves) failed";
+        return e;
+      }
+      moda_bwd_seq_h_kernel<<<unsigned(BG) * nkb, kSeqHThreads, SeqCfg<128>::kSmemBytes,
+                              stream>>>(mQ, mDO, mK, mV, sa);
+    } else {
+      CUtensorMap mDQ;
       // fp32 dq accumulator viewed like q: [bg][t][head-in-group][c]; a box is 32 columns
       // (128 bytes) of one tile's rows (token, head), 128B-swizzled.
       const cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(p.G), cuuint64_t(p.T), BG};
@@ -1458,41 +1568,15 @@ cudaError_t launch_backward_d(const Problem& p, const void* q, const void* k, co
         *why = "cuTensorMapEncodeTiled failed for the dq accumulator";
         return cudaErrorInvalidValue;
       }
-    }
-    SeqArgs sa;
-    sa.dk = static_cast<__nv_bfloat16*>(dk);
-    sa.dv = static_cast<__nv_bfloat16*>(dv);
-    sa.dqacc = dqacc;
-    sa.lse = lse;
-    sa.drow = drow;
-    sa.Hkv = p.Hkv;
-    sa.T = p.T;
-    sa.G = p.G;
-    sa.TQ = tg.TQ;
-    sa.nqt = tg.nqt;
-    sa.BG = int(BG);
-    sa.causal = p.causal;
-    sa.scale = p.scale;
-    sa.scale_log2 = p.scale * kLog2eBwd;
-    e = cudaFuncSetAttribute(moda_bwd_seq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             SeqCfg<D>::kSmemBytes);
-    if (e != cudaSuccess) {
-      *why = "cudaFuncSetAttribute(sequence backward) failed";
-      return e;
-    }
-    const int nkb = (p.T + 127) / 128;
-    if ((stages & kStageSeq) && D == 128) {
-      e = cudaFuncSetAttribute(moda_bwd_seq_h_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               SeqCfg<128>::kSmemBytes);
+      e = cudaFuncSetAttribute(moda_bwd_seq_kernel<D>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               SeqCfg<D>::kSmemBytes);
       if (e != cudaSuccess) {
-        *why = "cudaFuncSetAttribute(sequence backward, halves) failed";
+        *why = "cudaFuncSetAttribute(sequence backward) failed";
         return e;
       }
-      moda_bwd_seq_h_kernel<<<unsigned(BG) * nkb, kSeqHThreads, SeqCfg<128>::kSmemBytes,
-                              stream>>>(mQ, mDO, mK, mV, sa);
-    } else if (stages & kStageSeq) {
       moda_bwd_seq_kernel<D><<<unsigned(BG) * nkb, kSeqThreads, SeqCfg<D>::kSmemBytes, stream>>>(
-        mQ, mDO, mK, mV, mDQ, sa);
+          mQ, mDO, mK, mV, mDQ, sa);
     }
     e = cudaGetLastError();
     if (e != cudaSuccess) {
@@ -1516,8 +1600,8 @@ cudaError_t launch_backward_d(const Problem& p, const void* q, const void* k, co
 }  // namespace
 
 size_t backward_workspace_bytes(const Problem& p) {
-  const size_t rows = size_t(p.B) * p.Hq * p.T;
-  size_t bytes = rows * p.d * 4 + rows * 4 + 256;
+  const BwdLayout lay = bwd_layout(p);
+  size_t bytes = lay.acc;
   // groups above kDepthMaxG heads: fp32 dkd and dvd accumulators for the chunked depth part
   if (p.G > kDepthMaxG) bytes += 2 * size_t(p.B) * p.Hkv * p.T * size_t(p.L) * p.d * 4;
   return bytes;

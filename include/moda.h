@@ -173,9 +173,10 @@ moda_status_t moda_depth_kv_write(const void *x, const void *w, void *kd, void *
 
 /*
  * Bytes of device workspace moda_backward needs for these sizes (fp32 dQ accumulator
- * [B][Hq][T][d] plus the fp32 row terms D = <dO, out> [B][Hq][T]; for groups Hq / Hkv
- * above 16 also fp32 dkd and dvd accumulators, 2 x [B][Hkv][T][L][d]).  0 for invalid
- * sizes.
+ * [B][Hq][T][d] plus the fp32 row terms: D = <dO, out> as [B][Hq][T] at d = 64, and at
+ * d = 128 both -lse*log2(e) and -D per query tile of floor(128 / G) tokens, 1 KB per tile
+ * and (batch, KV head); for groups Hq / Hkv above 16 also fp32 dkd and dvd accumulators,
+ * 2 x [B][Hkv][T][L][d]).  0 for invalid sizes.
  */
 size_t moda_backward_workspace_size(int B, int Hq, int Hkv, int T, int L, int d);
 
@@ -229,7 +230,7 @@ moda_status_t moda_backward_stages(const void *q, const void *k, const void *v,
  * it from a static device array of 64 MiB that every GPU loading the library holds until
  * the process exits.  Neither the caller nor the library allocates anything.
  *   - Sizes whose moda_backward_workspace_size() exceeds 64 MiB are rejected with
- *     MODA_ERR_UNSUPPORTED (about B*Hq*T <= 130000 rows at d = 128).
+ *     MODA_ERR_UNSUPPORTED (about B*Hq*T <= 128000 rows at d = 128).
  *   - Argument checks come first and need no device: a bad pointer or size is refused
  *     (MODA_ERR_INVALID_ARGUMENT, or MODA_ERR_UNSUPPORTED for sizes beyond 64 MiB)
  *     before anything touches the GPU.
