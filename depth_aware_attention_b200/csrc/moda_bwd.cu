@@ -1101,8 +1101,11 @@ __global__ void __launch_bounds__(kSeqHThreads, 1)
       constexpr uint32_t idesc_q = make_idesc_bf16(128, 64, 1, 1);  // dQ^T_h = K^T dS_h^T
       mbar_wait(bar(bars->kv_full), 0, abort_flag);
       // S^T_h(i) = K Q_h(i)^T, dP^T_h(i) = V dO_h(i)^T : B = the half's 64 rows, K-major
-      auto issue_s = [&](int i, int h) {
+      auto wait_q = [&](int i) {
         mbar_wait(bar(bars->q_full[i & 1]), (i >> 1) & 1, abort_flag);
+      };
+      // (q_full of tile i waited for beforehand)
+      auto issue_s = [&](int i, int h) {
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
@@ -1131,24 +1134,31 @@ __global__ void __launch_bounds__(kSeqHThreads, 1)
       auto issue_grads = [&](int i, int h) {
         mbar_wait(bar(bars->pds_full[h]), i & 1, abort_flag);
         tc_fence_after();
-        // the P/dS warps marked the half before arriving on pds_full
-        const bool lo = lo_tile[h] == i + 1;
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
           const uint32_t col = (ks >> 1) * 32 + (ks & 1) * 8;
-          const uint64_t bd =
-              make_sdesc_sw128(sDO(i & 1) + (4 * h + ks) * 2048, kBwdRegion, 1024);
-          mma_ts(tDV, tA(h) + col, bd, idesc_g, 1u);
-          if (lo) mma_ts(tDV, tA(h) + col + 16, bd, idesc_g, 1u);
+          mma_ts(tDV, tA(h) + col,
+                 make_sdesc_sw128(sDO(i & 1) + (4 * h + ks) * 2048, kBwdRegion, 1024), idesc_g,
+                 1u);
+          mma_ts(tDK, tB(h) + col,
+                 make_sdesc_sw128(sQ(i & 1) + (4 * h + ks) * 2048, kBwdRegion, 1024), idesc_g,
+                 1u);
         }
+        // the lo products, if the P/dS warps marked the half (before arriving on pds_full);
+        // the flag is read only now, so that its latency overlaps the products above
+        if (lo_tile[h] == i + 1) {
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          const uint32_t col = (ks >> 1) * 32 + (ks & 1) * 8;
-          const uint64_t bq =
-              make_sdesc_sw128(sQ(i & 1) + (4 * h + ks) * 2048, kBwdRegion, 1024);
-          mma_ts(tDK, tB(h) + col, bq, idesc_g, 1u);
-          if (lo) mma_ts(tDK, tB(h) + col + 16, bq, idesc_g, 1u);
+          for (int ks = 0; ks < 4; ++ks) {
+            const uint32_t col = (ks >> 1) * 32 + (ks & 1) * 8 + 16;
+            mma_ts(tDV, tA(h) + col,
+                   make_sdesc_sw128(sDO(i & 1) + (4 * h + ks) * 2048, kBwdRegion, 1024),
+                   idesc_g, 1u);
+            mma_ts(tDK, tB(h) + col,
+                   make_sdesc_sw128(sQ(i & 1) + (4 * h + ks) * 2048, kBwdRegion, 1024),
+                   idesc_g, 1u);
+          }
         }
+        // dQ^T_h overwrites P^T_h (hi and lo): issued after every product that reads it
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
           mma_ss(tA(h), make_sdesc_sw128(sK + ks * 2048, kBwdRegion, 1024),
@@ -1156,6 +1166,7 @@ __global__ void __launch_bounds__(kSeqHThreads, 1)
                  ks > 0 ? 1u : 0u);
         tc_commit(bar(bars->dq_full[h]));
       };
+      wait_q(0);
       issue_s(0, h);
       issue_dp(0, h);
       mbar_wait(bar(bars->acc_zero), 0, abort_flag);
@@ -1166,6 +1177,8 @@ __global__ void __launch_bounds__(kSeqHThreads, 1)
         tc_commit(bar(bars->q_empty[i & 1]));   // Q(i): S and dK of this half read
         if (i + 1 < ntiles) {
           issue_dp(i + 1, h);  // region B_h: dK has read dS^T_h
+          // the next Q first, so that only the dQ readout stands between it and S'
+          wait_q(i + 1);
           mbar_wait(bar(bars->dq_free[h]), i & 1, abort_flag);
           issue_s(i + 1, h);
         }
