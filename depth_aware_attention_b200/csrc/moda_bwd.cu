@@ -894,17 +894,18 @@ __global__ void __launch_bounds__(kSeqThreads, 1)
 //
 // Tensor-core issue order of half h's issuer per tile i (primes: tile i+1; brackets: the
 // barrier waited for):
-//   [pds_h] dV_h dK_h dQ_h dP_h'  [dqfree_h] S_h'
-// The two issuers share the tensor pipe, so one half's products run while the P/dS warps
-// work on the other half, and neither issuer waits behind the other half's barriers.
+//   [pds_h] dV_h dQ_h dK_h  [qdo'] dP_h'  [dqfree_h] S_h'
+// dQ_h comes second so that its readout, which S_h' waits for, starts early.  The two
+// issuers share the tensor pipe, so one half's products run while the P/dS warps work on
+// the other half, and neither issuer waits behind the other half's barriers.  (So the two
+// halves' dV and dK products are summed in whichever order they reach the pipe.)
 // warps 0-7 P/dS, 8-11 dQ, 12 TMA, 13 and 14 tcgen05 issuers of halves 0 and 1
 constexpr int kSeqHThreads = 480;
 constexpr uint32_t kRowTermBytes = 2 * 128 * 4;  // one tile's -lse*log2e and -D records
 
 struct SeqHBars {
   uint64_t kv_full;
-  uint64_t q_full[2], q_empty[2];
-  uint64_t do_full[2], do_empty[2];
+  uint64_t qdo_full[2], qdo_empty[2];  // Q, dO and row terms of a tile stage
   uint64_t s_full[2], dp_full[2], pds_full[2], dq_full[2], dq_free[2];
   uint64_t kv_done, acc_zero;
   uint32_t tmem_base;
@@ -1016,10 +1017,8 @@ __global__ void __launch_bounds__(kSeqHThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(bar(bars->kv_full), 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(bar(bars->q_full[i]), 1);
-      mbar_init(bar(bars->q_empty[i]), 2);  // one commit from each issuer
-      mbar_init(bar(bars->do_full[i]), 1);
-      mbar_init(bar(bars->do_empty[i]), 2);
+      mbar_init(bar(bars->qdo_full[i]), 1);
+      mbar_init(bar(bars->qdo_empty[i]), 2);  // one commit from each issuer
       mbar_init(bar(bars->s_full[i]), 1);
       mbar_init(bar(bars->dp_full[i]), 1);
       mbar_init(bar(bars->pds_full[i]), 256);
@@ -1073,19 +1072,16 @@ __global__ void __launch_bounds__(kSeqHThreads, 1)
       for (int i = 0; i < ntiles; ++i) {
         const int st = i & 1;
         const int t0 = (first_qt + i) * a.TQ;
-        // q_empty also means every P/dS warp is done with tile i-2's row terms
-        if (i >= 2) mbar_wait(bar(bars->q_empty[st]), ((i >> 1) - 1) & 1, abort_flag);
-        mbar_expect_tx(bar(bars->q_full[st]), qbytes + kRowTermBytes);
+        // qdo_empty also means every P/dS warp is done with tile i-2's row terms
+        if (i >= 2) mbar_wait(bar(bars->qdo_empty[st]), ((i >> 1) - 1) & 1, abort_flag);
+        const uint32_t full = bar(bars->qdo_full[st]);
+        mbar_expect_tx(full, 2 * qbytes + kRowTermBytes);
         bulk_load(sLD(st), a.rt + ((long long)bg * a.nqt + first_qt + i) * 256, kRowTermBytes,
-                  bar(bars->q_full[st]));
-        for (int rg = 0; rg < Cfg::kRegions; ++rg)
-          tma_load_4d(sQ(st) + rg * kBwdRegion, &tmQ, bar(bars->q_full[st]), rg * 64, 0, t0,
-                      bg);
-        if (i >= 2) mbar_wait(bar(bars->do_empty[st]), ((i >> 1) - 1) & 1, abort_flag);
-        mbar_expect_tx(bar(bars->do_full[st]), qbytes);
-        for (int rg = 0; rg < Cfg::kRegions; ++rg)
-          tma_load_4d(sDO(st) + rg * kBwdRegion, &tmDO, bar(bars->do_full[st]), rg * 64, 0,
-                      t0, bg);
+                  full);
+        for (int rg = 0; rg < Cfg::kRegions; ++rg) {
+          tma_load_4d(sQ(st) + rg * kBwdRegion, &tmQ, full, rg * 64, 0, t0, bg);
+          tma_load_4d(sDO(st) + rg * kBwdRegion, &tmDO, full, rg * 64, 0, t0, bg);
+        }
       }
     }
     __syncwarp();
@@ -1101,10 +1097,10 @@ __global__ void __launch_bounds__(kSeqHThreads, 1)
       constexpr uint32_t idesc_q = make_idesc_bf16(128, 64, 1, 1);  // dQ^T_h = K^T dS_h^T
       mbar_wait(bar(bars->kv_full), 0, abort_flag);
       // S^T_h(i) = K Q_h(i)^T, dP^T_h(i) = V dO_h(i)^T : B = the half's 64 rows, K-major
-      auto wait_q = [&](int i) {
-        mbar_wait(bar(bars->q_full[i & 1]), (i >> 1) & 1, abort_flag);
+      auto wait_qdo = [&](int i) {
+        mbar_wait(bar(bars->qdo_full[i & 1]), (i >> 1) & 1, abort_flag);
       };
-      // (q_full of tile i waited for beforehand)
+      // (qdo_full of tile i waited for beforehand)
       auto issue_s = [&](int i, int h) {
         tc_fence_after();
 #pragma unroll
@@ -1117,7 +1113,6 @@ __global__ void __launch_bounds__(kSeqHThreads, 1)
         tc_commit(bar(bars->s_full[h]));
       };
       auto issue_dp = [&](int i, int h) {
-        mbar_wait(bar(bars->do_full[i & 1]), (i >> 1) & 1, abort_flag);
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
@@ -1134,51 +1129,49 @@ __global__ void __launch_bounds__(kSeqHThreads, 1)
       auto issue_grads = [&](int i, int h) {
         mbar_wait(bar(bars->pds_full[h]), i & 1, abort_flag);
         tc_fence_after();
+        // dV (reads P^T_h), then dQ^T_h over P^T_h, then dK (reads dS^T_h from B_h): the
+        // dQ readout, which the next S product waits for, starts as early as it can
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          const uint32_t col = (ks >> 1) * 32 + (ks & 1) * 8;
-          mma_ts(tDV, tA(h) + col,
+        for (int ks = 0; ks < 4; ++ks)
+          mma_ts(tDV, tA(h) + (ks >> 1) * 32 + (ks & 1) * 8,
                  make_sdesc_sw128(sDO(i & 1) + (4 * h + ks) * 2048, kBwdRegion, 1024), idesc_g,
                  1u);
-          mma_ts(tDK, tB(h) + col,
-                 make_sdesc_sw128(sQ(i & 1) + (4 * h + ks) * 2048, kBwdRegion, 1024), idesc_g,
-                 1u);
-        }
         // the lo products, if the P/dS warps marked the half (before arriving on pds_full);
         // the flag is read only now, so that its latency overlaps the products above
-        if (lo_tile[h] == i + 1) {
+        const bool lo = lo_tile[h] == i + 1;
+        if (lo) {
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            const uint32_t col = (ks >> 1) * 32 + (ks & 1) * 8 + 16;
-            mma_ts(tDV, tA(h) + col,
+          for (int ks = 0; ks < 4; ++ks)
+            mma_ts(tDV, tA(h) + (ks >> 1) * 32 + (ks & 1) * 8 + 16,
                    make_sdesc_sw128(sDO(i & 1) + (4 * h + ks) * 2048, kBwdRegion, 1024),
                    idesc_g, 1u);
-            mma_ts(tDK, tB(h) + col,
-                   make_sdesc_sw128(sQ(i & 1) + (4 * h + ks) * 2048, kBwdRegion, 1024),
-                   idesc_g, 1u);
-          }
         }
-        // dQ^T_h overwrites P^T_h (hi and lo): issued after every product that reads it
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
           mma_ss(tA(h), make_sdesc_sw128(sK + ks * 2048, kBwdRegion, 1024),
                  make_sdesc_sw128(sDS + h * kBwdRegion + ks * 2048, kBwdRegion, 1024), idesc_q,
                  ks > 0 ? 1u : 0u);
         tc_commit(bar(bars->dq_full[h]));
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint32_t col = (ks >> 1) * 32 + (ks & 1) * 8;
+          const uint64_t bq =
+              make_sdesc_sw128(sQ(i & 1) + (4 * h + ks) * 2048, kBwdRegion, 1024);
+          mma_ts(tDK, tB(h) + col, bq, idesc_g, 1u);
+          if (lo) mma_ts(tDK, tB(h) + col + 16, bq, idesc_g, 1u);
+        }
       };
-      wait_q(0);
+      wait_qdo(0);
       issue_s(0, h);
       issue_dp(0, h);
       mbar_wait(bar(bars->acc_zero), 0, abort_flag);
       tc_fence_after();
       for (int i = 0; i < ntiles; ++i) {
         issue_grads(i, h);
-        tc_commit(bar(bars->do_empty[i & 1]));  // dO(i): dP and dV of this half read
-        tc_commit(bar(bars->q_empty[i & 1]));   // Q(i): S and dK of this half read
+        tc_commit(bar(bars->qdo_empty[i & 1]));  // Q(i), dO(i): this half's products read
         if (i + 1 < ntiles) {
+          wait_qdo(i + 1);
           issue_dp(i + 1, h);  // region B_h: dK has read dS^T_h
-          // the next Q first, so that only the dQ readout stands between it and S'
-          wait_q(i + 1);
           mbar_wait(bar(bars->dq_free[h]), i & 1, abort_flag);
           issue_s(i + 1, h);
         }
@@ -1210,9 +1203,8 @@ __global__ void __launch_bounds__(kSeqHThreads, 1)
     for (int i = 0; i < ntiles; ++i) {
       const int qt = first_qt + i;
       const int b = i & 1;
-      // the tile's row terms, bulk-loaded with its Q (the wait orders their bytes before the
-      // reads below; the phase completed before S was computed)
-      mbar_wait(bar(bars->q_full[b]), (i >> 1) & 1, abort_flag);
+      // The tile's row terms came with its Q and dO: the issuer saw them land (qdo_full)
+      // before it issued S, and the s_full wait below orders them before the reads.
       int r_min = 0;
       if (key >= a.T)
         r_min = 1 << 30;

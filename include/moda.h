@@ -187,8 +187,10 @@ size_t moda_backward_workspace_size(int B, int Hq, int Hkv, int T, int L, int d)
  *   dq = scale * sum dS * key,  dk/dkd = scale * sum dS * q,  dv/dvd = sum P * dout.
  * The pages give no backward design; this is the exact gradient of the definition.
  * Groups above 16 heads run the depth part once per 16 heads, summing dkd and dvd in fp32
- * accumulators that the workspace then also holds.  dq is summed with fp32 atomics,
- * so its last bits may differ between runs; dk, dv, dkd and dvd are deterministic.
+ * accumulators that the workspace then also holds.  dq is summed with fp32 atomics, and
+ * dk and dv add the two 64-row halves of each query tile in the order their products
+ * reach the tensor cores, so the last bits of dq, dk and dv may differ between runs;
+ * dkd and dvd are deterministic.
  * `out` and `lse` must be the forward's outputs for the same inputs.  `workspace`
  * (device, >= moda_backward_workspace_size bytes, 256-byte aligned) is scratch owned
  * by the caller; its contents on entry do not matter.

@@ -84,15 +84,21 @@ def test_backward_small_full(name, cfg, causal):
         compare_grad(g[n], ref[n], f"{name}:{n}")
 
 
-def test_backward_is_deterministic_in_dk_dv_and_leaves_inputs_intact():
+def test_backward_is_deterministic_in_dkd_dvd_and_leaves_inputs_intact():
     cfg = dict(B=1, T=515, Hq=8, Hkv=2, d=128, L=6)
     x = gpu_inputs(cfg, seed_base=250, with_dout=True)
     before = {k: v.clone() for k, v in x.items() if v is not None}
     a = run_gpu(x, 1 / math.sqrt(128), True)
     b = run_gpu(x, 1 / math.sqrt(128), True)
-    # dk, dv, dkd, dvd have one writer per element; dq sums fp32 atomics (order varies)
-    for n in ("dk", "dv", "dkd", "dvd"):
+    # dkd and dvd have one writer per element.  dq sums fp32 atomics, and dk, dv sum the
+    # two half tiles' products in whichever order their issuers reach the tensor pipe:
+    # those may differ between runs by the fp32 summation order, at most one bf16 step
+    # after rounding.
+    for n in ("dkd", "dvd"):
         assert torch.equal(a[n], b[n]), n
+    for n in ("dk", "dv"):
+        d = (a[n].float() - b[n].float()).abs()
+        assert (d <= a[n].float().abs() * 2.0 ** -7 + 1e-6).all().item(), n
     assert (a["dq"].float() - b["dq"].float()).abs().max().item() < 1e-3
     for k, v in before.items():
         assert torch.equal(v, x[k]), k
