@@ -353,10 +353,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       };
       auto release = [&](int e) { tc_commit(bar(bars->empty[e % NKV])); };
       // A sequence block's K and V are released after tile 1 (the last user) has read
-      // them; a depth block is its tile's own.
+      // them; a depth block is its tile's own.  Tile 1 does not wait again for a sequence
+      // block's entries that tile 0 (same thread, earlier) already saw land: each wait is
+      // a shared-memory round trip on the path from P to the next product.
+      auto seen_by_tile0 = [&](int t, int j) { return t == 1 && j < N0 && !sm.is_depth(j); };
       auto issue_s = [&](int t, int j) {
         const int e = kidx(t, j);
-        wait_entry(e);
+        if (seen_by_tile0(t, j))
+          tc_fence_after();
+        else
+          wait_entry(e);
         const uint32_t kbase = sKV(e % NKV);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
@@ -368,9 +374,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (sm.is_depth(j) || t == 1) release(e);
       };
       auto issue_pv = [&](int t, int j) {
-        mbar_wait(bar(bars->p_full[t]), j & 1, abort_flag);
         const int e = vidx(t, j);
-        wait_entry(e);
+        // V's entry first: it has normally landed long before P is ready
+        if (!seen_by_tile0(t, j)) wait_entry(e);
+        mbar_wait(bar(bars->p_full[t]), j & 1, abort_flag);
+        tc_fence_after();
         const uint32_t vbase = sKV(e % NKV);
         const uint32_t tO = tmem + 256 + t * D;
 #pragma unroll
