@@ -104,7 +104,9 @@ __host__ __device__ constexpr int bf_head(int lane, int i) {
   return (base + i) % (NV / 2);
 }
 
-template <int D, int GM>
+// kRT: also write the tiled row-term records (a.rt, the d = 128 sequence kernel's input);
+// the instantiation without them is the one depth-only attention and d = 64 run.
+template <int D, int GM, bool kRT>
 // (GM <= 4: at most 168 registers, three CTAs per SM; measured faster than 188 registers
 // and two CTAs)
 __global__ void __launch_bounds__(kDepthThreads, GM <= 4 ? 3 : 1)
@@ -136,8 +138,8 @@ __global__ void __launch_bounds__(kDepthThreads, GM <= 4 ? 3 : 1)
     const long long tkc = valid ? tk : a.ntok - 1;
     const long long bg = tkc / a.T;
     const int t = int(tkc - bg * a.T);
-    const int qt = a.rt ? t / a.TQ : 0, tq = t - qt * a.TQ;
-    float* const rt_tile = a.rt ? a.rt + ((bg * a.nqt + qt) << 8) : nullptr;
+    const int qt = kRT ? t / a.TQ : 0, tq = t - qt * a.TQ;
+    float* const rt_tile = kRT ? a.rt + ((bg * a.nqt + qt) << 8) : nullptr;
     const int r0 = tq * a.Gfull + a.head0;  // tile row of this chunk's head 0
 
     float lse2[GM], drw[GM];
@@ -176,7 +178,7 @@ __global__ void __launch_bounds__(kDepthThreads, GM <= 4 ? 3 : 1)
         for (int o = NT / 2; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
         drw[h] = part;
         if (valid && cs == 0 && a.drow) a.drow[row] = part;
-        if (valid && cs == (h & (NT - 1)) && a.rt) {
+        if (kRT && valid && cs == (h & (NT - 1))) {
           rt_tile[r0 + h] = -lse2[h];
           rt_tile[128 + r0 + h] = -part * a.scale;
         }
@@ -184,7 +186,7 @@ __global__ void __launch_bounds__(kDepthThreads, GM <= 4 ? 3 : 1)
     }
     // the last token of a tile fills the tile's records past its rows (once, in the first
     // head chunk)
-    if (valid && a.rt && a.head0 == 0 && (tq == a.TQ - 1 || t == a.T - 1)) {
+    if (kRT && valid && a.head0 == 0 && (tq == a.TQ - 1 || t == a.T - 1)) {
       for (int r = r0 + a.Gfull + cs; r < 128; r += NT) {
         rt_tile[r] = -INFINITY;
         rt_tile[128 + r] = 0.f;
@@ -1393,25 +1395,25 @@ int sm_count() {
   return n > 0 ? n : 148;
 }
 
-template <int D, int GM>
+template <int D, int GM, bool kRT>
 cudaError_t launch_depth(const BwdDepthArgs& a, cudaStream_t stream, const char** why) {
   const int tpb = kDepthThreads / (D / 8);
   // q/dO slots (not needed when they live in registers) + the per-thread cp.async ring
   const size_t smem = (GM <= 4 ? 0 : size_t(tpb) * 2 * a.G * D * 2) + kDepthRingBytes;
-  cudaError_t e = cudaFuncSetAttribute(moda_bwd_depth_kernel<D, GM>,
+  cudaError_t e = cudaFuncSetAttribute(moda_bwd_depth_kernel<D, GM, kRT>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) {
     *why = "cudaFuncSetAttribute(depth backward) failed";
     return e;
   }
   int per_sm = 1;
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, moda_bwd_depth_kernel<D, GM>,
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, moda_bwd_depth_kernel<D, GM, kRT>,
                                                 kDepthThreads, smem);
   if (per_sm < 1) per_sm = 1;
   const long long need = (a.ntok + tpb - 1) / tpb;
   const long long cap = (long long)sm_count() * per_sm;
   const unsigned grid = unsigned(need < cap ? need : cap);
-  moda_bwd_depth_kernel<D, GM><<<grid, kDepthThreads, smem, stream>>>(a);
+  moda_bwd_depth_kernel<D, GM, kRT><<<grid, kDepthThreads, smem, stream>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) *why = "depth backward launch failed";
   return e;
@@ -1481,11 +1483,19 @@ cudaError_t launch_backward_d(const Problem& p, const void* q, const void* k, co
   cudaError_t e = cudaSuccess;
   if (stages & kStageDepth) {
     auto launch = [&]() {
-      if (da.G <= 1) return launch_depth<D, 1>(da, stream, why);
-      if (da.G <= 2) return launch_depth<D, 2>(da, stream, why);
-      if (da.G <= 4) return launch_depth<D, 4>(da, stream, why);
-      if (da.G <= 8) return launch_depth<D, 8>(da, stream, why);
-      return launch_depth<D, 16>(da, stream, why);
+      constexpr bool kRT = D == 128;  // (depth-only attention: rt is null, below)
+      if (da.rt == nullptr) {
+        if (da.G <= 1) return launch_depth<D, 1, false>(da, stream, why);
+        if (da.G <= 2) return launch_depth<D, 2, false>(da, stream, why);
+        if (da.G <= 4) return launch_depth<D, 4, false>(da, stream, why);
+        if (da.G <= 8) return launch_depth<D, 8, false>(da, stream, why);
+        return launch_depth<D, 16, false>(da, stream, why);
+      }
+      if (da.G <= 1) return launch_depth<D, 1, kRT>(da, stream, why);
+      if (da.G <= 2) return launch_depth<D, 2, kRT>(da, stream, why);
+      if (da.G <= 4) return launch_depth<D, 4, kRT>(da, stream, why);
+      if (da.G <= 8) return launch_depth<D, 8, kRT>(da, stream, why);
+      return launch_depth<D, 16, kRT>(da, stream, why);
     };
     if (p.G <= kDepthMaxG) {
       e = launch();
