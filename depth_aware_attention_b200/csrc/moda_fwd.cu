@@ -27,12 +27,15 @@
 //            lane r).  Fold path: the depth fold first.  Then per block (depth blocks of
 //            the dense path, then sequence blocks): S row from TMEM -> mask -> exp2 -> P
 //            (bf16) back into TMEM over S; O is rescaled only when the row max grows by
-//            more than 2^8.  Last the epilogue.
+//            more than 2^8.  A sequence block's P is published in two halves of 64 keys
+//            (O rescaled before the first), so that the products of the first half run
+//            while the warps compute the second.  Last the epilogue.
 //   warp 8   TMA producer: lane 0 streams the Q tiles and the K/V blocks (dense path:
 //            preceded by each depth step's kd/vd blocks of both tiles) through the K/V
 //            ring; fold path: lanes 1 and 2 stream tile 0's and tile 1's depth chunks
 //            through their own depth rings.  Every ring has exactly one in-order consumer.
-//   warp 9   tcgen05 issuer, in the order S0(0) S1(0) { PV0(j) S0(j+1) PV1(j) S1(j+1) }:
+//   warp 9   tcgen05 issuer, in the order S0(0) S1(0) { PV0(j) S0(j+1) PV1(j) S1(j+1) }
+//            (each PV in two halves of 64 keys, the first after P's first half):
 //            while one tile's warps turn S into P, the tensor cores work for the other
 //            tile.  Because S_t(j+1) is issued after PV_t(j), a tile's warps that have
 //            seen S_t(j+1) know PV_t(j) has finished, so rescaling O_t needs no extra wait.
@@ -89,6 +92,7 @@ struct Bars {
   uint64_t dfull[2][3];   // depth ring of tile t: data landed
   uint64_t dempty[2][3];  // depth ring of tile t: stage released by tile t's warps
   uint64_t s_full[2];     // S_t(j) in TMEM
+  uint64_t p_half[2];     // keys [0, 64) of P_t(j) in TMEM, O_t rescaled (all 128 threads)
   uint64_t p_full[2];     // P_t(j) in TMEM (and O_t rescaled)
   uint64_t o_final[2];    // last PV_t done
   uint64_t drain;         // abort path: every product issued so far has finished
@@ -209,6 +213,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         mbar_init(bar(bars->dempty[t][s]), 128);
       }
       mbar_init(bar(bars->s_full[t]), 1);
+      mbar_init(bar(bars->p_half[t]), 128);
       mbar_init(bar(bars->p_full[t]), 1);
       mbar_init(bar(bars->o_final[t]), 1);
     }
@@ -377,15 +382,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const int e = vidx(t, j);
         // V's entry first: it has normally landed long before P is ready
         if (!seen_by_tile0(t, j)) wait_entry(e);
-        mbar_wait(bar(bars->p_full[t]), j & 1, abort_flag);
-        tc_fence_after();
         const uint32_t vbase = sKV(e % NKV);
         const uint32_t tO = tmem + 256 + t * D;
+        // keys [0, 64) as soon as their P is in (while the warps compute the rest), then
+        // keys [64, 128)
 #pragma unroll
-        for (int ks = 0; ks < kBN / 16; ++ks)
-          mma_ts(tO, tmem + t * 128 + ks * 8,
-                 make_sdesc_sw128(vbase + ks * 2048, kRegion, 1024), idesc_o,
-                 (ks > 0 || j > 0 || NC > 0) ? 1u : 0u);
+        for (int part = 0; part < 2; ++part) {
+          mbar_wait(bar(part ? bars->p_full[t] : bars->p_half[t]), j & 1, abort_flag);
+          tc_fence_after();
+#pragma unroll
+          for (int kq = 0; kq < kBN / 32; ++kq) {
+            const int ks = part * (kBN / 32) + kq;
+            mma_ts(tO, tmem + t * 128 + ks * 8,
+                   make_sdesc_sw128(vbase + ks * 2048, kRegion, 1024), idesc_o,
+                   (ks > 0 || j > 0 || NC > 0) ? 1u : 0u);
+          }
+        }
         if (sm.is_depth(j) || t == 1) release(e);
       };
       // (no steps at all: depth-only attention on the fold path, whose O is the fold's)
@@ -560,6 +572,24 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const float m_new = grow ? m_cand : m;
       const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
       const float alpha = ex2(m - m_use);
+      // O_t holds every PV_t issued so far (S_t(jb) was issued after PV_t(jb-1)).  It is
+      // rescaled before the first half of P is published, since that half's PV may start
+      // at once.
+      const bool has_o = NC > 0 || jb > 0;
+      auto rescale_o = [&]() {
+        if (__any_sync(0xffffffffu, grow && has_o)) {
+          const float f = grow ? alpha : 1.f;
+#pragma unroll 1
+          for (int cc = 0; cc < D / 16; ++cc) {
+            uint32_t o[16];
+            tmem_ld16(tO + cc * 16, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+            tmem_st16(tO + cc * 16, o);
+          }
+        }
+      };
       float ps0 = 0.f, ps1 = 0.f;
       if (dstep) {
         uint32_t pk[16];
@@ -574,6 +604,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         uint32_t zero[16];
 #pragma unroll
         for (int c = 0; c < 16; ++c) zero[c] = 0u;
+        rescale_o();
         // packed P columns [16q, 16q+16) hold keys [32q, 32q+32): this warp's are pk
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -582,6 +613,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           else
             tmem_st16(tS + 16 * q, zero);
         }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(bars->p_half[tt]));  // (the whole P: a depth step's keys interleave)
       } else {
         // p = 2^(s*scale*log2e - m): one packed FFMA feeds each pair of exp2, one packed
         // add accumulates each pair
@@ -600,7 +634,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             ps2 = fadd2(ps2, p);
             pk[c / 2] = pack_bf16x2(p.x, p.y);
           }
-          tmem_st32(tS + half * 32, pk);
+          if (half == 0) {
+            rescale_o();
+            tmem_st32(tS, pk);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(bars->p_half[tt]));
+          } else {
+            tmem_st32(tS + 32, pk);
+          }
         }
         ps0 = ps2.x;
         ps1 = ps2.y;
@@ -608,20 +650,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const float ps = ps0 + ps1;
       l = l * alpha + ps;
       m = m_new;
-      // O_t holds every PV_t issued so far (S_t(jb) was issued after PV_t(jb-1)).
-      const bool has_o = NC > 0 || jb > 0;
-      if (__any_sync(0xffffffffu, grow && has_o)) {
-        const float f = grow ? alpha : 1.f;
-#pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t o[32];
-          tmem_ld32(tO + cc * 32, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
-          tmem_st32(tO + cc * 32, o);
-        }
-      }
       tmem_wait_st();
       tc_fence_before();
       named_bar_sync(wg_bar, 128);
