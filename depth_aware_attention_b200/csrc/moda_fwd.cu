@@ -45,6 +45,8 @@
 #include <cuda_runtime.h>
 #include <math.h>
 
+#include <type_traits>
+
 #include "moda_internal.h"
 #include "sm100.cuh"
 
@@ -528,10 +530,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     // token-major, so row r (token r / G) owns keys [r - hl, r - hl + G): all inside the
     // 32 keys of its warp's rows.  Only those 32 columns are read; P is zero elsewhere.
     const int key_lim = a.causal ? t : a.T - 1;
-    for (int jb = 0; jb < NS; ++jb) {
+    // Steps before K(R+1) may be either kind; then come the remaining depth steps, then
+    // sequence blocks only.  Each run has its own copy of the loop body, without the code
+    // of the kind it never meets, which keeps the hot loop small.
+    auto run_step = [&](const int jb, auto depth_c) {
       mbar_wait(bar(bars->s_full[tt]), jb & 1, abort_flag);
       tc_fence_after();
-      const bool dstep = kDense && sm.is_depth(jb);
+      // kind: 0 sequence block, 1 depth step, 2 either (StepMap decides)
+      constexpr int kind = decltype(depth_c)::value;
+      const bool dstep = kDense && (kind == 1 || (kind == 2 && sm.is_depth(jb)));
       const int ix = sm.index(jb);  // depth step or sequence block index
       uint32_t s[kBN];
       float mx = -INFINITY;  // row max on the raw scores (scale > 0); masked keys -> -inf
@@ -654,7 +661,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       tc_fence_before();
       named_bar_sync(wg_bar, 128);
       if (r == 0) mbar_arrive(bar(bars->p_full[tt]));
-    }
+    };
+    const int J0 = kDense ? min(NS, sm.K * (sm.R + 1)) : 0;
+    const int J1 = kDense ? min(NS, J0 + (sm.ND - sm.K)) : 0;
+#pragma unroll 1
+    for (int jb = 0; jb < J0; ++jb) run_step(jb, std::integral_constant<int, 2>{});
+#pragma unroll 1
+    for (int jb = J0; jb < J1; ++jb) run_step(jb, std::integral_constant<int, 1>{});
+#pragma unroll 1
+    for (int jb = J1; jb < NS; ++jb) run_step(jb, std::integral_constant<int, 0>{});
 
     // ---- epilogue
     if (NS > 0) mbar_wait(bar(bars->o_final[tt]), 0, abort_flag);
