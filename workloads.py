@@ -27,11 +27,13 @@ CONFIGS = {
     # deep-stack head layout at 4K tokens: small enough (2.2 GB of depth cache) for an
     # ncu capture of the depth-dominated regime
     "deep-4k": dict(B=1, T=4096, Hq=32, Hkv=8, d=128, L=128),
+    # the 16K fwd+bwd shape at head dimension 64, for the d = 64 kernels' ncu captures
+    "fwd-bwd-16k-d64": dict(B=1, T=16384, Hq=16, Hkv=4, d=64, L=48),
 }
 
 # seed base per workload (inputs use base*1000 + index, index 0..5 = q,k,v,kd,vd,dout)
 SEED_BASE = {"tiny": 0, "layer-4k": 1, "long-64k": 2, "long-64k-L0": 2, "deep-stack": 3,
-             "fwd-bwd-16k": 4, "deep-4k": 5}
+             "fwd-bwd-16k": 4, "deep-4k": 5, "fwd-bwd-16k-d64": 6}
 
 NAMES = ("q", "k", "v", "kd", "vd", "dout")
 
