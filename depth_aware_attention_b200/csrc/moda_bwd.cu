@@ -1233,10 +1233,9 @@ __global__ void __launch_bounds__(kSeqHThreads, 1)
         // dS = P * scale*(dP - D) (both row terms stored negated, D pre-scaled).  The first
         // pass stores the bf16 P^T / dS^T words (hi, chunk columns 8k..) and returns the
         // largest P or |dS|; kLo passes store what the rounding dropped (lo, 16 columns
-        // further).  kMask applies the causal / past-the-end mask: r_min <= 32c for a
-        // thread that has no masked row, so the test is exact for every thread.
-        auto pass = [&](auto mask_c, auto lo_c) {
-          constexpr bool kMask = decltype(mask_c)::value, kLo = decltype(lo_c)::value;
+        // further).
+        auto pass = [&](auto lo_c) {
+          constexpr bool kLo = decltype(lo_c)::value;
           float mx = 0.f;
 #pragma unroll
           for (int k = 0; k < 2; ++k) {  // 16-row sub-chunks
@@ -1248,15 +1247,11 @@ __global__ void __launch_bounds__(kSeqHThreads, 1)
               const float4 nd = *reinterpret_cast<const float4*>(ndr + r4);
 #pragma unroll
               for (int u = 0; u < 2; ++u) {
-                const int e = 16 * k + e4 + 2 * u, r = r4 + 2 * u, w = (e4 >> 1) + u;
+                const int e = 16 * k + e4 + 2 * u, w = (e4 >> 1) + u;
                 const float2 arg = ffma2(
                     make_float2(__uint_as_float(s[e]), __uint_as_float(s[e + 1])), sl2,
                     u ? make_float2(nl.z, nl.w) : make_float2(nl.x, nl.y));
-                float P0 = ex2(arg.x), P1 = ex2(arg.y);
-                if constexpr (kMask) {
-                  if (r < r_min) P0 = 0.f;
-                  if (r + 1 < r_min) P1 = 0.f;
-                }
+                const float P0 = ex2(arg.x), P1 = ex2(arg.y);
                 const float2 dd = ffma2(
                     make_float2(__uint_as_float(dp[e]), __uint_as_float(dp[e + 1])), sc2,
                     u ? make_float2(nd.z, nd.w) : make_float2(nd.x, nd.y));
@@ -1294,10 +1289,17 @@ __global__ void __launch_bounds__(kSeqHThreads, 1)
         };
         using kNo = std::integral_constant<bool, false>;
         using kYes = std::integral_constant<bool, true>;
-        // warp-uniform choice: most warps of a causal pass hold no masked row
-        const float mx = __any_sync(0xffffffffu, masked) ? pass(kYes{}, kNo{}) : pass(kNo{}, kNo{});
+        // A masked score (causal, or a key past the end) becomes -inf before the pass, so
+        // its P and dS are 0, in the few warps that hold a masked row (r_min <= 32c for a
+        // thread without one); the pass itself has one form.
+        if (__any_sync(0xffffffffu, masked)) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (c * 32 + e < r_min) s[e] = __float_as_uint(-INFINITY);
+        }
+        const float mx = pass(kNo{});
         if (__any_sync(0xffffffffu, mx > kLoKeep)) {
-          pass(kYes{}, kYes{});
+          pass(kYes{});
           // mark the half for its lo passes (ordered before this lane's arrival below)
           if ((threadIdx.x & 31) == 0) lo_tile[h] = i + 1;
         } else {
