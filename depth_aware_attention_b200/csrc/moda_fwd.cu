@@ -536,7 +536,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     auto run_step = [&](const int jb, auto depth_c) {
       mbar_wait(bar(bars->s_full[tt]), jb & 1, abort_flag);
       tc_fence_after();
-      // kind: 0 sequence block, 1 depth step, 2 either (StepMap decides)
+      // kind: 0 sequence block that needs no mask, 1 depth step, 2 either (StepMap
+      // decides), 3 sequence block that may need the causal or past-the-end mask
       constexpr int kind = decltype(depth_c)::value;
       const bool dstep = kDense && (kind == 1 || (kind == 2 && sm.is_depth(jb)));
       const int ix = sm.index(jb);  // depth step or sequence block index
@@ -559,7 +560,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         tmem_ld32(tS + 96, &s[96]);
         tmem_wait_ld();
         const int kbase = ix * kBN;
-        const bool need_mask = a.causal ? (kbase + kBN - 1 > t0) : (kbase + kBN > a.T);
+        const bool need_mask =
+            kind != 0 && (a.causal ? (kbase + kBN - 1 > t0) : (kbase + kBN > a.T));
         if (need_mask) {
 #pragma unroll
           for (int c = 0; c < kBN; ++c)
@@ -664,12 +666,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     };
     const int J0 = kDense ? min(NS, sm.K * (sm.R + 1)) : 0;
     const int J1 = kDense ? min(NS, J0 + (sm.ND - sm.K)) : 0;
+    // From J1 on, step j is sequence block j - J1 + K*R.  Blocks from ix_m on may hold
+    // keys past a row's token (causal) or past the end; the blocks before it need no mask.
+    const int ix_m = a.causal ? (t0 + 1) / kBN : a.T / kBN;
+    const int JM = min(NS, J1 + max(0, ix_m - (kDense ? sm.K * sm.R : 0)));
 #pragma unroll 1
     for (int jb = 0; jb < J0; ++jb) run_step(jb, std::integral_constant<int, 2>{});
 #pragma unroll 1
     for (int jb = J0; jb < J1; ++jb) run_step(jb, std::integral_constant<int, 1>{});
 #pragma unroll 1
-    for (int jb = J1; jb < NS; ++jb) run_step(jb, std::integral_constant<int, 0>{});
+    for (int jb = J1; jb < JM; ++jb) run_step(jb, std::integral_constant<int, 0>{});
+#pragma unroll 1
+    for (int jb = JM; jb < NS; ++jb) run_step(jb, std::integral_constant<int, 3>{});
 
     // ---- epilogue
     if (NS > 0) mbar_wait(bar(bars->o_final[tt]), 0, abort_flag);
