@@ -908,7 +908,7 @@ constexpr uint32_t kRowTermBytes = 2 * 128 * 4;  // one tile's -lse*log2e and -D
 struct SeqHBars {
   uint64_t kv_full;
   uint64_t qdo_full[2], qdo_empty[2];  // Q, dO and row terms of a tile stage
-  uint64_t s_full[2], dp_full[2], pds_full[2], dq_full[2], dq_free[2];
+  uint64_t s_full[2], pds_full[2], dq_full[2], dq_free[2];  // s_full: S and dP landed
   uint64_t kv_done, acc_zero;
   uint32_t tmem_base;
   int abort;
@@ -1022,7 +1022,6 @@ __global__ void __launch_bounds__(kSeqHThreads, 1)
       mbar_init(bar(bars->qdo_full[i]), 1);
       mbar_init(bar(bars->qdo_empty[i]), 2);  // one commit from each issuer
       mbar_init(bar(bars->s_full[i]), 1);
-      mbar_init(bar(bars->dp_full[i]), 1);
       mbar_init(bar(bars->pds_full[i]), 256);
       mbar_init(bar(bars->dq_full[i]), 1);
       mbar_init(bar(bars->dq_free[i]), 128);
@@ -1123,7 +1122,8 @@ __global__ void __launch_bounds__(kSeqHThreads, 1)
                  make_sdesc_sw128(sDO(i & 1) + off + 8192 * h, 16, 1024), idesc_t,
                  ks > 0 ? 1u : 0u);
         }
-        tc_commit(bar(bars->dp_full[h]));
+        // no commit of its own: the S product's commit, always issued later by this
+        // thread, tracks these products too
       };
       // dV += P_h^T dO_h, dK += dS_h^T Q_h (hi then lo; K-step ks covers the half's rows
       // 16ks..16ks+15: packed columns 32(ks/2) + 8(ks%2) of the region, lo +16), then
@@ -1163,16 +1163,23 @@ __global__ void __launch_bounds__(kSeqHThreads, 1)
           if (lo) mma_ts(tDK, tB(h) + col + 16, bq, idesc_g, 1u);
         }
       };
+      // dP before S in every tile: the commit of S then also covers dP, so the P/dS warps
+      // wait for S alone
       wait_qdo(0);
-      issue_s(0, h);
       issue_dp(0, h);
+      issue_s(0, h);
       mbar_wait(bar(bars->acc_zero), 0, abort_flag);
       tc_fence_after();
       for (int i = 0; i < ntiles; ++i) {
+        // one early test for the next tile's Q and dO, while this half's P/dS is still
+        // being computed: when they have landed, dP' below needs no wait of its own
+        const bool qdo_seen =
+            i + 1 < ntiles &&
+            mbar_try_wait(bar(bars->qdo_full[(i + 1) & 1]), ((i + 1) >> 1) & 1);
         issue_grads(i, h);
         tc_commit(bar(bars->qdo_empty[i & 1]));  // Q(i), dO(i): this half's products read
         if (i + 1 < ntiles) {
-          wait_qdo(i + 1);
+          if (!qdo_seen) wait_qdo(i + 1);
           issue_dp(i + 1, h);  // region B_h: dK has read dS^T_h
           mbar_wait(bar(bars->dq_free[h]), i & 1, abort_flag);
           issue_s(i + 1, h);
@@ -1216,14 +1223,27 @@ __global__ void __launch_bounds__(kSeqHThreads, 1)
       const float* ndr = ld_s + b * 256 + 128;   // -D * scale per tile row
 #pragma unroll 1
       for (int h = 0; h < 2; ++h) {
+        // S's commit came after dP's from the same issuer, so it covers both products
         mbar_wait(bar(bars->s_full[h]), i & 1, abort_flag);
-        mbar_wait(bar(bars->dp_full[h]), i & 1, abort_flag);
         tc_fence_after();
         const int c = 2 * h + g;  // 32-row chunk of the tile
         // the packed results overwrite these columns: load all 32 before storing any
         uint32_t s[32], dp[32];
         tmem_ld32(tA(h) + lane_base + g * 32, s);
         tmem_ld32(tB(h) + lane_base + g * 32, dp);
+        // row terms of one 16-row sub-chunk, read while the TMEM loads are in flight (the
+        // TMEM wait and the stores below order shared memory, so loads placed after them
+        // would wait for them)
+        float4 nlk[4], ndk[4];
+        auto load_rt = [&](int k) {
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const int r4 = c * 32 + 16 * k + 4 * q4;
+            nlk[q4] = *reinterpret_cast<const float4*>(nlse2 + r4);
+            ndk[q4] = *reinterpret_cast<const float4*>(ndr + r4);
+          }
+        };
+        load_rt(0);
         tmem_wait_ld();
         const bool masked = r_min > c * 32;
         // dS for the dQ^T product: region h, this key's row, rows 32g..32g+31 of the half
@@ -1237,14 +1257,13 @@ __global__ void __launch_bounds__(kSeqHThreads, 1)
         auto pass = [&](auto lo_c) {
           constexpr bool kLo = decltype(lo_c)::value;
           float mx = 0.f;
+          if constexpr (kLo) load_rt(0);
 #pragma unroll
           for (int k = 0; k < 2; ++k) {  // 16-row sub-chunks
             uint32_t hp[8], hd[8], lp[8], ld[8];
 #pragma unroll
             for (int e4 = 0; e4 < 16; e4 += 4) {
-              const int r4 = c * 32 + 16 * k + e4;
-              const float4 nl = *reinterpret_cast<const float4*>(nlse2 + r4);
-              const float4 nd = *reinterpret_cast<const float4*>(ndr + r4);
+              const float4 nl = nlk[e4 >> 2], nd = ndk[e4 >> 2];
 #pragma unroll
               for (int u = 0; u < 2; ++u) {
                 const int e = 16 * k + e4 + 2 * u, w = (e4 >> 1) + u;
@@ -1271,6 +1290,7 @@ __global__ void __launch_bounds__(kSeqHThreads, 1)
                 }
               }
             }
+            if (k == 0) load_rt(1);  // before the stores, which order shared memory
             if constexpr (kLo) {
               tmem_st8(tP + 16 + 8 * k, lp);
               tmem_st8(tS + 16 + 8 * k, ld);
