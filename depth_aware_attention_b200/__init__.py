@@ -34,7 +34,8 @@ EXPORTED = ("moda_forward", "moda_forward_depth_path", "moda_depth_attention_for
             "moda_depth_kv_write",
             "moda_backward", "moda_backward_workspace_size",
             "moda_backward_stages", "moda_backward_noalloc", "moda_check_device_errors",
-            "moda_test_set_device_fault", "moda_status_string", "moda_last_error_message")
+            "moda_test_set_device_fault", "moda_test_exp2_fma", "moda_status_string",
+            "moda_last_error_message")
 
 
 class ModaError(RuntimeError):
@@ -74,6 +75,8 @@ def _load():
     lib.moda_backward_noalloc.restype = I
     lib.moda_test_set_device_fault.argtypes = [I, ctypes.c_uint64]
     lib.moda_test_set_device_fault.restype = I
+    lib.moda_test_exp2_fma.argtypes = [P, P, I, P]
+    lib.moda_test_exp2_fma.restype = I
     lib.moda_check_device_errors.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
     lib.moda_check_device_errors.restype = I
     lib.moda_status_string.argtypes = [I]
@@ -177,6 +180,25 @@ def moda_test_set_device_fault(fault, wait_limit_ns=0):
     """TEST ONLY: set the kernels' injected fault and bounded-wait limit on the current
     device (0, 0 restores the normal state).  Returns the status."""
     return lib.moda_test_set_device_fault(int(fault), int(wait_limit_ns))
+
+
+def moda_test_exp2_fma(x_ptr, y_ptr, n, stream=None):
+    """TEST ONLY: raw call of the forward's FMA-pipe exp2 over n fp32 values; returns the
+    status."""
+    return lib.moda_test_exp2_fma(x_ptr, y_ptr, int(n), stream)
+
+
+def test_exp2_fma(x):
+    """TEST ONLY: 2^x for a contiguous fp32 CUDA tensor, by the forward kernel's FMA-pipe
+    exponential, on the current stream."""
+    import torch
+    if not (x.is_cuda and x.dtype == torch.float32 and x.is_contiguous()):
+        raise ValueError("x must be a contiguous float32 CUDA tensor")
+    y = torch.empty_like(x)
+    st = lib.moda_test_exp2_fma(x.data_ptr(), y.data_ptr(), x.numel(),
+                                torch.cuda.current_stream(x.device).cuda_stream)
+    _check(st, "moda_test_exp2_fma")
+    return y
 
 
 def moda_status_string(status):

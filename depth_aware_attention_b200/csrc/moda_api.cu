@@ -475,6 +475,23 @@ moda_status_t moda_test_set_device_fault(int fault, uint64_t wait_limit_ns) {
   return MODA_OK;
 }
 
+moda_status_t moda_test_exp2_fma(const float* x, float* y, int n, moda_stream_t stream) {
+  g_msg[0] = 0;
+  if (n < 0 || n > (1 << 30))
+    return fail(MODA_ERR_INVALID_ARGUMENT, "n must lie in [0, 2^30]");
+  if (n > 0 && (x == nullptr || y == nullptr))
+    return fail(MODA_ERR_INVALID_ARGUMENT, "x and y must be non-NULL when n > 0");
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(y)) & 3u)
+    return fail(MODA_ERR_INVALID_ARGUMENT, "x and y must be 4-byte aligned");
+  moda_status_t s = check_device();
+  if (s != MODA_OK) return s;
+  const cudaError_t e =
+      moda::launch_test_exp2_fma(x, y, n, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess)
+    return fail(MODA_ERR_CUDA, "exp2 test kernel launch failed: %s", cudaGetErrorString(e));
+  return MODA_OK;
+}
+
 moda_status_t moda_check_device_errors(moda_stream_t stream, uint32_t* flags) {
   g_msg[0] = 0;
   if (flags) *flags = 0;

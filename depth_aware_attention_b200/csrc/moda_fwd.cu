@@ -61,6 +61,32 @@ constexpr int kRegion = 16384;     // one 128-row x 128-byte swizzled region
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only past 256x
+// In sequence blocks that need no mask, every kExpFmaPeriod-th pair of exponentials is
+// computed by exp2_fma2 on the FMA pipe: at d = 128 the exponent unit is as busy as the
+// tensor cores, and moving a quarter of its work off it shortens each block's softmax.
+constexpr int kExpFmaPeriod = 4;
+
+// 2^x for a pair of scores on the FMA and integer pipes, leaving the exponent unit free:
+// adding 1.5 * 2^23 (whose float spacing is 1) rounds x to the nearest integer j, a cubic
+// fitted for least maximum relative error gives 2^(x - j) on [-1/2, 1/2] (at most 7.5e-5
+// in fp32, far inside the bf16 rounding of P), and j is added to the exponent field.  x
+// is clamped below at -125, whose 2^-125 is negligible beside any row sum it joins.
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  constexpr float kRound = 12582912.f;  // 1.5 * 2^23
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
+  const float2 t = fadd2(x, make_float2(kRound, kRound));
+  const float2 jf = fadd2(t, make_float2(-kRound, -kRound));
+  const float2 f = ffma2(jf, make_float2(-1.f, -1.f), x);
+  float2 p = ffma2(make_float2(0.05517132f, 0.05517132f), f,
+                   make_float2(0.24261054f, 0.24261054f));
+  p = ffma2(p, f, make_float2(0.69326097f, 0.69326097f));
+  p = ffma2(p, f, make_float2(0.99992812f, 0.99992812f));
+  // t's low mantissa bits hold j (two's complement): shifted to the exponent field they
+  // add j to p's exponent, and the constant's own bits shift out
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
 constexpr int kFwdThreads = 320;
 
 // kDense selects the depth path: false = CUDA-core fold from two depth rings, true =
@@ -639,7 +665,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             const float2 x = ffma2(make_float2(__uint_as_float(s[half * 64 + c]),
                                                __uint_as_float(s[half * 64 + c + 1])),
                                    sl2, nm2);
-            const float2 p = make_float2(ex2(x.x), ex2(x.y));
+            float2 p;
+            if constexpr (kind == 0) {
+              if ((c / 2) % kExpFmaPeriod == kExpFmaPeriod - 1)
+                p = exp2_fma2(x);
+              else
+                p = make_float2(ex2(x.x), ex2(x.y));
+            } else {
+              p = make_float2(ex2(x.x), ex2(x.y));
+            }
             ps2 = fadd2(ps2, p);
             pk[c / 2] = pack_bf16x2(p.x, p.y);
           }
@@ -813,10 +847,28 @@ cudaError_t launch_forward_d(const Problem& p, const void* q, const void* k, con
   return e;
 }
 
+// Test only: the FMA-pipe exp2 of the forward, one pair of elements per thread.
+__global__ void moda_test_exp2_fma_kernel(const float* __restrict__ x, float* __restrict__ y,
+                                          int n) {
+  const long long i = 2ll * ((long long)blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const bool two = i + 1 < n;
+  const float2 r = exp2_fma2(make_float2(x[i], two ? x[i + 1] : 0.f));
+  y[i] = r.x;
+  if (two) y[i + 1] = r.y;
+}
+
 }  // namespace
 
 // A dense depth block gives row r only the 32 columns of its own warp, which hold the G
 // entries of the row's token only when G <= 32 (and the block is whole when G divides 128).
+cudaError_t launch_test_exp2_fma(const float* x, float* y, int n, cudaStream_t stream) {
+  if (n <= 0) return cudaSuccess;
+  const int pairs = (n + 1) / 2, threads = 256;
+  moda_test_exp2_fma_kernel<<<(pairs + threads - 1) / threads, threads, 0, stream>>>(x, y, n);
+  return cudaGetLastError();
+}
+
 bool dense_depth_supported(const Problem& p) { return 128 % p.G == 0 && p.G <= 32; }
 
 bool dense_depth_default(const Problem& p) {

@@ -52,6 +52,9 @@ bool dense_depth_supported(const Problem& p);
 bool dense_depth_default(const Problem& p);
 
 // Forward launcher: returns a CUDA error code (cudaSuccess when enqueued).
+// Test only: y[i] = the forward's FMA-pipe 2^x (exp2_fma2) of x[i], i < n (device arrays).
+cudaError_t launch_test_exp2_fma(const float* x, float* y, int n, cudaStream_t stream);
+
 cudaError_t launch_forward(const Problem& p, const void* q, const void* k, const void* v,
                            const void* kd, const void* vd, void* out, float* lse,
                            int depth_path, EncodeTiledFn encode, cudaStream_t stream,

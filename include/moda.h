@@ -278,6 +278,21 @@ moda_status_t moda_check_device_errors(moda_stream_t stream, uint32_t *flags);
  */
 moda_status_t moda_test_set_device_fault(int fault, uint64_t wait_limit_ns);
 
+/*
+ * TEST ONLY: y[i] = 2^x[i] for 0 <= i < n, computed by the forward kernel's FMA-pipe
+ * exponential (the one that takes a quarter of the exponentials of unmasked sequence
+ * blocks off the exponent unit, in the softmax of the fused kernel of the hyper.ai
+ * summary of arXiv 2603.15619, section "Hardware-efficient implementation").  x and y:
+ * device arrays of n
+ * fp32 values, 4-byte aligned, owned by the caller; y may not overlap x.  Enqueued on
+ * `stream`.  Accuracy: relative error at most 8e-5 for x in [-125, 8]; below -125 the
+ * result is that of -125 (about 2.35e-38).  MODA_ERR_INVALID_ARGUMENT for n outside
+ * [0, 2^30], NULL or misaligned pointers (checked before any CUDA call); MODA_ERR_CUDA
+ * or MODA_ERR_UNSUPPORTED from the device check or the launch.  Not part of the paper's
+ * operator.
+ */
+moda_status_t moda_test_exp2_fma(const float *x, float *y, int n, moda_stream_t stream);
+
 /* Static English description of a status code.  Never NULL. */
 const char *moda_status_string(moda_status_t status);
 

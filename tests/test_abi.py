@@ -20,7 +20,7 @@ A = 1 << 20
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(moda_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(moda_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_every_declared_symbol_is_exported():
