@@ -119,6 +119,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   const int ndep = (split == 0 && a.L > 0) ? (a.L + kDecKeys - 1) / kDecKeys : 0;
   const int nblk = ndep + (sb1 - sb0);  // depth blocks first, then sequence blocks
   const int warp = threadIdx.x >> 5;
+  // the combine grid may be scheduled now: it waits for this grid's completion itself
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kDecStages; ++s) {
@@ -313,6 +315,8 @@ __global__ void __launch_bounds__(D) moda_decode_combine_kernel(const DecArgs a)
   const int d = threadIdx.x;
   const size_t base = size_t(bg) * a.nsplit * a.Gfull;
   const int ns = a.nsplit;
+  // the split grid's partials: wait for its completion (a no-op for an ordinary launch)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   for (int s = d; s < ns; s += D) {
     const size_t r = base + size_t(s) * a.Gfull + h;
     wgt[s] = a.ws_ml[r * 2];
@@ -334,6 +338,18 @@ __global__ void __launch_bounds__(D) moda_decode_combine_kernel(const DecArgs a)
   const float* accp = a.ws_acc + base * D + size_t(h) * D + d;  // split s at + s * G * D
   const size_t stride = size_t(a.Gfull) * D;
   int s = 0;
+  for (; s + 16 <= ns; s += 16) {  // sixteen independent loads in flight
+    float x[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) x[u] = accp[size_t(s + u) * stride];
+#pragma unroll
+    for (int u = 0; u < 16; u += 4) {
+      n0 = fmaf(wgt[s + u], x[u], n0);
+      n1 = fmaf(wgt[s + u + 1], x[u + 1], n1);
+      n2 = fmaf(wgt[s + u + 2], x[u + 2], n2);
+      n3 = fmaf(wgt[s + u + 3], x[u + 3], n3);
+    }
+  }
   for (; s + 4 <= ns; s += 4) {
     const float x0 = accp[size_t(s) * stride], x1 = accp[size_t(s + 1) * stride];
     const float x2 = accp[size_t(s + 2) * stride], x3 = accp[size_t(s + 3) * stride];
@@ -429,7 +445,26 @@ cudaError_t launch_decode_d(const Problem& p, const DecodeSplit& sp, const void*
     *why = "decode split kernel launch failed";
     return e;
   }
-  moda_decode_combine_kernel<D><<<unsigned(BG) * a.Gfull, D, 0, stream>>>(a);
+  {
+    // programmatic dependent launch: the combine grid is scheduled while the split grid
+    // runs (it triggers at its start) and waits for the split grid's completion and
+    // memory in its first instruction, so the launch gap overlaps the split grid's tail
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(BG) * a.Gfull);
+    cfg.blockDim = dim3(D);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, moda_decode_combine_kernel<D>, a);
+    if (e != cudaSuccess) {
+      *why = "decode combine kernel launch failed";
+      return e;
+    }
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) *why = "decode combine kernel launch failed";
   return e;
