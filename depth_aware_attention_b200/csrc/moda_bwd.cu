@@ -47,6 +47,7 @@ constexpr int kDepthMaxG = 16;  // heads of one depth-kernel launch (registers h
 constexpr int kDepthU = 2;     // depth entries per load batch
 constexpr int kDepthRing = 8;  // per-thread cp.async ring stages (batches in flight: 7)
 constexpr int kDepthRingBytes = kDepthRing * kDepthU * 2 * kDepthThreads * 16;
+constexpr int kDepthStageBytes = kDepthRingBytes / 2;  // staged mode: the ring's second half
 
 struct BwdDepthArgs {
   const __nv_bfloat16 *q, *out, *dout, *kd, *vd;
@@ -66,6 +67,11 @@ struct BwdDepthArgs {
   // D = sum_j P_j <dO, vd_j>, in a first pass over the token's entries, instead of from
   // the rounded out.  Every key of such a row is a depth key, so this is the exact D.
   int exact_rows;
+  // Set by the launcher for depth-only attention when the kernel keeps q and dO in
+  // registers (at most 4 heads) and TPB * L * heads * 8 bytes fit in half the ring: the
+  // first pass then stages each entry's (P, <dO, vd>) per head in shared memory, and the
+  // gradient pass reads those instead of recomputing them, streaming kd alone.
+  int staged;
   // Groups above kDepthMaxG heads run as several launches, one per chunk of at most
   // kDepthMaxG heads: G is this chunk's head count, head0 its first head, Gfull the group
   // size.  dkd/dvd sum over all the group's heads, so the chunks add their contributions
@@ -130,6 +136,15 @@ __global__ void __launch_bounds__(kDepthThreads, GM <= 4 ? 3 : 1)
     return ring + uint32_t((((stg * kU + u) * 2 + kv) * kDepthThreads + tid) * 16);
   };
   const long long L = a.L;
+  // Staged depth-only attention (see BwdDepthArgs::staged): the ring's first half carries
+  // kd alone, its second half holds each token's [L][GM] (P, <dO, vd>) pairs.
+  constexpr bool kCanStage = !kRT && kReg;
+  const bool staged = kCanStage && a.staged != 0;
+  auto rslot_kd = [&](int stg, int u) {
+    return ring + uint32_t(((stg * kU + u) * kDepthThreads + tid) * 16);
+  };
+  const uint32_t stage_slot =
+      ring + uint32_t(kDepthStageBytes) + uint32_t(slot) * uint32_t(L) * uint32_t(GM * 8);
 
   for (long long base = (long long)blockIdx.x * TPB; base < a.ntok;
        base += (long long)gridDim.x * TPB) {
@@ -201,96 +216,153 @@ __global__ void __launch_bounds__(kDepthThreads, GM <= 4 ? 3 : 1)
       for (int e = 0; e < 8; ++e) dq[h][e] = 0.f;
 
     const long long tok_off = (bg * a.T + t) * L * D + cs * 8;
-    if (a.exact_rows) {
-      // D_h = sum_j P_hj <dO_h, vd_j> with P_hj = 2^(y_hj * scale * log2(e) - lse_h * log2(e)),
-      // the same weights the gradient loop below recomputes; kd and vd are read once more.
-      // The dot products are finished by the butterfly of the gradient loop (below), each
-      // lane summing P * p for the heads it ends up holding; one broadcast per token.
-      constexpr int kNV0 = 2 * GM, kBC0 = bf_count<NT, kNV0>();
-      float lse_mine[kBC0], dsum[kBC0];
-#pragma unroll
-      for (int i = 0; i < kBC0; ++i) {
-        lse_mine[i] = dsum[i] = 0.f;
-#pragma unroll
-        for (int h = 0; h < GM; ++h)
-          if (h == bf_head<NT, kNV0>(cs, i)) lse_mine[i] = lse2[h];
-      }
-      const bool is_y = (cs & (NT / 2)) == 0;
-#pragma unroll 2
-      for (long long j = 0; j < L; ++j) {
-        uint4 kw = make_uint4(0, 0, 0, 0), vw = make_uint4(0, 0, 0, 0);
-        if (valid) {
-          kw = ldg_nc_v4(a.kd + tok_off + j * D);
-          vw = ldg_nc_v4(a.vd + tok_off + j * D);
-        }
-        float kf[8], vf[8];
-        unpack8(kw, kf);
-        unpack8(vw, vf);
-        float bv[kNV0];
-#pragma unroll
-        for (int h = 0; h < GM; ++h) {
-          bv[h] = bv[GM + h] = 0.f;
-          if (h < G) {
-            float qf[8], df[8];
-            if constexpr (kReg) {
-#pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                qf[e] = qreg[h][e];
-                df[e] = dreg[h][e];
-              }
-            } else {
-              unpack8(lds128(q_s + uint32_t((h * D + cs * 8) * 2)), qf);
-              unpack8(lds128(do_s + uint32_t((h * D + cs * 8) * 2)), df);
-            }
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              bv[h] = fmaf(qf[e], kf[e], bv[h]);
-              bv[GM + h] = fmaf(df[e], vf[e], bv[GM + h]);
-            }
-          }
-        }
-        int c = kNV0;
-#pragma unroll
-        for (int o = NT / 2; o > 0; o >>= 1) {
-          if (c > 1) {
-            const bool up = (cs & o) != 0;
-#pragma unroll
-            for (int i = 0; i < kNV0 / 2; ++i) {
-              if (i < c / 2) {
-                const float send = up ? bv[i] : bv[c / 2 + i];
-                const float keep = up ? bv[c / 2 + i] : bv[i];
-                bv[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-              }
-            }
-            c /= 2;
-          } else {
-            bv[0] += __shfl_xor_sync(0xffffffffu, bv[0], o);
-          }
-        }
+    // (depth-only attention only: the d = 128 MoDA instantiation, with its row-term
+    // records, never takes this path and is compiled without it)
+    if constexpr (!kRT) {
+      if (a.exact_rows) {
+        // D_h = sum_j P_hj <dO_h, vd_j>, P_hj = 2^(y_hj * scale * log2(e) - lse_h * log2(e)):
+        // the weights the gradient pass uses, which it reads back from the staged pairs or
+        // (not staged) recomputes, reading kd and vd once more.  The dot products are
+        // finished by the same butterfly as the gradient pass's (below), each lane summing
+        // P * p for the heads it ends up holding; one broadcast per token.
+        constexpr int kNV0 = 2 * GM, kBC0 = bf_count<NT, kNV0>();
+        float lse_mine[kBC0], dsum[kBC0];
 #pragma unroll
         for (int i = 0; i < kBC0; ++i) {
-          const float other = __shfl_xor_sync(0xffffffffu, bv[i], NT / 2);
-          const float yy = is_y ? bv[i] : other, pp = is_y ? other : bv[i];
-          dsum[i] = fmaf(ex2(yy * a.scale_log2 - lse_mine[i]), pp, dsum[i]);
+          lse_mine[i] = dsum[i] = 0.f;
+#pragma unroll
+          for (int h = 0; h < GM; ++h)
+            if (h == bf_head<NT, kNV0>(cs, i)) lse_mine[i] = lse2[h];
         }
-      }
-      const int slot0 = (threadIdx.x & 31) & ~(NT - 1);
+        const bool is_y = (cs & (NT / 2)) == 0;
+        // one entry of the first pass: the dot products, their butterfly, P and the row term
+        auto pre_entry = [&](const long long j, const uint4 kw, const uint4 vw) {
+          float kf[8], vf[8];
+          unpack8(kw, kf);
+          unpack8(vw, vf);
+          float bv[kNV0];
 #pragma unroll
-      for (int h = 0; h < GM; ++h) {
-        int src = 0, si = 0;
+          for (int h = 0; h < GM; ++h) {
+            bv[h] = bv[GM + h] = 0.f;
+            if (h < G) {
+              float qf[8], df[8];
+              if constexpr (kReg) {
 #pragma unroll
-        for (int l2 = NT / 2 - 1; l2 >= 0; --l2)
+                for (int e = 0; e < 8; ++e) {
+                  qf[e] = qreg[h][e];
+                  df[e] = dreg[h][e];
+                }
+              } else {
+                unpack8(lds128(q_s + uint32_t((h * D + cs * 8) * 2)), qf);
+                unpack8(lds128(do_s + uint32_t((h * D + cs * 8) * 2)), df);
+              }
 #pragma unroll
-          for (int i = 0; i < kBC0; ++i)
-            if (bf_head<NT, kNV0>(l2, i) == h) { src = l2; si = i; }
-        const float dh = __shfl_sync(0xffffffffu, dsum[si], slot0 + src);
-        if (h < G) {
-          drw[h] = dh;
-          if (valid && cs == 0 && a.drow) a.drow[(bg * a.Gfull + a.head0 + h) * a.T + t] = dh;
+              for (int e = 0; e < 8; ++e) {
+                bv[h] = fmaf(qf[e], kf[e], bv[h]);
+                bv[GM + h] = fmaf(df[e], vf[e], bv[GM + h]);
+              }
+            }
+          }
+          int c = kNV0;
+#pragma unroll
+          for (int o = NT / 2; o > 0; o >>= 1) {
+            if (c > 1) {
+              const bool up = (cs & o) != 0;
+#pragma unroll
+              for (int i = 0; i < kNV0 / 2; ++i) {
+                if (i < c / 2) {
+                  const float send = up ? bv[i] : bv[c / 2 + i];
+                  const float keep = up ? bv[c / 2 + i] : bv[i];
+                  bv[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+                }
+              }
+              c /= 2;
+            } else {
+              bv[0] += __shfl_xor_sync(0xffffffffu, bv[0], o);
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < kBC0; ++i) {
+            const float other = __shfl_xor_sync(0xffffffffu, bv[i], NT / 2);
+            const float yy = is_y ? bv[i] : other, pp = is_y ? other : bv[i];
+            const float Pw = ex2(yy * a.scale_log2 - lse_mine[i]);
+            dsum[i] = fmaf(Pw, pp, dsum[i]);
+            if constexpr (kCanStage) {
+              // one lane per head writes: a y lane whose all-reduce bits are 0 (lanes that
+              // differ only in those bits hold the same sums)
+              constexpr int kDup = NT / kNV0 - 1;
+              if (staged && is_y && (cs & kDup) == 0)
+                sts64f(stage_slot + uint32_t((j * GM + bf_head<NT, kNV0>(cs, i)) * 8), Pw, pp);
+            }
+          }
+        };
+        // kd and vd stream through a cp.async ring: staged, a four-stage one in the first
+        // half of the ring memory (the gradient pass reuses it for kd alone once this pass
+        // has drained); otherwise the whole ring, which the gradient pass then refills
+        auto pre_ring = [&](auto stages_c, auto slot_fn) {
+          constexpr int kPS = decltype(stages_c)::value;
+          auto issue_pre = [&](long long b) {
+            const int stg = int(b % kPS);
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+              const long long j = b * kU + u;
+              if (valid && j < L) {
+                cp_async16(slot_fn(stg, u, 0), a.kd + tok_off + j * D);
+                cp_async16(slot_fn(stg, u, 1), a.vd + tok_off + j * D);
+              }
+            }
+            cp_async_commit();
+          };
+#pragma unroll
+          for (int b = 0; b < kPS - 1; ++b) issue_pre(b);
+          for (long long j0 = 0; j0 < L; j0 += kU) {
+            const long long b = j0 / kU;
+            issue_pre(b + kPS - 1);
+            cp_async_wait<kPS - 1>();  // batch b has landed
+            const int stg = int(b % kPS);
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+              if (j0 + u >= L) break;
+              uint4 kw = make_uint4(0, 0, 0, 0), vw = make_uint4(0, 0, 0, 0);
+              if (valid) {
+                kw = lds128(slot_fn(stg, u, 0));
+                vw = lds128(slot_fn(stg, u, 1));
+              }
+              pre_entry(j0 + u, kw, vw);
+            }
+          }
+          cp_async_wait<0>();  // (only empty groups remain) before the ring is reused
+        };
+        if (staged) {
+          if constexpr (kCanStage) {
+            auto rslot_pre = [&](int stg, int u, int kv) {
+              return ring + uint32_t((((stg * kU + u) * 2 + kv) * kDepthThreads + tid) * 16);
+            };
+            pre_ring(std::integral_constant<int, 4>{}, rslot_pre);
+          }
+        } else {
+          pre_ring(std::integral_constant<int, kDNS>{}, rslot);
         }
+        const int slot0 = (threadIdx.x & 31) & ~(NT - 1);
+#pragma unroll
+        for (int h = 0; h < GM; ++h) {
+          int src = 0, si = 0;
+#pragma unroll
+          for (int l2 = NT / 2 - 1; l2 >= 0; --l2)
+#pragma unroll
+            for (int i = 0; i < kBC0; ++i)
+              if (bf_head<NT, kNV0>(l2, i) == h) { src = l2; si = i; }
+          const float dh = __shfl_sync(0xffffffffu, dsum[si], slot0 + src);
+          if (h < G) {
+            drw[h] = dh;
+            if (valid && cs == 0 && a.drow) a.drow[(bg * a.Gfull + a.head0 + h) * a.T + t] = dh;
+          }
+        }
+        if (staged) __syncwarp();  // the staged pairs, written by some lanes, read by all
       }
     }
-    // (after the exact row terms above, when they apply) row terms of the heads whose P and dS this lane computes (see the butterfly below)
+    // (after the exact row terms above, when they apply) row terms of the heads whose P and
+    // dS this lane computes (see the butterfly below)
     constexpr int kNV = 2 * GM, kBC = bf_count<NT, kNV>();
     float my_lse2[kBC], my_drw[kBC];
 #pragma unroll
@@ -303,6 +375,72 @@ __global__ void __launch_bounds__(kDepthThreads, GM <= 4 ? 3 : 1)
           my_drw[i] = drw[h];
         }
     }
+    if (staged) {
+      if constexpr (kCanStage) {
+        // gradient pass over the staged pairs: kd streams alone through the ring's first
+        // half, P and <dO, vd> of every head come from shared memory, dS = P (p - D)
+        auto issue_kd = [&](long long b) {
+          const int stg = int(b % kDNS);
+#pragma unroll
+          for (int u = 0; u < kU; ++u) {
+            const long long j = b * kU + u;
+            if (valid && j < L) cp_async16(rslot_kd(stg, u), a.kd + tok_off + j * D);
+          }
+          cp_async_commit();
+        };
+#pragma unroll
+        for (int b = 0; b < kDNS - 1; ++b) issue_kd(b);
+        for (long long j0 = 0; j0 < L; j0 += kU) {
+          const long long b = j0 / kU;
+          issue_kd(b + kDNS - 1);
+          cp_async_wait<kDNS - 1>();  // batch b has landed
+          const int stg = int(b % kDNS);
+          uint4 kwu[kU];
+#pragma unroll
+          for (int u = 0; u < kU; ++u) {
+            kwu[u] = make_uint4(0, 0, 0, 0);
+            if (valid && j0 + u < L) kwu[u] = lds128(rslot_kd(stg, u));
+          }
+#pragma unroll
+          for (int u = 0; u < kU; ++u) {
+            if (j0 + u >= L) break;
+            const long long j = j0 + u;
+            float kf[8];
+            unpack8(kwu[u], kf);
+            float dv[8], dk[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) dv[e] = dk[e] = 0.f;
+#pragma unroll
+            for (int h = 0; h < GM; ++h) {
+              if (h < G) {
+                const float2 Pp = lds64f(stage_slot + uint32_t((j * GM + h) * 8));
+                const float2 P2 = make_float2(Pp.x, Pp.x);
+                const float dSv = Pp.x * (Pp.y - drw[h]);
+                const float2 dS2 = make_float2(dSv, dSv);
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) {
+                  const float2 v2 = ffma2(P2, make_float2(dreg[h][e], dreg[h][e + 1]),
+                                          make_float2(dv[e], dv[e + 1]));
+                  const float2 k2 = ffma2(dS2, make_float2(qreg[h][e], qreg[h][e + 1]),
+                                          make_float2(dk[e], dk[e + 1]));
+                  const float2 q2 = ffma2(dS2, make_float2(kf[e], kf[e + 1]),
+                                          make_float2(dq[h][e], dq[h][e + 1]));
+                  dv[e] = v2.x; dv[e + 1] = v2.y;
+                  dk[e] = k2.x; dk[e + 1] = k2.y;
+                  dq[h][e] = q2.x; dq[h][e + 1] = q2.y;
+                }
+              }
+            }
+            if (valid) {  // (one launch holds the whole group here: acc_mode 0)
+              const long long o = tok_off + j * D;
+              *reinterpret_cast<uint4*>(a.dvd + o) = pack8(dv, 1.f);
+              *reinterpret_cast<uint4*>(a.dkd + o) = pack8(dk, a.scale);
+            }
+          }
+        }
+        cp_async_wait<0>();  // (only empty groups remain) before the ring is reused
+      }
+    } else {
     const long long nbat = (L + kU - 1) / kU;
     // batch b's copies (an empty group past the last batch keeps the group count uniform)
     auto issue = [&](long long b) {
@@ -481,6 +619,7 @@ __global__ void __launch_bounds__(kDepthThreads, GM <= 4 ? 3 : 1)
     }
     cp_async_wait<0>();  // (only empty groups remain) before the ring is reused
     (void)nbat;
+    }
     if (valid) {
 #pragma unroll
       for (int h = 0; h < GM; ++h) {
@@ -1418,8 +1557,15 @@ int sm_count() {
 }
 
 template <int D, int GM, bool kRT>
-cudaError_t launch_depth(const BwdDepthArgs& a, cudaStream_t stream, const char** why) {
+cudaError_t launch_depth(const BwdDepthArgs& args, cudaStream_t stream, const char** why) {
   const int tpb = kDepthThreads / (D / 8);
+  BwdDepthArgs a = args;
+  // depth-only attention with q and dO in registers: stage the first pass's (P, <dO, vd>)
+  // pairs when a CTA's tokens' pairs fit in the ring's second half
+  a.staged = (!kRT && GM <= 4 && a.exact_rows && a.acc_mode == 0 &&
+              (long long)tpb * a.L * GM * 8 <= kDepthStageBytes)
+                 ? 1
+                 : 0;
   // q/dO slots (not needed when they live in registers) + the per-thread cp.async ring
   const size_t smem = (GM <= 4 ? 0 : size_t(tpb) * 2 * a.G * D * 2) + kDepthRingBytes;
   cudaError_t e = cudaFuncSetAttribute(moda_bwd_depth_kernel<D, GM, kRT>,
@@ -1500,6 +1646,7 @@ cudaError_t launch_backward_d(const Problem& p, const void* q, const void* k, co
   da.acc_mode = 0;
   da.dkd_acc = da.dvd_acc = nullptr;
   da.exact_rows = p.depth_only;
+  da.staged = 0;  // (decided per launch in launch_depth)
   da.scale = p.scale;
   da.scale_log2 = p.scale * kLog2eBwd;
   cudaError_t e = cudaSuccess;

@@ -31,6 +31,11 @@ CASES = [
     ("g32-d128", dict(B=1, T=90, Hq=64, Hkv=2, d=128, L=6)),
     ("g64-d64", dict(B=1, T=70, Hq=64, Hkv=1, d=64, L=4)),
     ("longL", dict(B=1, T=64, Hq=4, Hkv=1, d=128, L=130)),
+    # the gradient pass over staged (P, <dO, vd>) pairs at its shared-memory limit (tokens
+    # per CTA x L x 4 heads x 8 bytes = 32 KB) and just past it (the recomputing pass)
+    ("stage-limit-d128", dict(B=1, T=40, Hq=8, Hkv=2, d=128, L=128)),
+    ("stage-limit-d64", dict(B=1, T=50, Hq=4, Hkv=1, d=64, L=64)),
+    ("stage-over-d64", dict(B=1, T=50, Hq=4, Hkv=1, d=64, L=65)),
 ]
 
 
